@@ -1,0 +1,297 @@
+"""Pins for the CPU oracle: it is checked here against things other than
+itself -- values worked out by hand from the page's definitions
+(tests/golden/hand_worked.json), closed forms, identities and invariants --
+so that a dropped term, a wrong sign, an off-by-one in the cumulative sum or a
+transposed operand in it fails at least one test.
+
+Sources: 2Mamba2Furious (thelatestinai.com summary page), Algorithms 1-6.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from mamba_ssd_sequence_b200 import inputs
+
+
+def _case_arrays(case, q, k, v):
+    B, H, N, d = case["B"], case["H"], case["N"], case["d"]
+    q = np.asarray(q, dtype=np.float32).reshape(B, H, N, d)
+    k = np.asarray(k, dtype=np.float32).reshape(B, H, N, d)
+    v = np.asarray(v, dtype=np.float32).reshape(B, H, N, d)
+    dt_p = np.asarray(case["dt_p"], dtype=np.float32).reshape(B, H, N)
+    A_log = np.asarray(case["A_log"], dtype=np.float32)
+    dt_bias = np.asarray(case["dt_bias"], dtype=np.float32)
+    return q, k, v, dt_p, A_log, dt_bias
+
+
+@pytest.fixture(scope="module")
+def golden(golden_dir):
+    with open(os.path.join(golden_dir, "hand_worked.json")) as f:
+        return {c["name"]: c for c in json.load(f)["cases"]}
+
+
+# ---------------------------------------------------------------- hand-worked
+def test_hand_constant_decay(golden):
+    """Algorithms 1/3/4/5 on a 3-token, d=2 case worked out by hand."""
+    c = golden["constant-half-decay"]
+    q, k, v, dt_p, A_log, dt_bias = _case_arrays(c, c["q"], c["k"], c["v"])
+    acs = oracle.log_decay(dt_p, A_log, dt_bias)[0, 0]
+    np.testing.assert_allclose(acs, c["acs"], rtol=1e-15)
+    Dres = np.asarray(c["D"], dtype=np.float32)
+    for e in c["expect"]:
+        D = Dres if e["residual"] else None
+        for form in (oracle.ssd_quadratic, oracle.ssd_recurrent):
+            y, n = form(q, k, v, dt_p, A_log, dt_bias, D, e["order"], e["normalize"],
+                        return_norm=True)
+            np.testing.assert_allclose(y[0, 0], e["y"], rtol=1e-14, atol=1e-14,
+                                       err_msg=f"{form.__name__} {e}")
+            if "norm" in e:
+                np.testing.assert_allclose(n[0, 0], e["norm"], rtol=1e-14, atol=1e-14)
+
+
+def test_hand_varying_decay_inclusive_cumsum(golden):
+    """The inclusive cumulative sum (decay-then-add, Algorithm 6) on a case
+    where an exclusive sum would give different numbers."""
+    c = golden["varying-decay-inclusive-cumsum"]
+    for var in c["variants"]:
+        q, k, v, dt_p, A_log, dt_bias = _case_arrays(c, var["q"], var["k"], var["v"])
+        acs = oracle.log_decay(dt_p, A_log, dt_bias)[0, 0]
+        # dt_p = ln 3 is stored as float32, so the decay is ln 4 to ~1e-7.
+        np.testing.assert_allclose(acs, c["acs"], rtol=1e-7)
+        for form in (oracle.ssd_quadratic, oracle.ssd_recurrent):
+            y, n = form(q, k, v, dt_p, A_log, dt_bias, None, var["order"], var["normalize"],
+                        return_norm=True)
+            np.testing.assert_allclose(y[0, 0], var["y"], rtol=2e-7, err_msg=form.__name__)
+            if "norm" in var:
+                np.testing.assert_allclose(n[0, 0], var["norm"], rtol=2e-7)
+
+
+# ------------------------------------------------------------ scalar helpers
+def test_softplus_closed_forms():
+    assert oracle.softplus(0.0) == pytest.approx(math.log(2.0), rel=1e-16)
+    assert oracle.softplus(math.log(3.0)) == pytest.approx(math.log(4.0), rel=1e-15)
+    assert oracle.softplus(50.0) == pytest.approx(50.0, rel=1e-16)
+    assert oracle.softplus(-50.0) == pytest.approx(math.exp(-50.0), rel=1e-12)
+    # softplus(x) - softplus(-x) = x for every x
+    for x in (-7.3, -0.1, 0.4, 3.9, 25.0):
+        assert oracle.softplus(x) - oracle.softplus(-x) == pytest.approx(x, rel=1e-13, abs=1e-15)
+
+
+def test_dt_bias_is_softplus_inverse():
+    """Algorithm 2: dt_bias = softplus^-1(dt_init), dt_init in [1e-3, 1e-1]."""
+    x = inputs.make_inputs(1, 64, 4, 4, "f32", seed=3)
+    dt0 = np.array([oracle.softplus(float(b)) for b in x["dt_bias"]])
+    assert np.all(dt0 >= inputs.DT_MIN * (1 - 1e-5))
+    assert np.all(dt0 <= inputs.DT_MAX * (1 + 1e-5))
+    assert np.all((x["A_log"] >= 0) & (x["A_log"] <= math.log(16.0) + 1e-6))
+
+
+def test_feature_tensor_square_identity():
+    """(q . k)^2 = (q (x) q) . (k (x) k)  (Algorithm 5 vs Algorithm 6)."""
+    rng = np.random.default_rng(5)
+    for d in (1, 3, 16):
+        q = rng.standard_normal(d)
+        k = rng.standard_normal(d)
+        fq, fk = oracle.feature(q, 2), oracle.feature(k, 2)
+        assert fq.shape == (d * d,)
+        assert np.dot(fq, fk) == pytest.approx(np.dot(q, k) ** 2, rel=1e-12)
+        assert np.array_equal(oracle.feature(q, 1), q)
+        # entry (a, b) at a*d + b
+        assert fq[(d - 1) * d + 0] == pytest.approx(q[d - 1] * q[0])
+
+
+def test_mask_properties():
+    """Algorithm 4: M_ii = 1, 0 < M_ij <= 1 below the diagonal (A < 0, dt > 0),
+    zero above it."""
+    x = inputs.make_inputs(1, 3, 48, 4, "f32", seed=1)
+    acs = oracle.log_decay(x["dt_p"], x["A_log"], x["dt_bias"])
+    for h in range(3):
+        row = acs[0, h]
+        assert np.all(np.diff(row) < 0)  # strictly decreasing: every a_t < 0
+        for i in range(48):
+            assert oracle.mask(row, i, i) == 1.0
+            for j in range(48):
+                m = oracle.mask(row, i, j)
+                if j > i:
+                    assert m == 0.0
+                elif j < i:
+                    assert 0.0 < m <= 1.0
+
+
+# --------------------------------------------------------- brute force forms
+def _brute(q, k, v, dt_p, A_log, dt_bias, D, order, normalize):
+    """Matrix form with explicit N x N A^M and M and explicit tensor-square
+    features (Algorithm 4 / 5 as printed), in numpy float64."""
+    B, H, N, d = q.shape
+    y = np.zeros((B, H, N, d))
+    for b in range(B):
+        for h in range(H):
+            A = -np.exp(np.float64(A_log[h]))
+            z = dt_p[b, h].astype(np.float64) + np.float64(dt_bias[h])
+            dt = np.log1p(np.exp(z))
+            acs = np.cumsum(A * dt)
+            AM = np.exp(acs[:, None] - acs[None, :])
+            M = np.tril(np.ones((N, N)))
+            Q = q[b, h].astype(np.float64)
+            K = k[b, h].astype(np.float64)
+            if order == 2:
+                Q = np.stack([np.kron(r, r) for r in Q])
+                K = np.stack([np.kron(r, r) for r in K])
+            W = (Q @ K.T) * np.where(M > 0, AM, 0.0)
+            yy = W @ v[b, h].astype(np.float64)
+            if normalize:
+                yy = yy / W.sum(axis=1, keepdims=True)
+            if D is not None:
+                yy = yy + D[h * d:(h + 1) * d][None, :].astype(np.float64) * v[b, h]
+            y[b, h] = yy
+    return y
+
+
+@pytest.mark.parametrize("order", [1, 2])
+@pytest.mark.parametrize("normalize", [False, True])
+@pytest.mark.parametrize("residual", [False, True])
+def test_quadratic_recurrent_brute_agree(order, normalize, residual):
+    """Three independent evaluations: loops over i >= j (Algorithm 5), the
+    token recurrence (Algorithm 6) and the explicit matrix form."""
+    x = inputs.make_inputs(2, 3, 37, 5, "f32", seed=11, residual=residual)
+    q, k = x["q"], x["k"]
+    if order == 1 and normalize:
+        # Order-1 row sums can pass through zero with SiLU features; positive
+        # scores keep the normalised case well conditioned.
+        q, k = np.abs(q), np.abs(k)
+    args = (q, k, x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"], order, normalize)
+    yq = oracle.ssd_quadratic(*args)
+    yr = oracle.ssd_recurrent(*args)
+    yb = _brute(*args)
+    scale = np.max(np.abs(yb))
+    assert np.max(np.abs(yq - yb)) <= 1e-12 * scale
+    assert np.max(np.abs(yr - yb)) <= 1e-12 * scale
+
+
+def test_sampled_rows_match_full():
+    x = inputs.make_inputs(1, 2, 70, 4, "bf16", seed=2)
+    args = (x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"], 2, True)
+    full = oracle.ssd_quadratic(*args)
+    rows = [0, 1, 33, 69, 5]
+    part = oracle.ssd_quadratic(*args, rows=rows)
+    np.testing.assert_array_equal(part, full[:, :, rows, :])
+
+
+# ------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("order", [1, 2])
+def test_no_decay_is_prefix_sum_linear_attention(order):
+    """A_log -> -inf makes A = 0 and every A^M_ij = 1: plain causal linear
+    attention (Algorithm 1 with M only), y_i = phi(q_i)^T sum_{j<=i} phi(k_j) v_j^T."""
+    x = inputs.make_inputs(1, 2, 29, 3, "f32", seed=7, residual=False)
+    A_log = np.full(2, -1000.0, dtype=np.float32)
+    y = oracle.ssd_quadratic(x["q"], x["k"], x["v"], x["dt_p"], A_log, x["dt_bias"], None,
+                             order, False)
+    for h in range(2):
+        Q = x["q"][0, h].astype(np.float64)
+        K = x["k"][0, h].astype(np.float64)
+        V = x["v"][0, h].astype(np.float64)
+        if order == 2:
+            Q = np.einsum("ta,tb->tab", Q, Q).reshape(29, -1)
+            K = np.einsum("ta,tb->tab", K, K).reshape(29, -1)
+        S = np.cumsum(np.einsum("tm,tc->tmc", K, V), axis=0)
+        ref = np.einsum("tm,tmc->tc", Q, S)
+        np.testing.assert_allclose(y[0, h], ref, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("order", [1, 2])
+def test_instant_decay_gives_diagonal(order):
+    """A_log huge: every off-diagonal A^M_ij underflows to 0 and only the
+    diagonal survives, y_i = (q_i . k_i)^order v_i; normalised, y_i = v_i."""
+    x = inputs.make_inputs(1, 2, 17, 4, "f32", seed=8, residual=False)
+    A_log = np.full(2, 80.0, dtype=np.float32)
+    args = (x["q"], x["k"], x["v"], x["dt_p"], A_log, x["dt_bias"], None, order)
+    y = oracle.ssd_quadratic(*args, False)
+    s = np.einsum("bhtc,bhtc->bht", x["q"].astype(np.float64), x["k"].astype(np.float64))
+    ref = (s ** order)[..., None] * x["v"]
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
+    yn = oracle.ssd_quadratic(*args, True)
+    np.testing.assert_allclose(yn, x["v"], rtol=1e-12)
+
+
+def test_constant_values_normalised_return_the_constant():
+    """With the normaliser, the output is a convex-like average of the v_j
+    (order 2 weights are >= 0): constant v gives back that constant."""
+    x = inputs.make_inputs(2, 2, 40, 6, "f32", seed=9, residual=False)
+    v = np.full_like(x["v"], 0.375)
+    y = oracle.ssd_quadratic(x["q"], x["k"], v, x["dt_p"], x["A_log"], x["dt_bias"], None, 2, True)
+    np.testing.assert_allclose(y, 0.375, rtol=1e-12)
+
+
+def test_zero_queries_leave_only_the_residual():
+    x = inputs.make_inputs(1, 2, 12, 4, "f32", seed=4)
+    D = np.arange(8, dtype=np.float32) * 0.25 - 1.0
+    q = np.zeros_like(x["q"])
+    for order in (1, 2):
+        y = oracle.ssd_quadratic(q, x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], D,
+                                 order, False)
+        ref = x["v"].astype(np.float64) * D.reshape(2, 4).astype(np.float64)[None, :, None, :]
+        np.testing.assert_array_equal(y, ref)
+
+
+def test_single_token():
+    x = inputs.make_inputs(1, 1, 1, 5, "f32", seed=6, residual=False)
+    s = float(np.dot(x["q"][0, 0, 0].astype(np.float64), x["k"][0, 0, 0].astype(np.float64)))
+    for order in (1, 2):
+        y = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"],
+                                 None, order, False)
+        np.testing.assert_allclose(y[0, 0, 0], s ** order * x["v"][0, 0, 0].astype(np.float64),
+                                   rtol=1e-13)
+
+
+# ---------------------------------------------------------------- invariants
+def test_linear_in_v_and_homogeneous_in_q():
+    x = inputs.make_inputs(1, 2, 25, 4, "f32", seed=12, residual=False)
+    base = (x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], None)
+    for order in (1, 2):
+        y = oracle.ssd_quadratic(x["q"], *base, order, False)
+        ya = oracle.ssd_quadratic(np.float32(2.0) * x["q"], *base, order, False)
+        np.testing.assert_allclose(ya, (2.0 ** order) * y, rtol=1e-12, atol=1e-13)
+        v2 = x["v"] * np.float32(-2.0)  # exact in float32
+        yv = oracle.ssd_quadratic(x["q"], x["k"], v2, x["dt_p"], x["A_log"], x["dt_bias"], None,
+                                  order, False)
+        np.testing.assert_allclose(yv, -2.0 * y, rtol=1e-12, atol=1e-13)
+    yn = oracle.ssd_quadratic(x["q"], *base, 2, True)
+    yna = oracle.ssd_quadratic(np.float32(4.0) * x["q"], *base, 2, True)
+    np.testing.assert_allclose(yna, yn, rtol=1e-12)
+
+
+def test_head_and_batch_permutation_equivariance():
+    x = inputs.make_inputs(2, 3, 20, 4, "f32", seed=13)
+    D = np.arange(12, dtype=np.float32) * 0.1
+    args = lambda q, k, v, dt, al, db, DD: (q, k, v, dt, al, db, DD, 2, True)
+    y = oracle.ssd_quadratic(*args(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"],
+                                   x["dt_bias"], D))
+    hp = [2, 0, 1]
+    bp = [1, 0]
+    Dp = D.reshape(3, 4)[hp].reshape(-1)
+    yp = oracle.ssd_quadratic(*args(x["q"][bp][:, hp], x["k"][bp][:, hp], x["v"][bp][:, hp],
+                                    x["dt_p"][bp][:, hp], x["A_log"][hp], x["dt_bias"][hp], Dp))
+    np.testing.assert_allclose(yp, y[bp][:, hp], rtol=1e-13)
+
+
+def test_recurrent_final_state_matches_definition():
+    """The final H_up from Algorithm 6 equals sum_j exp(A^CS_N-1 - A^CS_j) phi(k_j) v_j^T."""
+    x = inputs.make_inputs(1, 1, 15, 3, "f32", seed=14)
+    for order in (1, 2):
+        _, _, st, zst = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"],
+                                             x["dt_bias"], None, order, False, return_norm=True,
+                                             return_state=True)
+        acs = oracle.log_decay(x["dt_p"], x["A_log"], x["dt_bias"])[0, 0]
+        ref = np.zeros_like(st[0, 0])
+        zref = np.zeros_like(zst[0, 0])
+        for j in range(15):
+            fk = oracle.feature(x["k"][0, 0, j], order)
+            w = math.exp(acs[-1] - acs[j])
+            ref += w * np.outer(fk, x["v"][0, 0, j])
+            zref += w * fk
+        np.testing.assert_allclose(st[0, 0], ref, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(zst[0, 0], zref, rtol=1e-12, atol=1e-14)
