@@ -1,0 +1,378 @@
+"""Benchmark of the SSD forward operator on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step is one ssd_fwd() call -- the whole hot path (decay, intra-chunk
+quadratic form, carried state, normaliser / residual epilogue) -- over one
+batch of seeded synthetic input of the workload's shape, with the inputs
+resident in HBM.  The L2 is flushed (a 256 MiB write) before every step and
+each step is timed by its own CUDA-event pair on the launching stream, so the
+flush is outside the timed kernels.  With N > 1 (torchrun) every rank runs an
+independent replica of the workload on its own GPU (the operator has no
+cross-GPU step); the time is the max over ranks and `value` counts the tokens
+of all ranks ("weak" scaling).
+
+Rank 0 prints one JSON line.  `--impl reference` times the CPU oracle (the
+only other implementation of the method) on the host cores instead, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mamba_ssd_sequence_b200 import inputs  # noqa: E402
+
+METRIC = "SSD fwd tokens/s and TFLOP/s (frac. of bf16 TC peak) at H=16,d_h=64,N=2K–64K"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_work(w: inputs.Workload):
+    """Per-launch algorithmic bytes and FLOPs of one call.
+
+    bytes per token-head: q, k, v and out (d_h elements each) plus dt_p (fp32);
+    the carried state never leaves the chip and is not counted.
+    FLOPs per token-head: the causal half of the intra-chunk score and value
+    products 2(C+1)d, the state build and state readout 4*D_phi*d, and the
+    normaliser 4*D_phi + C + 1 when it is on."""
+    e = 2 if w.dtype == "bf16" else 4
+    d, C = w.d, w.chunk
+    dphi = d if w.order == 1 else d * d
+    per_tok_bytes = 4 * d * e + 4
+    per_tok_flops = 2 * (C + 1) * d + 4 * dphi * d + ((4 * dphi + C + 1) if w.normalize else 0)
+    T = w.token_heads
+    return T * per_tok_bytes, T * per_tok_flops, per_tok_bytes, per_tok_flops
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ssd_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(parts)
+                except ValueError:
+                    pass
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def make_device_inputs(w, seed, torch):
+    x = inputs.make_workload_inputs(w, seed=seed)
+    dev = {}
+    for name in ("q", "k", "v"):
+        if w.dtype == "bf16":
+            t = torch.from_numpy(x[name + "_bits"].view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(x[name])
+        dev[name] = t
+    for name in ("dt_p", "A_log", "dt_bias"):
+        dev[name] = torch.from_numpy(x[name])
+    dev["D"] = None if x["D"] is None else torch.from_numpy(x["D"])
+    return x, dev
+
+
+def _oracle_sample(w, x, heads):
+    """Arguments of the oracle for the first `heads` (b, h) rows of the
+    workload (batch-major), every token."""
+    bsel = (heads + w.H - 1) // w.H
+    q = x["q"][:bsel].reshape(-1, w.N, w.d)[:heads][None]
+    k = x["k"][:bsel].reshape(-1, w.N, w.d)[:heads][None]
+    v = x["v"][:bsel].reshape(-1, w.N, w.d)[:heads][None]
+    dt = x["dt_p"][:bsel].reshape(-1, w.N)[:heads][None]
+    hidx = np.arange(heads) % w.H
+    D = None if x["D"] is None else x["D"].reshape(w.H, w.d)[hidx].reshape(-1)
+    return q, k, v, dt, x["A_log"][hidx], x["dt_bias"][hidx], D
+
+
+def _time_oracle(w, x, budget_s):
+    """Times the oracle's quadratic form on a sample of (b, h) rows sized to
+    take about `budget_s` seconds; returns (tokens/s, threads, description)."""
+    import oracle
+    bh_all = w.B * w.H
+    t0 = time.perf_counter()
+    oracle.ssd_quadratic(*_oracle_sample(w, x, 1), w.order, w.normalize)
+    t1 = max(time.perf_counter() - t0, 1e-6)
+    heads = max(1, min(bh_all, int(budget_s / t1)))
+    reps = 1
+    if heads == bh_all:
+        reps = max(1, int(budget_s / (t1 * bh_all)))
+    args = _oracle_sample(w, x, heads)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.ssd_quadratic(*args, w.order, w.normalize)
+    t = time.perf_counter() - t0
+    tokens = reps * w.N * heads / w.H  # equivalent full (all-heads) tokens
+    desc = (f"quadratic form (float64, OpenMP) over {heads} of the {bh_all} (b, h) rows, "
+            f"all {w.N} tokens, {reps} pass(es): {t:.2f} s")
+    return tokens / t, oracle.num_threads(), desc
+
+
+def cpu_baseline(w, x, budget_s=12.0):
+    """The CPU oracle as it stands, timed on the host cores on a bounded
+    sample of the same workload (the JSON object of the bench line)."""
+    value, threads, desc = _time_oracle(w, x, budget_s)
+    return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": desc}
+
+
+def run_reference(args, w):
+    """The reference arm: the CPU oracle, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    x = inputs.make_workload_inputs(w, seed=0)
+    per_step = min(10.0, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _time_oracle(w, x, per_step / 4)
+    vals, descs = [], []
+    for _ in range(args.steps):
+        v_, threads, d_ = _time_oracle(w, x, per_step)
+        vals.append(v_)
+        descs.append(d_)
+    value = len(vals) / sum(1.0 / v_ for v_ in vals)
+    times = [w.tokens / v_ for v_ in vals]
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d_h": w.d,
+                       "chunk": w.chunk, "order": w.order, "normalize": w.normalize,
+                       "residual": w.residual},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads,
+                             "kind": "oracle",
+                             "sample": "each step: " + descs[-1]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=inputs.HEADLINE, choices=inputs.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import mamba_ssd_sequence_b200 as ssd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev_name = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(dev_name))
+
+    x, host = make_device_inputs(w, seed=rank, torch=torch)
+    dev = {k: (v.to(dev_name) if v is not None else None) for k, v in host.items()}
+    out = torch.empty_like(dev["q"])
+    dcode = ssd.SSD_BF16 if w.dtype == "bf16" else ssd.SSD_F32
+    ws = ssd.alloc_workspace(w.B, w.H, w.N, w.d, dcode, w.order, w.chunk, dev_name)
+    path, n_launch = ssd.ssd_fwd_path(w.B, w.H, w.N, w.d, dcode, w.order, w.chunk)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev_name)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssd.ssd_fwd(dev["q"], dev["k"], dev["v"], dev["dt_p"], dev["A_log"], dev["dt_bias"],
+                    dev["D"], w.order, w.normalize, w.chunk, out=out, workspace=ws,
+                    stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if ssd.ssd_status_from_workspace(ws) != 0:
+        raise RuntimeError("device status not clean after warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        # keep the sampler alive for at least a few samples on short runs
+        time.sleep(0.5)
+    if world > 1:
+        dist.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev_name)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    status = ssd.ssd_status_from_workspace(ws)
+
+    # end to end: pinned host inputs -> device -> ssd_fwd -> host, per step
+    e2e = None
+    if not args.no_e2e:
+        host_p = {k: (v.pin_memory() if v is not None else None) for k, v in host.items()}
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        scratch = dict(dev)
+        scratch["out"] = out
+        h2d = sum(v.numel() * v.element_size() for v in host_p.values() if v is not None)
+        d2h = out_h.numel() * out_h.element_size()
+
+        def e2e_step():
+            ssd.ssd_fwd_host(host_p["q"], host_p["k"], host_p["v"], host_p["dt_p"],
+                             host_p["A_log"], host_p["dt_bias"], host_p["D"], w.order,
+                             w.normalize, w.chunk, out_h, scratch, ws, stream=stream)
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev_name)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item())
+        e2e = {"value": world * w.tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    alg_bytes, alg_flops, bpt, fpt = algorithmic_work(w)
+    mean_ms = total_ms / args.steps
+    peaks, peak_src = load_peaks()
+    tflops = alg_flops / (mean_ms / 1e3) / 1e12
+    gbs = alg_bytes / (mean_ms / 1e3) / 1e9
+    if w.order == 1:
+        bound, achieved, peak, unit = "hbm", gbs, float(peaks["hbm_gbs"]), "GB/s"
+    else:
+        bound, achieved, peak, unit = "tensor", tflops, float(peaks["bf16_tflops"]), "TFLOP/s"
+    line = {
+        "metric": METRIC,
+        "value": world * w.tokens * args.steps / (total_ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": mean_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d_h": w.d,
+                   "chunk": w.chunk, "order": w.order, "normalize": w.normalize,
+                   "residual": w.residual, "parallelism": f"replicas{world}",
+                   "l2": "flushed before every step (256 MiB write); each step timed by its "
+                         "own CUDA-event pair", "path": path},
+        "tflops": tflops,
+        "tc_frac": tflops / float(peaks["bf16_tflops"]),
+        "hbm_gbs": gbs,
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+                     "algorithmic_bytes_per_launch": alg_bytes,
+                     "algorithmic_flops_per_launch": alg_flops},
+        "gpu_launches": n_launch * args.steps,
+        "device_status": status,
+        "clocks": clk.summary(),
+    }
+    if e2e is not None:
+        line["e2e"] = e2e
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, x)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

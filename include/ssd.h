@@ -1,0 +1,163 @@
+/*
+ * ssd.h -- C ABI of libssd.so, the B200 (sm_100a) implementation of the
+ * forward pass of the causal, decay-masked linear-attention ("SSD") operator
+ * of Mamba-2 / Mamba-2S / 2Mamba.
+ *
+ * The operator (2Mamba2Furious, Mongaras & Larson 2026; Algorithm 1 "Linear
+ * attention", Algorithm 3 "Mamba-2 Forward Pass", Algorithm 4 "Mamba-2S",
+ * Algorithm 5 "2Mamba"), per batch b and head h, for rows i and columns j of
+ * one sequence of N tokens:
+ *
+ *     A_h    = -exp(A_log[h])                              (Algorithm 3)
+ *     dt_t   = softplus(dt_p[b,h,t] + dt_bias[h])          (Algorithm 3)
+ *     A^CS_t = sum_{tau <= t} A_h dt_tau   (inclusive)     (Algorithm 3)
+ *     w_ij   = (q_i . k_j)^order * exp(A^CS_i - A^CS_j) * [i >= j]
+ *                                                   (Algorithms 1, 4 and 5)
+ *     y_i    = sum_j w_ij v_j                              (Algorithm 1 / 5)
+ *     y_i   /= sum_j w_ij            when normalize != 0   (Algorithm 1 / 5)
+ *     y_ic  += D[h*d_h + c] v_ic     when D != NULL        (Algorithm 3, D_res)
+ *
+ * order 1 is plain linear attention with the Mamba-2 decay mask; order 2 is
+ * 2Mamba's squared score, whose recurrent form (Algorithm 6 "2Mamba
+ * Inference") carries a d_h^2 x d_h state.  The library evaluates it in
+ * chunks of `chunk` tokens: a quadratic form inside each chunk plus a state
+ * carried across chunks.  The result does not depend on `chunk` except
+ * through rounding.
+ *
+ * Conventions for every entry point:
+ *  - Layouts are row-major and contiguous: q, k, v, out are [B, H, N, d_h];
+ *    dt_p is [B, H, N]; A_log and dt_bias are [H]; D is [H*d_h].
+ *  - Pointers marked "device" must point to device memory of the current
+ *    CUDA device, 16-byte aligned.  The caller owns every buffer; the library
+ *    allocates no memory and keeps no state between calls, so calls on
+ *    different streams with different buffers are independent.
+ *  - Work is enqueued asynchronously on `stream` (a cudaStream_t passed as
+ *    void*, NULL = the legacy default stream).  The return value reports
+ *    argument validation and launch errors only; errors detected on the
+ *    device are read back with ssd_status_from_workspace().
+ *  - Arithmetic is fp32 for the decay, the scores' products and all
+ *    accumulation; bf16 inputs feed the tensor cores as bf16 (the score
+ *    matrix P and the carried state are rounded to bf16 as MMA operands) and
+ *    the output is rounded to the input dtype with round-to-nearest-even.
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every entry point. */
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_NULL = 1,        /* a required pointer is NULL */
+    SSD_ERR_SHAPE = 2,       /* B, H, N or d_h out of range, or N % chunk != 0 */
+    SSD_ERR_DTYPE = 3,       /* dtype is not SSD_F32 or SSD_BF16 */
+    SSD_ERR_ORDER = 4,       /* order is not 1 or 2 */
+    SSD_ERR_CHUNK = 5,       /* chunk is not 64, 128 or 256 */
+    SSD_ERR_ALIGN = 6,       /* a device pointer is not 16-byte aligned */
+    SSD_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssd_workspace_bytes() */
+    SSD_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed */
+    SSD_ERR_TIMEOUT = 9,     /* a device-side wait ran out (read back from the workspace) */
+    SSD_ERR_UNSUPPORTED = 10 /* a valid combination this build has no kernel for */
+} ssd_status;
+
+/* Element type of q, k, v and out. */
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/*
+ * Bytes of device workspace ssd_fwd() needs for this problem.  Depends only
+ * on the arguments.  Returns 0 when the arguments are invalid (ssd_fwd
+ * would reject them).  Supported: B, H >= 1; N >= 1 with N % chunk == 0;
+ * d_h in {16, 32, 64}; order in {1, 2}; chunk in {64, 128, 256}.
+ */
+size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk);
+
+/*
+ * Forward pass of the operator above.
+ *   q, k, v    device, [B, H, N, d_h], element type `dtype`
+ *   dt_p       device, [B, H, N] fp32 (the per-token dt projection, Algorithm 3)
+ *   A_log      device, [H] fp32
+ *   dt_bias    device, [H] fp32
+ *   D          device, [H*d_h] fp32, or NULL for no residual
+ *   normalize  nonzero: divide each row by its row sum (Algorithm 1, y / N)
+ *   chunk      chunk length in tokens (64, 128 or 256), N % chunk == 0
+ *   out        device, [B, H, N, d_h], element type `dtype`; must not alias
+ *              an input
+ *   workspace  device, at least ssd_workspace_bytes(...) bytes, 256-byte
+ *              aligned; its contents on entry do not matter.  The first 16
+ *              bytes receive the device status read by
+ *              ssd_status_from_workspace().
+ * Returns SSD_OK or an error code; on error nothing is enqueued.
+ */
+int ssd_fwd(const void *q, const void *k, const void *v,
+            const float *dt_p, const float *A_log, const float *dt_bias,
+            const float *D,
+            int B, int H, int N, int d_h, int dtype,
+            int order, int normalize, int chunk,
+            void *out, void *workspace, size_t workspace_bytes,
+            void *stream);
+
+/*
+ * ssd_fwd() with the activations in HOST memory: enqueues on `stream` the
+ * host-to-device copies of q, k, v, dt_p, A_log, dt_bias and D (when
+ * non-NULL) into the caller's device buffers, the forward pass, and the
+ * device-to-host copy of the result into out_host.  Host buffers should be
+ * pinned (cudaHostAlloc / torch pin_memory) for the copies to be
+ * asynchronous.  The d_* buffers are device buffers of the shapes listed for
+ * ssd_fwd(); d_D may be NULL only when D_host is NULL.  The call returns once
+ * the work is enqueued; synchronise `stream` before reading out_host.
+ */
+int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                 const float *dt_p_host, const float *A_log_host,
+                 const float *dt_bias_host, const float *D_host,
+                 int B, int H, int N, int d_h, int dtype,
+                 int order, int normalize, int chunk,
+                 void *out_host,
+                 void *d_q, void *d_k, void *d_v, float *d_dt_p,
+                 float *d_A_log, float *d_dt_bias, float *d_D, void *d_out,
+                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Chunked decay (Algorithm 3, last line, evaluated per chunk):
+ *   acs[b,h,t]       = sum over tau in t's chunk, tau <= t, of A_h dt_tau
+ *                      (the chunk-local inclusive cumulative sum, fp32)
+ *   chunk_sum[b,h,c] = the same sum over the whole chunk c (= acs at the
+ *                      chunk's last token)
+ * A^CS_i - A^CS_j for i, j in one chunk equals acs[i] - acs[j]; across chunks
+ * the global value is recovered by adding the chunk_sum of the chunks in
+ * between.  dt_p, A_log, dt_bias, acs ([B,H,N]) and chunk_sum ([B,H,N/chunk])
+ * are device pointers.  chunk in {64, 128, 256}; N % chunk == 0.
+ */
+int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias,
+                     int B, int H, int N, int chunk,
+                     float *acs, float *chunk_sum, void *stream);
+
+/*
+ * Synchronises `stream`, then reads the device status that the kernels of
+ * the last ssd_fwd() on this workspace wrote (SSD_OK or SSD_ERR_TIMEOUT when
+ * a bounded inter-block wait gave up; the output is then incomplete).
+ * Returns SSD_ERR_CUDA if the synchronisation itself fails.
+ */
+int ssd_status_from_workspace(const void *workspace, void *stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *ssd_status_str(int status);
+
+/*
+ * Which kernel sequence ssd_fwd() runs for these arguments: 0 = the general
+ * SIMT path (any supported shape, fp32 or bf16), 1 = the order-1 tcgen05
+ * path, 2 = the order-2 tcgen05 path; -1 when the arguments are invalid.
+ * *n_launches (may be NULL) receives the number of kernels one call launches.
+ */
+int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
+                 int *n_launches);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H */

@@ -1,2 +1,181 @@
 """B200 (sm_100a) implementation of the decay-masked linear-attention (SSD)
-forward operator of Mamba-2 / Mamba-2S / 2Mamba."""
+forward operator of Mamba-2 / Mamba-2S / 2Mamba.
+
+This module is a thin ctypes binding over libssd.so (C ABI in
+include/ssd.h).  It only marshals arguments: every step of the operator runs
+in the library's CUDA kernels.  Tensors are torch tensors; device tensors must
+be contiguous and live on the current CUDA device.  If libssd.so has not been
+built, every call raises -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+SSD_F32 = 0
+SSD_BF16 = 1
+PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2"}
+
+_lib = None
+
+
+class SSDError(RuntimeError):
+    """A libssd.so entry point returned a non-zero ssd_status."""
+
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_str(code)} (code {code})")
+
+
+def load_library():
+    """Load libssd.so (ctypes) and declare the C signatures.  Raises if the
+    library has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with `python -m mamba_ssd_sequence_b200.build` "
+            "(there is no CPU or Python fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, sz, ci = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    lib.ssd_workspace_bytes.argtypes = [ci] * 7
+    lib.ssd_workspace_bytes.restype = sz
+    lib.ssd_fwd.argtypes = [vp] * 7 + [ci] * 8 + [vp, vp, sz, vp]
+    lib.ssd_fwd.restype = ci
+    lib.ssd_fwd_host.argtypes = [vp] * 7 + [ci] * 8 + [vp] + [vp] * 8 + [vp, sz, vp]
+    lib.ssd_fwd_host.restype = ci
+    lib.ssd_chunk_cumsum.argtypes = [vp] * 3 + [ci] * 4 + [vp, vp, vp]
+    lib.ssd_chunk_cumsum.restype = ci
+    lib.ssd_status_from_workspace.argtypes = [vp, vp]
+    lib.ssd_status_from_workspace.restype = ci
+    lib.ssd_status_str.argtypes = [ci]
+    lib.ssd_status_str.restype = ctypes.c_char_p
+    lib.ssd_fwd_path.argtypes = [ci] * 7 + [ctypes.POINTER(ci)]
+    lib.ssd_fwd_path.restype = ci
+    _lib = lib
+    return lib
+
+
+def status_str(code: int) -> str:
+    return load_library().ssd_status_str(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise SSDError(code, where)
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return SSD_F32
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libssd must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def ssd_workspace_bytes(B: int, H: int, N: int, d_h: int, dtype: int, order: int,
+                        chunk: int) -> int:
+    """Device workspace (bytes) ssd_fwd needs; 0 for invalid arguments."""
+    return int(load_library().ssd_workspace_bytes(B, H, N, d_h, dtype, order, chunk))
+
+
+def ssd_fwd_path(B: int, H: int, N: int, d_h: int, dtype: int, order: int, chunk: int):
+    """(path name, kernels launched per call) for these arguments."""
+    n = ctypes.c_int(0)
+    p = load_library().ssd_fwd_path(B, H, N, d_h, dtype, order, chunk, ctypes.byref(n))
+    if p < 0:
+        raise ValueError("invalid ssd arguments")
+    return PATH_NAMES[p], n.value
+
+
+def alloc_workspace(B, H, N, d_h, dtype, order, chunk, device=None):
+    """A torch uint8 device buffer of ssd_workspace_bytes() bytes."""
+    import torch
+    nbytes = ssd_workspace_bytes(B, H, N, d_h, dtype, order, chunk)
+    if nbytes == 0:
+        raise ValueError("invalid ssd arguments")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk: int,
+            out=None, workspace=None, stream=None):
+    """y = SSD forward (include/ssd.h, ssd_fwd) on CUDA tensors.
+
+    q, k, v: [B, H, N, d_h] float32 or bfloat16; dt_p: [B, H, N] float32;
+    A_log, dt_bias: [H] float32; D: [H*d_h] float32 or None.  Returns `out`
+    ([B, H, N, d_h], the input dtype), allocating it and the workspace with
+    torch when not given.  Asynchronous on `stream` (default: the current
+    torch stream)."""
+    import torch
+    B, H, N, d = q.shape
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device)
+    rc = load_library().ssd_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
+        B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk),
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "ssd_fwd")
+    return out
+
+
+def ssd_fwd_host(q_h, k_h, v_h, dt_p_h, A_log_h, dt_bias_h, D_h, order: int,
+                 normalize: bool, chunk: int, out_h, dev: dict, workspace, stream=None):
+    """ssd_fwd_host (include/ssd.h): host (pinned) tensors in and out, with the
+    caller's device buffers `dev` (keys q, k, v, dt_p, A_log, dt_bias, D, out)
+    receiving the copies.  Asynchronous on `stream`."""
+    B, H, N, d = q_h.shape
+    dt = _dtype_code(q_h)
+    rc = load_library().ssd_fwd_host(
+        _ptr(q_h), _ptr(k_h), _ptr(v_h), _ptr(dt_p_h), _ptr(A_log_h), _ptr(dt_bias_h),
+        _ptr(D_h), B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk), _ptr(out_h),
+        _ptr(dev["q"]), _ptr(dev["k"]), _ptr(dev["v"]), _ptr(dev["dt_p"]),
+        _ptr(dev["A_log"]), _ptr(dev["dt_bias"]), _ptr(dev.get("D")), _ptr(dev["out"]),
+        _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "ssd_fwd_host")
+    return out_h
+
+
+def ssd_chunk_cumsum(dt_p, A_log, dt_bias, chunk: int, acs=None, chunk_sum=None, stream=None):
+    """Kernel (a): chunk-local inclusive cumsum of A*dt and chunk totals
+    (include/ssd.h, ssd_chunk_cumsum).  Returns (acs [B,H,N], chunk_sum [B,H,N/chunk])."""
+    import torch
+    B, H, N = dt_p.shape
+    if acs is None:
+        acs = torch.empty_like(dt_p)
+    if chunk_sum is None:
+        chunk_sum = torch.empty((B, H, N // chunk), dtype=torch.float32, device=dt_p.device)
+    rc = load_library().ssd_chunk_cumsum(_ptr(dt_p), _ptr(A_log), _ptr(dt_bias), B, H, N,
+                                         int(chunk), _ptr(acs), _ptr(chunk_sum),
+                                         _stream_handle(stream))
+    _check(rc, "ssd_chunk_cumsum")
+    return acs, chunk_sum
+
+
+def ssd_status_from_workspace(workspace, stream=None) -> int:
+    """Synchronise and read the device status left in the workspace."""
+    return int(load_library().ssd_status_from_workspace(_ptr(workspace),
+                                                        _stream_handle(stream)))

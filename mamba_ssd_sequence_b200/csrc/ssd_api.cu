@@ -1,0 +1,168 @@
+// C entry points of libssd.so: argument validation, workspace planning and
+// dispatch to the kernel paths.  The operator and the conventions are
+// documented in include/ssd.h.
+#include <cuda_runtime.h>
+
+#include "ssd_internal.h"
+
+namespace ssd {
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int check_shape(int B, int H, int N, int d, int dtype, int order, int chunk) {
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_DTYPE;
+    if (order != 1 && order != 2) return SSD_ERR_ORDER;
+    if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_CHUNK;
+    if (B < 1 || H < 1 || N < 1) return SSD_ERR_SHAPE;
+    if (d != 16 && d != 32 && d != 64) return SSD_ERR_SHAPE;
+    if (N % chunk != 0) return SSD_ERR_SHAPE;
+    if ((long long)B * H > 65535) return SSD_ERR_SHAPE;
+    if ((long long)B * H * N * d >= (1ll << 40)) return SSD_ERR_SHAPE;
+    return SSD_OK;
+}
+
+bool make_plan(int B, int H, int N, int d, int dtype, int order, int chunk, Plan *plan) {
+    if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
+    const size_t BH = (size_t)B * H, nc = (size_t)N / chunk;
+    Plan p{};
+    if (order == 1 && tc_order1_supports(B, H, N, d, dtype, chunk)) {
+        p.path = PATH_TC_ORDER1;
+        p.n_launches = 1;
+        p.acs_off = p.lam_off = p.state_off = kStatusBytes;
+        p.total = kStatusBytes + tc_order1_workspace(B, H, N, d, chunk);
+    } else if (order == 2 && tc_order2_supports(B, H, N, d, dtype, chunk)) {
+        p.path = PATH_TC_ORDER2;
+        p.n_launches = 1;
+        p.acs_off = p.lam_off = p.state_off = kStatusBytes;
+        p.total = kStatusBytes + tc_order2_workspace(B, H, N, d, chunk);
+    } else {
+        const size_t Dphi = order == 1 ? (size_t)d : (size_t)d * d;
+        p.path = PATH_SIMT;
+        p.n_launches = 4;
+        p.acs_off = kStatusBytes;
+        p.lam_off = align_up(p.acs_off + BH * N * sizeof(float), 256);
+        p.state_off = align_up(p.lam_off + BH * nc * sizeof(float), 256);
+        p.total = align_up(p.state_off + BH * nc * Dphi * (d + 1) * sizeof(float), 256);
+    }
+    *plan = p;
+    return true;
+}
+
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk) {
+    Plan p;
+    if (!make_plan(B, H, N, d_h, dtype, order, chunk, &p)) return 0;
+    return p.total;
+}
+
+int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
+                 int *n_launches) {
+    Plan p;
+    if (!make_plan(B, H, N, d_h, dtype, order, chunk, &p)) return -1;
+    if (n_launches) *n_launches = p.n_launches;
+    return p.path;
+}
+
+int ssd_fwd(const void *q, const void *k, const void *v, const float *dt_p,
+            const float *A_log, const float *dt_bias, const float *D, int B, int H, int N,
+            int d_h, int dtype, int order, int normalize, int chunk, void *out,
+            void *workspace, size_t workspace_bytes, void *stream) {
+    if (!q || !k || !v || !dt_p || !A_log || !dt_bias || !out) return SSD_ERR_NULL;
+    int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    const void *ptrs[] = {q, k, v, dt_p, A_log, dt_bias, out};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    if (D && !aligned16(D)) return SSD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
+    Plan p;
+    if (!make_plan(B, H, N, d_h, dtype, order, chunk, &p)) return SSD_ERR_UNSUPPORTED;
+    if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
+    FwdArgs a{q, k, v, dt_p, A_log, dt_bias, D, B, H, N, d_h, dtype, order, normalize ? 1 : 0,
+              chunk, out, workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
+    switch (p.path) {
+    case PATH_TC_ORDER1: return launch_tc_order1(a, p);
+    case PATH_TC_ORDER2: return launch_tc_order2(a, p);
+    default: return launch_simt(a, p);
+    }
+}
+
+int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                 const float *dt_p_host, const float *A_log_host, const float *dt_bias_host,
+                 const float *D_host, int B, int H, int N, int d_h, int dtype, int order,
+                 int normalize, int chunk, void *out_host, void *d_q, void *d_k, void *d_v,
+                 float *d_dt_p, float *d_A_log, float *d_dt_bias, float *d_D, void *d_out,
+                 void *workspace, size_t workspace_bytes, void *stream) {
+    if (!q_host || !k_host || !v_host || !dt_p_host || !A_log_host || !dt_bias_host ||
+        !out_host)
+        return SSD_ERR_NULL;
+    if (D_host && !d_D) return SSD_ERR_NULL;
+    int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
+    if (rc != SSD_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t elem = dtype == SSD_F32 ? 4 : 2;
+    const size_t act = (size_t)B * H * N * d_h * elem;
+    const size_t tok = (size_t)B * H * N * sizeof(float);
+    const size_t hp = (size_t)H * sizeof(float);
+    struct Copy { void *dst; const void *src; size_t n; } h2d[] = {
+        {d_q, q_host, act}, {d_k, k_host, act}, {d_v, v_host, act}, {d_dt_p, dt_p_host, tok},
+        {d_A_log, A_log_host, hp}, {d_dt_bias, dt_bias_host, hp},
+        {d_D, D_host, (size_t)H * d_h * sizeof(float)}};
+    for (const Copy &c : h2d) {
+        if (!c.src) continue;
+        if (!c.dst) return SSD_ERR_NULL;
+        if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return SSD_ERR_CUDA;
+    }
+    rc = ssd_fwd(d_q, d_k, d_v, d_dt_p, d_A_log, d_dt_bias, D_host ? d_D : nullptr, B, H, N,
+                 d_h, dtype, order, normalize, chunk, d_out, workspace, workspace_bytes, stream);
+    if (rc != SSD_OK) return rc;
+    if (cudaMemcpyAsync(out_host, d_out, act, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return SSD_OK;
+}
+
+int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias, int B, int H,
+                     int N, int chunk, float *acs, float *chunk_sum, void *stream) {
+    if (!dt_p || !A_log || !dt_bias || !acs || !chunk_sum) return SSD_ERR_NULL;
+    if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_CHUNK;
+    if (B < 1 || H < 1 || N < 1 || N % chunk != 0 || (long long)B * H > 65535)
+        return SSD_ERR_SHAPE;
+    return launch_chunk_cumsum(dt_p, A_log, dt_bias, B, H, N, chunk, acs, chunk_sum, nullptr,
+                               static_cast<cudaStream_t>(stream));
+}
+
+int ssd_status_from_workspace(const void *workspace, void *stream) {
+    if (!workspace) return SSD_ERR_NULL;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SSD_ERR_CUDA;
+    DeviceStatus st;
+    if (cudaMemcpy(&st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return st.code;
+}
+
+const char *ssd_status_str(int status) {
+    switch (status) {
+    case SSD_OK: return "SSD_OK";
+    case SSD_ERR_NULL: return "SSD_ERR_NULL: a required pointer is NULL";
+    case SSD_ERR_SHAPE: return "SSD_ERR_SHAPE: B, H, N or d_h out of range, or N % chunk != 0";
+    case SSD_ERR_DTYPE: return "SSD_ERR_DTYPE: dtype must be SSD_F32 or SSD_BF16";
+    case SSD_ERR_ORDER: return "SSD_ERR_ORDER: order must be 1 or 2";
+    case SSD_ERR_CHUNK: return "SSD_ERR_CHUNK: chunk must be 64, 128 or 256";
+    case SSD_ERR_ALIGN: return "SSD_ERR_ALIGN: device pointer not 16-byte aligned (workspace: 256)";
+    case SSD_ERR_WORKSPACE: return "SSD_ERR_WORKSPACE: workspace missing or too small";
+    case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA runtime or launch error";
+    case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: no kernel for this combination";
+    default: return "unknown ssd status";
+    }
+}
+
+}  // extern "C"

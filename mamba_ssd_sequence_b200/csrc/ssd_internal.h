@@ -1,0 +1,63 @@
+// Internal declarations shared by the entry points and the kernel files of
+// libssd.so.  Nothing here is part of the public ABI (see include/ssd.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "ssd.h"
+
+namespace ssd {
+
+// Arguments of one forward call after validation.
+struct FwdArgs {
+    const void *q, *k, *v;
+    const float *dt_p, *A_log, *dt_bias, *D;
+    int B, H, N, d, dtype, order, normalize, chunk;
+    void *out;
+    void *workspace;
+    size_t workspace_bytes;
+    cudaStream_t stream;
+};
+
+// Device status block at the start of every workspace: status code (an
+// ssd_status value, 0 = fine) and a detail word (where a wait gave up).
+struct DeviceStatus {
+    int code;
+    int detail;
+    int pad[2];
+};
+
+constexpr size_t kStatusBytes = 256;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+enum Path { PATH_SIMT = 0, PATH_TC_ORDER1 = 1, PATH_TC_ORDER2 = 2 };
+
+// Workspace plan for one call: which path runs and where its buffers sit.
+struct Plan {
+    int path;
+    int n_launches;
+    size_t acs_off, lam_off, state_off, total;
+};
+
+// Fills `plan` for validated arguments; returns false if no kernel exists.
+bool make_plan(int B, int H, int N, int d, int dtype, int order, int chunk, Plan *plan);
+
+// Path launchers (each returns an ssd_status).
+int launch_simt(const FwdArgs &a, const Plan &p);
+int launch_tc_order1(const FwdArgs &a, const Plan &p);
+int launch_tc_order2(const FwdArgs &a, const Plan &p);
+bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);
+bool tc_order2_supports(int B, int H, int N, int d, int dtype, int chunk);
+size_t tc_order1_workspace(int B, int H, int N, int d, int chunk);
+size_t tc_order2_workspace(int B, int H, int N, int d, int chunk);
+
+// Kernel (a): chunk-local inclusive cumsum of A*dt and the chunk totals.
+// When `status` is non-NULL, block (0,0) thread 0 clears it.
+int launch_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias,
+                        int B, int H, int N, int chunk, float *acs, float *chunk_sum,
+                        DeviceStatus *status, cudaStream_t stream);
+
+}  // namespace ssd

@@ -1,0 +1,321 @@
+// General SIMT (CUDA-core, fp32 arithmetic) path of the SSD forward operator,
+// and kernel (a), the chunked decay.
+//
+// The path runs for every supported shape and is the one used for fp32
+// inputs, where the tolerance (1e-4 of max|y|) rules out bf16/tf32 tensor
+// cores.  It evaluates the chunked ("state passing") decomposition of
+// 2Mamba2Furious Algorithms 1/5 with the decay of Algorithm 3 in four
+// launches:
+//   (a) chunk_cumsum  : acs_t = chunk-local inclusive cumsum of A*dt,
+//                       lam_c = the chunk's total;
+//   (b) chunk_state   : U_c = sum_{j in c} exp(lam_c - acs_j) phi(k_j) [v_j, 1]^T,
+//                       the chunk's own contribution to the carried state
+//                       (the column of ones carries the normaliser state);
+//   (c) state_scan    : S_c = state entering chunk c,
+//                       S_0 = 0, S_{c+1} = exp(lam_c) S_c + U_c  (Algorithm 6
+//                       applied chunk by chunk);
+//   (d) chunk_output  : y_i = sum_{j in c, j<=i} (q_i.k_j)^p exp(acs_i-acs_j) v_j
+//                             + exp(acs_i) phi(q_i)^T S_c,
+//                       the same for the row sum, then /row sum, + D*v.
+// phi is the identity (order 1) or the tensor square (order 2), whose inner
+// product with phi(k) is (q.k)^2.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "ssd_internal.h"
+
+namespace ssd {
+namespace {
+
+__device__ __forceinline__ float load_elem(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float *p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// softplus(x) = log(1 + e^x) in the overflow-free form.
+__device__ __forceinline__ float softplus_f(float x) {
+    return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
+}
+
+// ---------------------------------------------------------------- kernel (a)
+// grid (n_chunks, B*H), block = chunk threads (64, 128 or 256).
+__global__ void chunk_cumsum_kernel(const float *__restrict__ dt_p,
+                                    const float *__restrict__ A_log,
+                                    const float *__restrict__ dt_bias, int H, int N,
+                                    int chunk, float *__restrict__ acs,
+                                    float *__restrict__ chunk_sum,
+                                    DeviceStatus *status) {
+    __shared__ float warp_tot[8];
+    const int c = blockIdx.x, bh = blockIdx.y, h = bh % H;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    if (status && c == 0 && bh == 0 && t == 0) {
+        status->code = 0;
+        status->detail = 0;
+    }
+    const size_t idx = (size_t)bh * N + (size_t)c * chunk + t;
+    const float A = -expf(A_log[h]);
+    float x = A * softplus_f(dt_p[idx] + dt_bias[h]);
+    // inclusive warp scan, then add the totals of the warps before
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[warp] = x;
+    __syncthreads();
+    float before = 0.0f;
+    for (int w = 0; w < warp; ++w) before += warp_tot[w];
+    x += before;
+    acs[idx] = x;
+    if (t == chunk - 1) chunk_sum[(size_t)bh * (N / chunk) + c] = x;
+}
+
+// ---------------------------------------------------------------- kernel (b)
+constexpr int kThreads = 256;
+constexpr int kJT = 32;      // tokens per shared-memory tile
+constexpr int kStateTM = 16; // state rows per block in chunk_state
+constexpr int kMaxOut = 5;   // ceil(16 * 65 / 256)
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
+                   const float *__restrict__ acs, const float *__restrict__ lam, int N,
+                   int d, int order, int chunk, float *__restrict__ states) {
+    __shared__ float ks[kJT * 64];
+    __shared__ float vs[kJT * 64];
+    __shared__ float ws[kJT];
+    const int mt = blockIdx.x, c = blockIdx.y, bh = blockIdx.z;
+    const int nc = N / chunk;
+    const int Dphi = order == 1 ? d : d * d;
+    const int ld = d + 1;
+    const int m0 = mt * kStateTM;
+    const int n_out = kStateTM * ld;
+    const float lam_c = lam[(size_t)bh * nc + c];
+    const size_t tok0 = (size_t)bh * N + (size_t)c * chunk;
+
+    int om[kMaxOut], oc[kMaxOut];
+    float acc[kMaxOut];
+#pragma unroll
+    for (int r = 0; r < kMaxOut; ++r) {
+        int o = threadIdx.x + r * kThreads;
+        om[r] = m0 + o / ld;
+        oc[r] = o % ld;
+        acc[r] = 0.0f;
+        if (o >= n_out || om[r] >= Dphi) om[r] = -1;
+    }
+    for (int j0 = 0; j0 < chunk; j0 += kJT) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < kJT * d; e += kThreads) {
+            int jj = e / d, cc = e % d;
+            ks[jj * d + cc] = load_elem(k, (tok0 + j0 + jj) * d + cc);
+            vs[jj * d + cc] = load_elem(v, (tok0 + j0 + jj) * d + cc);
+        }
+        if (threadIdx.x < kJT) ws[threadIdx.x] = expf(lam_c - acs[tok0 + j0 + threadIdx.x]);
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < kMaxOut; ++r) {
+            if (om[r] < 0) continue;
+            const int m = om[r], cc = oc[r];
+            const int ma = order == 1 ? m : m / d, mb = order == 1 ? -1 : m % d;
+            float s = acc[r];
+            for (int jj = 0; jj < kJT; ++jj) {
+                float f = ks[jj * d + ma];
+                if (mb >= 0) f *= ks[jj * d + mb];
+                float vv = cc < d ? vs[jj * d + cc] : 1.0f;
+                s = fmaf(ws[jj] * f, vv, s);
+            }
+            acc[r] = s;
+        }
+    }
+    float *dst = states + ((size_t)bh * nc + c) * (size_t)Dphi * ld;
+#pragma unroll
+    for (int r = 0; r < kMaxOut; ++r)
+        if (om[r] >= 0) dst[(size_t)om[r] * ld + oc[r]] = acc[r];
+}
+
+// ---------------------------------------------------------------- kernel (c)
+// One thread per state element; walks the chunks in order, replacing each
+// chunk's own contribution U_c by the state entering the chunk.
+__global__ void state_scan_kernel(float *__restrict__ states, const float *__restrict__ lam,
+                                  int nc, size_t elems_per_state, int BH) {
+    const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int bh = blockIdx.y;
+    if (e >= elems_per_state || bh >= BH) return;
+    float *base = states + (size_t)bh * nc * elems_per_state + e;
+    const float *lb = lam + (size_t)bh * nc;
+    float h = 0.0f;
+    for (int c = 0; c < nc; ++c) {
+        float u = base[(size_t)c * elems_per_state];
+        base[(size_t)c * elems_per_state] = h;
+        h = fmaf(expf(lb[c]), h, u);
+    }
+}
+
+// ---------------------------------------------------------------- kernel (d)
+constexpr int kTI = 16;  // output rows per block
+constexpr int kTM2 = 32; // state rows per shared-memory tile
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                    const T *__restrict__ v, const float *__restrict__ acs,
+                    const float *__restrict__ states, const float *__restrict__ D, int H,
+                    int N, int d, int order, int normalize, int chunk, T *__restrict__ out) {
+    __shared__ float qs[kTI * 64];
+    __shared__ float ks[kJT * 64];
+    __shared__ float vs[kJT * 64];
+    __shared__ float ps[kTI * kJT];
+    __shared__ float ss[kTM2 * 65];
+    __shared__ float ys[kTI * 65];
+    __shared__ float acs_i[kTI];
+
+    const int it = blockIdx.x, c = blockIdx.y, bh = blockIdx.z, h = bh % H;
+    const int nc = N / chunk;
+    const int Dphi = order == 1 ? d : d * d;
+    const int ld = d + 1;
+    const int i0 = it * kTI;  // first row of this block inside the chunk
+    const size_t tok0 = (size_t)bh * N + (size_t)c * chunk;
+    const int n_out = kTI * ld;
+
+    for (int e = threadIdx.x; e < kTI * d; e += kThreads)
+        qs[e] = load_elem(q, (tok0 + i0) * d + e);
+    if (threadIdx.x < kTI) acs_i[threadIdx.x] = acs[tok0 + i0 + threadIdx.x];
+
+    int oi[kMaxOut], oc[kMaxOut];
+    float acc[kMaxOut], off[kMaxOut];
+#pragma unroll
+    for (int r = 0; r < kMaxOut; ++r) {
+        int o = threadIdx.x + r * kThreads;
+        oi[r] = o < n_out ? o / ld : -1;
+        oc[r] = o % ld;
+        acc[r] = 0.0f;
+        off[r] = 0.0f;
+    }
+
+    // intra-chunk part: tokens j of this chunk with j <= last row of the block
+    const int j_end = i0 + kTI;
+    for (int j0 = 0; j0 < j_end; j0 += kJT) {
+        __syncthreads();
+        for (int e = threadIdx.x; e < kJT * d; e += kThreads) {
+            int jj = e / d, cc = e % d;
+            ks[jj * d + cc] = load_elem(k, (tok0 + j0 + jj) * d + cc);
+            vs[jj * d + cc] = load_elem(v, (tok0 + j0 + jj) * d + cc);
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < kTI * kJT; e += kThreads) {
+            int ii = e / kJT, jj = e % kJT;
+            int i = i0 + ii, j = j0 + jj;
+            float w = 0.0f;
+            if (j <= i) {
+                float s = 0.0f;
+                for (int cc = 0; cc < d; ++cc) s = fmaf(qs[ii * d + cc], ks[jj * d + cc], s);
+                float sc = order == 1 ? s : s * s;
+                w = sc * expf(acs_i[ii] - acs[tok0 + j]);
+            }
+            ps[e] = w;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < kMaxOut; ++r) {
+            if (oi[r] < 0) continue;
+            float s = acc[r];
+            const int ii = oi[r], cc = oc[r];
+            for (int jj = 0; jj < kJT; ++jj) {
+                float vv = cc < d ? vs[jj * d + cc] : 1.0f;
+                s = fmaf(ps[ii * kJT + jj], vv, s);
+            }
+            acc[r] = s;
+        }
+    }
+
+    // carried-state part: phi(q_i)^T S_c, scaled by exp(acs_i)
+    if (c > 0) {
+        const float *S = states + ((size_t)bh * nc + c) * (size_t)Dphi * ld;
+        for (int m0 = 0; m0 < Dphi; m0 += kTM2) {
+            __syncthreads();
+            for (int e = threadIdx.x; e < kTM2 * ld; e += kThreads) {
+                int mm = e / ld;
+                ss[e] = (m0 + mm < Dphi) ? S[(size_t)m0 * ld + e] : 0.0f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int r = 0; r < kMaxOut; ++r) {
+                if (oi[r] < 0) continue;
+                const int ii = oi[r], cc = oc[r];
+                float s = off[r];
+                const int mlim = min(kTM2, Dphi - m0);
+                for (int mm = 0; mm < mlim; ++mm) {
+                    int m = m0 + mm;
+                    float f;
+                    if (order == 1) f = qs[ii * d + m];
+                    else f = qs[ii * d + m / d] * qs[ii * d + m % d];
+                    s = fmaf(f, ss[mm * ld + cc], s);
+                }
+                off[r] = s;
+            }
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kMaxOut; ++r)
+        if (oi[r] >= 0) ys[oi[r] * ld + oc[r]] = fmaf(expf(acs_i[oi[r]]), off[r], acc[r]);
+    __syncthreads();
+    for (int e = threadIdx.x; e < kTI * d; e += kThreads) {
+        int ii = e / d, cc = e % d;
+        float y = ys[ii * ld + cc];
+        if (normalize) y = y / ys[ii * ld + d];
+        size_t gi = (tok0 + i0 + ii) * d + cc;
+        if (D) y = fmaf(D[h * d + cc], load_elem(v, gi), y);
+        store_elem(out, gi, y);
+    }
+}
+
+template <typename T>
+int run_simt(const FwdArgs &a, const Plan &p) {
+    char *ws = static_cast<char *>(a.workspace);
+    float *acs = reinterpret_cast<float *>(ws + p.acs_off);
+    float *lam = reinterpret_cast<float *>(ws + p.lam_off);
+    float *states = reinterpret_cast<float *>(ws + p.state_off);
+    DeviceStatus *status = reinterpret_cast<DeviceStatus *>(ws);
+    const int BH = a.B * a.H, nc = a.N / a.chunk;
+    const int Dphi = a.order == 1 ? a.d : a.d * a.d;
+    int rc = launch_chunk_cumsum(a.dt_p, a.A_log, a.dt_bias, a.B, a.H, a.N, a.chunk, acs, lam,
+                                 status, a.stream);
+    if (rc != SSD_OK) return rc;
+    const T *q = static_cast<const T *>(a.q);
+    const T *k = static_cast<const T *>(a.k);
+    const T *v = static_cast<const T *>(a.v);
+    dim3 g1((Dphi + kStateTM - 1) / kStateTM, nc, BH);
+    chunk_state_kernel<T><<<g1, kThreads, 0, a.stream>>>(k, v, acs, lam, a.N, a.d, a.order,
+                                                         a.chunk, states);
+    const size_t elems = (size_t)Dphi * (a.d + 1);
+    dim3 g2((unsigned)((elems + 255) / 256), BH);
+    state_scan_kernel<<<g2, 256, 0, a.stream>>>(states, lam, nc, elems, BH);
+    dim3 g3(a.chunk / kTI, nc, BH);
+    chunk_output_kernel<T><<<g3, kThreads, 0, a.stream>>>(
+        q, k, v, acs, states, a.D, a.H, a.N, a.d, a.order, a.normalize, a.chunk,
+        static_cast<T *>(a.out));
+    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias, int B,
+                        int H, int N, int chunk, float *acs, float *chunk_sum,
+                        DeviceStatus *status, cudaStream_t stream) {
+    dim3 grid(N / chunk, B * H);
+    chunk_cumsum_kernel<<<grid, chunk, 0, stream>>>(dt_p, A_log, dt_bias, H, N, chunk, acs,
+                                                    chunk_sum, status);
+    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+int launch_simt(const FwdArgs &a, const Plan &p) {
+    if (a.dtype == SSD_F32) return run_simt<float>(a, p);
+    return run_simt<__nv_bfloat16>(a, p);
+}
+
+}  // namespace ssd

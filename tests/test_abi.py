@@ -1,0 +1,93 @@
+"""The C ABI: libssd.so loads, exports every function include/ssd.h declares,
+and rejects bad arguments before touching the device (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mamba_ssd_sequence_b200 as ssd
+from mamba_ssd_sequence_b200 import build as ssd_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ssd_build.build()
+    return ssd.load_library()
+
+
+def _declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(ssd_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert "ssd_fwd" in names and "ssd_workspace_bytes" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_workspace_bytes_rejects_invalid(lib):
+    ok = ssd.ssd_workspace_bytes(4, 16, 2048, 64, ssd.SSD_BF16, 1, 128)
+    assert ok > 0 and ok % 256 == 0
+    assert ssd.ssd_workspace_bytes(4, 16, 2000, 64, ssd.SSD_BF16, 1, 128) == 0  # N % chunk
+    assert ssd.ssd_workspace_bytes(4, 16, 2048, 48, ssd.SSD_BF16, 1, 128) == 0  # d_h
+    assert ssd.ssd_workspace_bytes(4, 16, 2048, 64, 7, 1, 128) == 0             # dtype
+    assert ssd.ssd_workspace_bytes(4, 16, 2048, 64, ssd.SSD_BF16, 3, 128) == 0  # order
+    assert ssd.ssd_workspace_bytes(4, 16, 2048, 64, ssd.SSD_BF16, 1, 96) == 0   # chunk
+    assert ssd.ssd_workspace_bytes(0, 16, 2048, 64, ssd.SSD_BF16, 1, 128) == 0  # empty batch
+
+
+def _call_fwd(lib, **over):
+    a = dict(q=16, k=32, v=48, dt_p=64, A_log=80, dt_bias=96, D=None, B=1, H=2, N=256, d=16,
+             dtype=ssd.SSD_F32, order=1, normalize=0, chunk=64, out=112, ws=256, ws_bytes=1 << 30)
+    a.update(over)
+    return lib.ssd_fwd(a["q"], a["k"], a["v"], a["dt_p"], a["A_log"], a["dt_bias"], a["D"],
+                       a["B"], a["H"], a["N"], a["d"], a["dtype"], a["order"], a["normalize"],
+                       a["chunk"], a["out"], a["ws"], a["ws_bytes"], None)
+
+
+def test_fwd_validation_codes(lib):
+    """Every rejection happens on the host, before any CUDA call (the fake
+    pointers are never dereferenced)."""
+    assert _call_fwd(lib, q=None) == 1          # SSD_ERR_NULL
+    assert _call_fwd(lib, out=None) == 1
+    assert _call_fwd(lib, N=250) == 2           # SSD_ERR_SHAPE (N % chunk)
+    assert _call_fwd(lib, N=0) == 2
+    assert _call_fwd(lib, d=24) == 2
+    assert _call_fwd(lib, dtype=5) == 3         # SSD_ERR_DTYPE
+    assert _call_fwd(lib, order=0) == 4         # SSD_ERR_ORDER
+    assert _call_fwd(lib, chunk=32) == 5        # SSD_ERR_CHUNK
+    assert _call_fwd(lib, k=33) == 6            # SSD_ERR_ALIGN
+    assert _call_fwd(lib, D=8) == 6
+    assert _call_fwd(lib, ws=128) == 6          # workspace needs 256-byte alignment
+    assert _call_fwd(lib, ws=None) == 7         # SSD_ERR_WORKSPACE
+    assert _call_fwd(lib, ws_bytes=100) == 7
+
+
+def test_status_strings(lib):
+    for code in range(11):
+        s = ssd.status_str(code)
+        assert s.startswith("SSD_")
+    assert ssd.status_str(99) == "unknown ssd status"
+
+
+def test_path_selection(lib):
+    path, n = ssd.ssd_fwd_path(1, 2, 256, 16, ssd.SSD_F32, 1, 64)
+    assert path == "simt" and n == 4
+    with pytest.raises(ValueError):
+        ssd.ssd_fwd_path(1, 2, 250, 16, ssd.SSD_F32, 1, 64)
+
+
+def test_cumsum_validation(lib):
+    assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 100, 64, 64, 80, None) == 2
+    assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 128, 48, 64, 80, None) == 5
+    assert lib.ssd_chunk_cumsum(None, 32, 48, 1, 1, 128, 64, 64, 80, None) == 1
