@@ -140,7 +140,8 @@ def test_repeatable_and_status_clean():
 
 def test_output_guard_bands_untouched():
     """Nothing is written outside out[]: canaries before and after it."""
-    for dtype, order in [("f32", 1), ("bf16", 1), ("bf16", 2)]:
+    for dtype, order, chunk in [("f32", 1, 64), ("bf16", 1, 64), ("bf16", 1, 128),
+                                ("bf16", 2, 64)]:
         x = inputs.make_inputs(1, 2, 256, 64, dtype, seed=8)
         dev = to_device(x, dtype)
         n = dev["q"].numel()
@@ -148,7 +149,7 @@ def test_output_guard_bands_untouched():
         buf = torch.full((n + 2 * pad,), 7.0, dtype=dev["q"].dtype, device="cuda")
         out = buf[pad:pad + n].view_as(dev["q"])
         ssd.ssd_fwd(dev["q"], dev["k"], dev["v"], dev["dt_p"], dev["A_log"], dev["dt_bias"],
-                    dev["D"], order, order == 2, 64, out=out)
+                    dev["D"], order, order == 2, chunk, out=out)
         torch.cuda.synchronize()
         assert torch.all(buf[:pad] == 7.0) and torch.all(buf[pad + n:] == 7.0)
 
