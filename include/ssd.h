@@ -144,6 +144,38 @@ int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias
  */
 int ssd_status_from_workspace(const void *workspace, void *stream);
 
+/*
+ * ssd_fwd() for callers that cannot allocate device memory: a library or
+ * plugin whose host application owns the device memory pool and forbids
+ * cudaMalloc, or code that must not risk the device-wide synchronisation
+ * that cudaMalloc / cudaFree can cause.  The operator has no counterpart of
+ * this call on the pages; it only changes where the scratch lives.
+ *
+ * It runs the general SIMT path (four kernels) on a scratch buffer built
+ * into the library: a fixed 16 MiB array in device memory, which every GPU
+ * that loads the library holds until the process exits.  Nothing is
+ * allocated and no workspace is passed; inputs and output are the caller's
+ * device buffers, with the shapes and rules of ssd_fwd().
+ *  - Problems whose scratch (the same as ssd_fwd's SIMT path: about
+ *    4*B*H*N + 4*B*H*(N/chunk)*d_h^order*(d_h+1) bytes) exceeds 16 MiB are
+ *    rejected with SSD_ERR_WORKSPACE before anything is enqueued.
+ *  - The first call on a device looks up the buffer's device address on
+ *    that device (cudaGetSymbolAddress); make that first call before any
+ *    stream capture.
+ *  - All calls on one device share the one buffer and it keeps the last
+ *    call's contents (the kernels write everything they later read).  Calls
+ *    that can overlap on the GPU -- on different streams without ordering
+ *    between them -- race on it and give wrong results; serialise them.
+ *  - The path has no device-side waits, so there is no device status to
+ *    read back.
+ */
+int ssd_fwd_noalloc(const void *q, const void *k, const void *v,
+                    const float *dt_p, const float *A_log, const float *dt_bias,
+                    const float *D,
+                    int B, int H, int N, int d_h, int dtype,
+                    int order, int normalize, int chunk,
+                    void *out, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *ssd_status_str(int status);
 
