@@ -21,11 +21,21 @@ static int check_shape(int B, int H, int N, int d, int dtype, int order, int chu
     return SSD_OK;
 }
 
-bool make_plan(int B, int H, int N, int d, int dtype, int order, int chunk, Plan *plan) {
-    if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
+static size_t simt_total(int B, int H, int N, int d, int order, int chunk, Plan *p) {
     const size_t BH = (size_t)B * H, nc = (size_t)N / chunk;
+    const size_t Dphi = order == 1 ? (size_t)d : (size_t)d * d;
+    p->acs_off = kStatusBytes;
+    p->lam_off = align_up(p->acs_off + BH * N * sizeof(float), 256);
+    p->state_off = align_up(p->lam_off + BH * nc * sizeof(float), 256);
+    p->total = align_up(p->state_off + BH * nc * Dphi * (d + 1) * sizeof(float), 256);
+    return p->total;
+}
+
+bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
+               Plan *plan) {
+    if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
     Plan p{};
-    if (order == 1 && tc_order1_supports(B, H, N, d, dtype, chunk)) {
+    if (order == 1 && !normalize && tc_order1_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER1;
         p.n_launches = 1;
         p.acs_off = p.lam_off = p.state_off = kStatusBytes;
@@ -36,13 +46,9 @@ bool make_plan(int B, int H, int N, int d, int dtype, int order, int chunk, Plan
         p.acs_off = p.lam_off = p.state_off = kStatusBytes;
         p.total = kStatusBytes + tc_order2_workspace(B, H, N, d, chunk);
     } else {
-        const size_t Dphi = order == 1 ? (size_t)d : (size_t)d * d;
         p.path = PATH_SIMT;
         p.n_launches = 4;
-        p.acs_off = kStatusBytes;
-        p.lam_off = align_up(p.acs_off + BH * N * sizeof(float), 256);
-        p.state_off = align_up(p.lam_off + BH * nc * sizeof(float), 256);
-        p.total = align_up(p.state_off + BH * nc * Dphi * (d + 1) * sizeof(float), 256);
+        simt_total(B, H, N, d, order, chunk, &p);
     }
     *plan = p;
     return true;
@@ -55,15 +61,17 @@ using namespace ssd;
 extern "C" {
 
 size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk) {
-    Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, chunk, &p)) return 0;
-    return p.total;
+    // the size covers both settings of `normalize`, which can select different paths
+    Plan p0, p1;
+    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, &p0)) return 0;
+    if (!make_plan(B, H, N, d_h, dtype, order, 1, chunk, &p1)) return 0;
+    return p0.total > p1.total ? p0.total : p1.total;
 }
 
 int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
                  int *n_launches) {
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, chunk, &p)) return -1;
+    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, &p)) return -1;
     if (n_launches) *n_launches = p.n_launches;
     return p.path;
 }
@@ -82,7 +90,7 @@ int ssd_fwd(const void *q, const void *k, const void *v, const float *dt_p,
     if (D && !aligned16(D)) return SSD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, chunk, &p)) return SSD_ERR_UNSUPPORTED;
+    if (!make_plan(B, H, N, d_h, dtype, order, normalize, chunk, &p)) return SSD_ERR_UNSUPPORTED;
     if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
     FwdArgs a{q, k, v, dt_p, A_log, dt_bias, D, B, H, N, d_h, dtype, order, normalize ? 1 : 0,
               chunk, out, workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};

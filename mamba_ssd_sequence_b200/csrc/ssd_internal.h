@@ -43,7 +43,8 @@ struct Plan {
 };
 
 // Fills `plan` for validated arguments; returns false if no kernel exists.
-bool make_plan(int B, int H, int N, int d, int dtype, int order, int chunk, Plan *plan);
+bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
+               Plan *plan);
 
 // Path launchers (each returns an ssd_status).
 int launch_simt(const FwdArgs &a, const Plan &p);

@@ -1,22 +1,33 @@
 // Order-1 tensor-core path (tcgen05 + TMEM, TMA) of the SSD forward operator
-// for bf16 inputs, d_h = 64, chunk = 128.
+// for bf16 inputs, d_h = 64, chunk = 128, no normaliser.
 //
-// One CTA per (batch, head) walks that head's chunks in order, keeping the
-// carried state h (d_h x d_h, fp32) in tensor memory, so every q/k/v tile is
-// read from HBM exactly once and the state never leaves the SM.  Per chunk
-// (2Mamba2Furious, Algorithms 1, 3, 4 and 6; the chunked split is the
-// standard state-passing form of the semiseparable mask):
-//   acs_t   = chunk-local inclusive cumsum of A*dt          (kernel (a), fused)
-//   S       = Q K^T                                        (tcgen05, TMEM)
-//   P_ij    = S_ij exp(acs_i - acs_j) [i >= j]              (CUDA cores -> smem bf16)
-//   Y       = P V                                          (tcgen05, TMEM)
-//   Y_off   = Q h_{c-1}                                    (tcgen05, TMEM)
-//   h_c     = exp(lam_c) h_{c-1} + K'^T V,  K'_j = exp(lam_c - acs_j) k_j
-//                                                          (tcgen05, accumulating in TMEM)
-//   y_i     = Y_i + exp(acs_i) Y_off_i  [/ row sum] [+ D v_i]  (epilogue, TMA store)
-// All exponentials are of non-positive arguments (chunk-local differences),
-// so nothing overflows.  The normaliser state z (d_h floats) is kept in
-// shared memory in fp32.
+// Each (batch, head) is split into R segments of whole chunks; one CTA per
+// segment.  A CTA first folds the chunks before its segment into the carried
+// state (K and V only, no output), then produces its own chunks; so it never
+// waits for another CTA, and the state it carries never leaves the SM.  Per
+// chunk c (2Mamba2Furious, Algorithms 1, 3, 4 and 6, evaluated in the
+// chunked state-passing form of the semiseparable mask):
+//   acs_t = chunk-local inclusive cumsum of A*dt (log2 units)  (kernel (a), fused)
+//   S     = Q K^T                                  tcgen05, fp32 in TMEM
+//   P_ij  = S_ij 2^(acs_i - acs_j) [i >= j]        CUDA cores, bf16 back into TMEM
+//   U_c   = K'^T V,   K'_j = 2^(lam_c - acs_j) k_j  tcgen05 (the chunk's own state term)
+//   h_c   = 2^(lam_c) h_{c-1} + U_c                 CUDA cores, fp32
+//   Y     = P V + Q' h_{c-1},  Q'_i = 2^(acs_i) q_i  tcgen05 (P from TMEM)
+//   y_i   = Y_i [+ D v_i]                           epilogue, 16-byte stores
+//
+// Warp roles (608 threads): warp 0 issues TMA loads into a 3-stage ring;
+// warps 1 and 2 each issue the MMAs of one compute group in a fixed order
+// (blocking, bounded waits: no polling); warps 3-10 and 11-18 are two compute
+// groups that take even and odd chunks (ping-pong), so one group's
+// exponentials overlap the other's MMAs and epilogue.  In a group the two
+// warps that share a TMEM lane quarter split each row's columns.  Each group
+// keeps its own copy of the carried state and advances it two chunks at a
+// time, h_{c-1} = 2^(lam_{c-1}) h_{c-2} + U_{c-1}, where U_{c-1} is the other
+// group's chunk term read from TMEM: the only cross-group dependency is an
+// MMA result, never a chain of group-to-group hand-offs.  All exponentials
+// are of non-positive arguments (chunk-local differences).  Every wait is
+// bounded; a timeout sets SSD_ERR_TIMEOUT in the workspace status and all
+// roles leave their loops.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -30,347 +41,471 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kC = 128;         // chunk length (rows of every tile)
-constexpr int kD = 64;          // head dim
-constexpr int kThreads = 128;   // one thread per chunk row / TMEM lane
+constexpr int kC = 128;             // chunk length = rows of every tile
+constexpr int kD = 64;              // head dim
+constexpr int kStages = 3;          // TMA ring depth
+constexpr int kGroupThreads = 256;  // one compute group: 8 warps, 2 per TMEM lane quarter
+constexpr int kFirstGroupWarp = 3;
+constexpr int kThreads = 32 * kFirstGroupWarp + 2 * kGroupThreads;
 constexpr uint32_t kTileBytes = kC * kD * 2;  // 16 KiB bf16 tile
 constexpr uint32_t kStageBytes = 3 * kTileBytes;
 
-// shared-memory map (offsets from a 1024-aligned base)
-constexpr uint32_t kOffStage = 0;                               // 2 x {Q, K, V}
-constexpr uint32_t kOffP = kOffStage + 2 * kStageBytes;         // P: 2 column blocks
-constexpr uint32_t kOffKp = kOffP + 2 * kTileBytes;             // K' (MN-major operand)
-constexpr uint32_t kOffHs = kOffKp + kTileBytes;                // h_{c-1} bf16, 64 x 64
-constexpr uint32_t kOffMisc = kOffHs + kD * kD * 2;
-constexpr uint32_t kSmemBytes = kOffMisc + 1024 + 1024;         // misc + alignment slack
+constexpr uint32_t kHRow = kD + 4;                               // padded fp32 row of h
+constexpr uint32_t kOffStage = 0;                                // kStages x {Q, K, V}
+constexpr uint32_t kOffHs = kOffStage + kStages * kStageBytes;   // 2 x h_{c-1} bf16 (64 x 64)
+constexpr uint32_t kOffH32 = kOffHs + 2 * kD * kD * 2;           // 2 x own state h (fp32)
+constexpr uint32_t kOffDres = kOffH32 + 2 * kD * kHRow * 4;      // D of this head (fp32)
+constexpr uint32_t kOffMisc = kOffDres + kD * 4;
+constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;          // misc + alignment slack
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S: 128 x 128 fp32
-constexpr uint32_t kColY = 128;    // Y: 128 x 64
-constexpr uint32_t kColYoff = 192; // Y_off: 128 x 64
-constexpr uint32_t kColH = 256;    // h: 64 x 64 (M=64 layout: rows at lanes 32w + 0..15)
+constexpr uint32_t kColS = 0;     // 2 x 128: S (fp32), then P (bf16 pairs) at [32, 96)
+constexpr uint32_t kColP = 32;    // offset of P inside an S slot
+constexpr uint32_t kColY = 256;   // 2 x 64: Y
+constexpr uint32_t kColU = 384;   // 2 x 64: U (M = 64 layout, rows at lanes 32g + 0..15)
 
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Misc {
-    float acs2[kC];      // chunk-local cumsum, log2 units
-    float z[kD];         // normaliser state
-    float wtot[4];
-    uint64_t bar_tma[2];
-    uint64_t bar_s;
-    uint64_t bar_mma;
+    float acs2[2][kC];
+    float wtot[2][4];
+    float lam_red[2][4];
+    uint64_t stage_full[kStages];
+    uint64_t stage_empty[kStages];
+    uint64_t s_full[2], kp_full[2], p_full[2], u_full[2], u_free[2], hs_full[2], y_full[2],
+        y_free[2];
     uint32_t tmem_base;
     int abort_flag;
 };
+static_assert(sizeof(Misc) <= 2048, "misc block");
 
 __device__ __forceinline__ float softplus_f(float x) {
     return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
-
-__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) {  // K-major, 128B swizzle
-    return make_sdesc(saddr, 16, 1024);
-}
-__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {  // MN-major, 128B swizzle
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) { return make_sdesc(saddr, 16, 1024); }
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {
     return make_sdesc(saddr, kTileBytes, 1024);
 }
+// bf16 pair (low, high) -> float2
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) { return pack_bf16x2(v.x, v.y); }
 
-__device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+// Scales columns [32 hf, 32 hf + 32) of row `row` of a 128B-swizzled bf16 tile.
+__device__ __forceinline__ void scale_half_row_inplace(uint8_t *tile, int row, int hf, float s) {
+    const float2 s2 = make_float2(s, s);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    for (int q = 0; q < 4; ++q) {
+        uint4 *p = reinterpret_cast<uint4 *>(tile + sw128_chunk(row, hf * 4 + q));
+        uint4 u = *p;
+        u.x = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.x), s2));
+        u.y = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.y), s2));
+        u.z = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.z), s2));
+        u.w = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.w), s2));
+        *p = u;
     }
 }
-__device__ __forceinline__ uint4 pack8(const float *f) {
-    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
-                      pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+
+// P for 16 columns (tokens j0 .. j0+15, all inside column block jb) of this
+// thread's row, from the S values `sv` already loaded; writes 8 packed bf16
+// columns of TMEM at column j0 / 2.  Blocks entirely above the diagonal
+// (jb > g) are written as zeros.
+__device__ __forceinline__ void build_p16(uint32_t tP, int j0, int jb, int g, int row, float acs2,
+                                          const float *acs_row, const float (&sv)[16]) {
+    uint32_t pk[8];
+    if (jb > g) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pk[e] = 0u;
+    } else {
+        const float2 ai = make_float2(acs2, acs2);
+        const float4 *ac = reinterpret_cast<const float4 *>(acs_row + j0);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 aj = ac[q4];
+            const float2 d0 = __fadd2_rn(ai, make_float2(-aj.x, -aj.y));
+            const float2 d1 = __fadd2_rn(ai, make_float2(-aj.z, -aj.w));
+            float2 p0 = __fmul2_rn(make_float2(sv[q4 * 4], sv[q4 * 4 + 1]),
+                                   make_float2(ex2_approx(d0.x), ex2_approx(d0.y)));
+            float2 p1 = __fmul2_rn(make_float2(sv[q4 * 4 + 2], sv[q4 * 4 + 3]),
+                                   make_float2(ex2_approx(d1.x), ex2_approx(d1.y)));
+            if (jb == g) {  // the diagonal block: keep j <= i
+                const int j = j0 + q4 * 4;
+                if (j > row) p0.x = 0.0f;
+                if (j + 1 > row) p0.y = 0.0f;
+                if (j + 2 > row) p1.x = 0.0f;
+                if (j + 3 > row) p1.y = 0.0f;
+            }
+            pk[q4 * 2] = f2_to_bf2(p0);
+            pk[q4 * 2 + 1] = f2_to_bf2(p1);
+        }
+    }
+    tmem_st8(tP + j0 / 2, pk);
 }
 
-__device__ __forceinline__ void record_timeout(DeviceStatus *status, int where, Misc *misc) {
+__device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
     if (status) {
         atomicCAS(&status->code, 0, (int)SSD_ERR_TIMEOUT);
-        atomicExch(&status->detail, where);
+        atomicCAS(&status->detail, 0, where);
     }
-    misc->abort_flag = 1;
+    *reinterpret_cast<volatile int *>(&misc->abort_flag) = 1;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
 tc_order1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                  const float *__restrict__ dt_p, const float *__restrict__ A_log,
                  const float *__restrict__ dt_bias, const float *__restrict__ Dres, int H, int N,
-                 int normalize, DeviceStatus *status) {
+                 int BH, int R, DeviceStatus *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Misc *misc = reinterpret_cast<Misc *>(smem + kOffMisc);
-    const uint32_t sbase = smem_u32(smem);
+    const volatile int *abort_flag = &misc->abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, h = bh % H;
+    const int bh = blockIdx.x % BH, seg = blockIdx.x / BH, h = bh % H;
     const int nc = N / kC;
     const int row0 = bh * N;
+    // This CTA produces the outputs of chunks [c_begin, c_end) of its head.
+    // Chunks [0, c_begin) are only folded into the carried state (K and V
+    // are read, no output), so the CTA starts its own segment from the exact
+    // state without waiting for another CTA.
+    const int c_begin = (seg * nc) / R, c_end = ((seg + 1) * nc) / R;
+    // index of own chunk c among the own chunks of its parity (phases of the
+    // barriers that only own chunks use)
+    auto own_idx = [&](int c) { return (c - (c_begin + ((c ^ c_begin) & 1))) >> 1; };
 
     if (tid == 0) {
-        if (bh == 0 && status) {
+        if (blockIdx.x == 0 && status) {
             status->code = 0;
             status->detail = 0;
         }
-        mbar_init(&misc->bar_tma[0], 1);
-        mbar_init(&misc->bar_tma[1], 1);
-        mbar_init(&misc->bar_s, 1);
-        mbar_init(&misc->bar_mma, 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&misc->stage_full[i], 1);
+            mbar_init(&misc->stage_empty[i], kGroupThreads);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&misc->s_full[s], 1);
+            mbar_init(&misc->kp_full[s], kGroupThreads);
+            mbar_init(&misc->p_full[s], kGroupThreads);
+            mbar_init(&misc->u_full[s], 1);
+            mbar_init(&misc->u_free[s], 2 * kGroupThreads);
+            mbar_init(&misc->hs_full[s], kGroupThreads);
+            mbar_init(&misc->y_full[s], 1);
+            mbar_init(&misc->y_free[s], kGroupThreads);
+        }
         misc->abort_flag = 0;
         fence_mbar_init();
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
-        prefetch_tmap(&tm_o);
     }
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(&misc->tmem_base, kTmemCols);
         tmem_relinquish();
     }
-    if (tid < kD) misc->z[tid] = 0.0f;
+    {
+        float *sD = reinterpret_cast<float *>(smem + kOffDres);
+        float *sH32 = reinterpret_cast<float *>(smem + kOffH32);
+        for (int i = tid; i < kD; i += kThreads) sD[i] = Dres ? Dres[h * kD + i] : 0.0f;
+        for (int i = tid; i < 2 * kD * (int)kHRow; i += kThreads) sH32[i] = 0.0f;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
-    const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
 
-    const float A2 = -expf(A_log[h]) * kLog2e;  // decay rate in log2 units
-    const float bias = dt_bias[h];
-    float dt_next = dt_p[(size_t)row0 + tid];
-
-    constexpr uint32_t idesc_S = make_idesc_bf16(128, 128, 0, 0);
-    constexpr uint32_t idesc_Y = make_idesc_bf16(128, 64, 0, 1);
-    constexpr uint32_t idesc_U = make_idesc_bf16(64, 64, 1, 1);
-
-    if (tid == 0) {
-        mbar_arrive_expect_tx(&misc->bar_tma[0], kStageBytes);
-        tma_load_2d(smem + kOffStage, &tm_q, 0, row0, &misc->bar_tma[0]);
-        tma_load_2d(smem + kOffStage + kTileBytes, &tm_k, 0, row0, &misc->bar_tma[0]);
-        tma_load_2d(smem + kOffStage + 2 * kTileBytes, &tm_v, 0, row0, &misc->bar_tma[0]);
-    }
-
-    for (int c = 0; c < nc; ++c) {
-        const int st = c & 1;
-        uint8_t *sQ = smem + kOffStage + st * kStageBytes;
-        uint8_t *sK = sQ + kTileBytes;
-        uint8_t *sV = sK + kTileBytes;
-        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
-
-        // ---- decay: chunk-local inclusive cumsum (log2 units), one token per thread
-        const float dtv = dt_next;
-        if (c + 1 < nc) dt_next = dt_p[(size_t)row0 + (size_t)(c + 1) * kC + tid];
-        float acs2 = A2 * softplus_f(dtv + bias);
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            float y = __shfl_up_sync(0xffffffffu, acs2, o);
-            if (lane >= o) acs2 += y;
-        }
-        if (lane == 31) misc->wtot[warp] = acs2;
-        __syncthreads();
-        for (int w = 0; w < warp; ++w) acs2 += misc->wtot[w];
-        misc->acs2[tid] = acs2;
-
-        // ---- q/k/v of this chunk
-        if (!mbar_wait_bounded(&misc->bar_tma[st], (c >> 1) & 1)) record_timeout(status, 1, misc);
-        __syncthreads();  // acs2[] complete; abort flag visible
-        if (misc->abort_flag) break;
-        const float lam2 = misc->acs2[kC - 1];
-
-        if (tid == 0) {
-            if (c + 1 < nc) {  // prefetch the next chunk into the other stage
-                bulk_wait_group_read0();  // staging of chunk c-1's output has been read
-                uint8_t *nQ = smem + kOffStage + (st ^ 1) * kStageBytes;
-                const int nrow = row0 + (c + 1) * kC;
-                mbar_arrive_expect_tx(&misc->bar_tma[st ^ 1], kStageBytes);
-                tma_load_2d(nQ, &tm_q, 0, nrow, &misc->bar_tma[st ^ 1]);
-                tma_load_2d(nQ + kTileBytes, &tm_k, 0, nrow, &misc->bar_tma[st ^ 1]);
-                tma_load_2d(nQ + 2 * kTileBytes, &tm_v, 0, nrow, &misc->bar_tma[st ^ 1]);
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < kD / 16; ++ks)
-                mma_bf16(tmem + kColS, desc_k(aQ + ks * 32), desc_k(aK + ks * 32), idesc_S, ks > 0);
-            mma_commit(&misc->bar_s);
-        }
-
-        // ---- K'_j = exp(lam - acs_j) k_j (row tid), same layout as K
-        {
-            const float wj = exp2f(lam2 - acs2);
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                uint4 u = *reinterpret_cast<const uint4 *>(sK + sw128_chunk(tid, ch));
-                float f[8];
-                unpack8(u, f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] *= wj;
-                *reinterpret_cast<uint4 *>(smem + kOffKp + sw128_chunk(tid, ch)) = pack8(f);
-            }
-        }
-        // ---- h_{c-1}: bf16 copy for Y_off, then scale by exp(lam) in place
-        if (c > 0) {
-            const float decay = exp2f(lam2);
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float hv[32];
-                tmem_ld32(tmem + t_lane + kColH + half * 32, hv);
-                tmem_wait_ld();
-                if (lane < 16) {
-                    const int m = warp * 16 + lane;
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<uint4 *>(smem + kOffHs + sw128_chunk(m, half * 4 + q4)) =
-                            pack8(hv + q4 * 8);
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            for (int c = 0; c < c_end; ++c) {
+                const int st = c % kStages;
+                if (c >= kStages &&
+                    !mbar_wait_abortable(&misc->stage_empty[st], ((c / kStages) - 1) & 1, abort_flag)) {
+                    raise_timeout(misc, status, 10);
+                    break;
                 }
-#pragma unroll
-                for (int e = 0; e < 32; ++e) hv[e] *= decay;
-                tmem_st32(tmem + t_lane + kColH + half * 32, hv);
-            }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            // h (+)= K'^T V      (M = 64, N = 64, K = 128 tokens; both MN-major)
-#pragma unroll
-            for (int ks = 0; ks < kC / 16; ++ks)
-                mma_bf16(tmem + kColH, desc_mn(sbase + kOffKp + ks * 2048), desc_mn(aV + ks * 2048),
-                         idesc_U, (c > 0 || ks > 0) ? 1u : 0u);
-            // Y_off = Q h_{c-1}  (M = 128, N = 64, K = 64)
-            if (c > 0) {
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks)
-                    mma_bf16(tmem + kColYoff, desc_k(aQ + ks * 32),
-                             desc_mn(sbase + kOffHs + ks * 2048), idesc_Y, ks > 0);
+                uint8_t *dst = smem + kOffStage + st * kStageBytes;
+                const int r = row0 + c * kC;
+                const bool own = c >= c_begin;
+                mbar_arrive_expect_tx(&misc->stage_full[st], own ? kStageBytes : 2 * kTileBytes);
+                if (own) tma_load_2d(dst, &tm_q, 0, r, &misc->stage_full[st]);
+                tma_load_2d(dst + kTileBytes, &tm_k, 0, r, &misc->stage_full[st]);
+                tma_load_2d(dst + 2 * kTileBytes, &tm_v, 0, r, &misc->stage_full[st]);
             }
         }
+    } else if (warp < 3) {
+        // ------------------------------------------------------ MMA issuers
+        // Warp 1 issues every MMA of group 0's chunks, warp 2 of group 1's, in
+        // chunk order: S, U, P V, Q' h.  Same-thread issue order keeps the
+        // slot reuse of S / P, Y and h_{c-1} in order; U slots are shared with
+        // the other group and are guarded by u_free.
+        const int s = warp - 1;
+        if (lane == 0) {
+            constexpr uint32_t idesc_S = make_idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idesc_Y = make_idesc_bf16(128, 64, 0, 1);
+            constexpr uint32_t idesc_U = make_idesc_bf16(64, 64, 1, 1);
+            const uint32_t sbase = smem_u32(smem);
+            bool ok = true;
+            for (int c = s; ok && c < c_end; c += 2) {
+                const int k = c >> 1, st = c % kStages;
+                const bool own = c >= c_begin;
+                const int ko = own ? own_idx(c) : 0;
+                const uint32_t aQ = sbase + kOffStage + st * kStageBytes;
+                const uint32_t aK = aQ + kTileBytes, aV = aK + kTileBytes;
+                if (own) {  // S = Q K^T
+                    if (!(ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag)))
+                        break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_bf16(tmem + kColS + s * 128, desc_k(aQ + ks * 32), desc_k(aK + ks * 32),
+                                 idesc_S, ks > 0);
+                    mma_commit(&misc->s_full[s]);
+                }
+                // U_c = K'^T V   (M = 64, N = 64, K = 128 tokens; K' and V MN-major)
+                if (!(ok = mbar_wait_abortable(&misc->kp_full[s], k & 1, abort_flag))) break;
+                if (c >= 2 && !(ok = mbar_wait_abortable(&misc->u_free[s], (k - 1) & 1, abort_flag)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_bf16(tmem + kColU + s * 64, desc_mn(aK + ks * 2048), desc_mn(aV + ks * 2048),
+                             idesc_U, ks > 0);
+                mma_commit(&misc->u_full[s]);
+                if (!own) continue;
+                // Y = P V   (A = P from TMEM, 8 packed columns per 16 tokens)
+                if (!(ok = mbar_wait_abortable(&misc->p_full[s], ko & 1, abort_flag))) break;
+                if (ko >= 1 && !(ok = mbar_wait_abortable(&misc->y_free[s], (ko - 1) & 1, abort_flag)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_bf16_ts(tmem + kColY + s * 64, tmem + kColS + s * 128 + kColP + ks * 8,
+                                desc_mn(aV + ks * 2048), idesc_Y, ks > 0);
+                // Y += Q' h_{c-1}
+                if (!(ok = mbar_wait_abortable(&misc->hs_full[s], ko & 1, abort_flag))) break;
+                tc_fence_after();
+                if (c >= 1) {
+                    const uint32_t aH = sbase + kOffHs + s * (kD * kD * 2);
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks)
+                        mma_bf16(tmem + kColY + s * 64, desc_k(aQ + ks * 32), desc_mn(aH + ks * 2048),
+                                 idesc_Y, 1);
+                }
+                mma_commit(&misc->y_full[s]);
+            }
+            if (!ok) raise_timeout(misc, status, 20 + s);
+        }
+    } else if (warp >= kFirstGroupWarp) {
+        // ------------------------------------------------------ compute groups
+        const int s = (warp - kFirstGroupWarp) >> 3;  // 0: even chunks, 1: odd chunks
+        const int wi = (warp - kFirstGroupWarp) & 7;  // warp inside the group
+        const int g = warp & 3;                       // TMEM lane quarter = row block
+        const int hf = wi >> 2;                       // which half of each row's columns
+        const int row = g * 32 + lane;                // chunk row owned (shared by the halves)
+        const int wt = wi * 32 + lane;                // 0..255 inside the group
+        const int bar_id = 1 + s;                     // group barrier
+        const uint32_t lane_off = (uint32_t)(g * 32) << 16;
+        const float A2 = -expf(A_log[h]) * kLog2e;
+        const float bias = dt_bias[h];
+        // own carried state h_{c-2}, fp32 in shared memory (row m = 16g + lane)
+        float *hown = reinterpret_cast<float *>(smem + kOffH32) + s * kD * kHRow;
+        const float *sD = reinterpret_cast<const float *>(smem + kOffDres);
+        // half 0 scans this chunk's decay; half 1 sums the previous chunk's
+        // (the other group's), so each loads one dt per chunk, one ahead
+        const int dt_off = hf == 0 ? 0 : -1;
+        float dt_next = (s + dt_off >= 0 && s + dt_off < c_end)
+                            ? dt_p[(size_t)row0 + (s + dt_off) * kC + row] : 0.0f;
 
-        // ---- P = S (.) exp(acs_i - acs_j) [i >= j], row tid, bf16 into smem
-        if (!mbar_wait_bounded(&misc->bar_s, c & 1)) record_timeout(status, 2, misc);
-        tc_fence_after();
-        float rowsum = 0.0f;
+        for (int c = s; c < c_end; c += 2) {
+            const int k = c >> 1, st = c % kStages;
+            const bool own = c >= c_begin;  // produce outputs (else: state only)
+            const int ko = own ? own_idx(c) : 0;
+            uint8_t *sQ = smem + kOffStage + st * kStageBytes;
+            uint8_t *sK = sQ + kTileBytes;
+            uint8_t *sV = sK + kTileBytes;
+            const float dtv = dt_next;
+            const int cn = c + 2 + dt_off;
+            if (cn < c_end) dt_next = dt_p[(size_t)row0 + (size_t)cn * kC + row];
+
+            // ---- decay: scan of this chunk (half 0), total of chunk c-1 (half 1)
+            float a = (hf == 0 || c >= 1) ? A2 * softplus_f(dtv + bias) : 0.0f;
+            if (hf == 0) {
 #pragma unroll
-        for (int jb = 0; jb < kC / 32; ++jb) {
-            uint8_t *pblk = smem + kOffP + (jb >> 1) * kTileBytes;
-            if (jb > warp) {  // every column of this block is above the diagonal
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, a, o);
+                    if (lane >= o) a += y;
+                }
+                if (lane == 31) misc->wtot[s][g] = a;
+            } else {
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(pblk + sw128_chunk(tid, (jb & 1) * 4 + q4)) =
-                        make_uint4(0, 0, 0, 0);
+                for (int o = 1; o < 32; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                if (lane == 0) misc->lam_red[s][g] = a;
+            }
+            named_bar_sync(bar_id, kGroupThreads);
+            const float lam2 = misc->wtot[s][0] + misc->wtot[s][1] + misc->wtot[s][2] + misc->wtot[s][3];
+            const float lam2_prev = misc->lam_red[s][0] + misc->lam_red[s][1] + misc->lam_red[s][2] +
+                                    misc->lam_red[s][3];
+            if (hf == 0) {
+                for (int w = 0; w < g; ++w) a += misc->wtot[s][w];
+                misc->acs2[s][row] = a;
+            }
+
+            // ---- wait for this chunk's tiles and for S = Q K^T (after which Q and K
+            //      may be rewritten in place)
+            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
+            bad = bad || (own && !mbar_wait_abortable(&misc->s_full[s], ko & 1, abort_flag));
+            if (named_bar_any(bar_id, kGroupThreads, bad)) {
+                if (wt == 0) raise_timeout(misc, status, 32 + s);
+                break;
+            }
+            tc_fence_after();
+            const float acs2 = misc->acs2[s][row];
+
+            // ---- K'_j = 2^(lam - acs_j) k_j, in place in the stage's K tile (half row)
+            scale_half_row_inplace(sK, row, hf, ex2_approx(lam2 - acs2));
+            fence_proxy_async_smem();
+            mbar_arrive(&misc->kp_full[s]);
+
+            if (own) {
+                // ---- P = S (.) 2^(acs_i - acs_j) [i >= j] -> bf16 pairs back into TMEM,
+                // at columns [32, 96) of the S slot (token j at 32 + j / 2).  Half 0
+                // covers tokens 0-63 and writes columns 32-63, which only it reads
+                // (S columns 0-63); half 1 covers tokens 64-127 and writes 64-95
+                // (inside its S columns 64-127).  The 16-token pieces go in an
+                // order in which every write lands on S values already consumed.
+                const uint32_t tS = tmem + lane_off + kColS + s * 128;
+#pragma unroll 1
+                for (int t = 0; t < 4; ++t) {
+                    // half 0: tokens 48, 32, 16, 0; half 1: 64, 80, 96, 112
+                    const int j0 = hf == 0 ? 48 - 16 * t : 64 + 16 * t;
+                    const int jb = j0 >> 5;
+                    float sv[16];
+                    if (jb <= g) {
+                        tmem_ld16(tS + j0, sv);
+                        tmem_wait_ld();
+                    }
+                    build_p16(tS + kColP, j0, jb, g, row, acs2, misc->acs2[s], sv);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&misc->p_full[s]);
+
+                // ---- Q'_i = 2^(acs_i) q_i, in place (the S MMA of this chunk is done)
+                scale_half_row_inplace(sQ, row, hf, ex2_approx(acs2));
+            }
+
+            // ---- carried state: h_{c-1} (bf16, for Y) and own h_c; this warp does
+            //      columns [32 hf, 32 hf + 32) of rows m = 16g + lane (lane < 16)
+            bad = (c >= 1) && !mbar_wait_abortable(&misc->u_full[s ^ 1], ((c - 1) >> 1) & 1, abort_flag);
+            bad = bad || !mbar_wait_abortable(&misc->u_full[s], k & 1, abort_flag);
+            if (named_bar_any(bar_id, kGroupThreads, bad)) {
+                if (wt == 0) raise_timeout(misc, status, 34 + s);
+                break;
+            }
+            tc_fence_after();
+            {
+                const float dp = ex2_approx(lam2_prev), dc = ex2_approx(lam2);
+                const float2 dprev = make_float2(dp, dp), dcur = make_float2(dc, dc);
+                const uint32_t tUo = tmem + lane_off + kColU + (s ^ 1) * 64 + hf * 32;
+                const uint32_t tUs = tmem + lane_off + kColU + s * 64 + hf * 32;
+                uint8_t *sH = smem + kOffHs + s * (kD * kD * 2);
+                const int m = g * 16 + lane;  // state row (valid for lane < 16)
+#pragma unroll
+                for (int qt = 0; qt < 2; ++qt) {
+                    float uo[16], us[16];
+                    if (c >= 1) tmem_ld16(tUo + qt * 16, uo);
+                    tmem_ld16(tUs + qt * 16, us);
+                    tmem_wait_ld();
+                    if (lane < 16) {
+                        const int col0 = hf * 32 + qt * 16;
+                        uint32_t hb[8];
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            float4 *hp4 = reinterpret_cast<float4 *>(hown + m * kHRow + col0 + e4 * 4);
+                            const float4 hv = *hp4;
+                            float2 h0 = make_float2(0.0f, 0.0f), h1 = h0;
+                            if (c >= 1) {
+                                h0 = __ffma2_rn(dprev, make_float2(hv.x, hv.y),
+                                                make_float2(uo[e4 * 4], uo[e4 * 4 + 1]));
+                                h1 = __ffma2_rn(dprev, make_float2(hv.z, hv.w),
+                                                make_float2(uo[e4 * 4 + 2], uo[e4 * 4 + 3]));
+                            }
+                            hb[e4 * 2] = f2_to_bf2(h0);
+                            hb[e4 * 2 + 1] = f2_to_bf2(h1);
+                            const float2 n0 = __ffma2_rn(dcur, h0, make_float2(us[e4 * 4], us[e4 * 4 + 1]));
+                            const float2 n1 = __ffma2_rn(dcur, h1, make_float2(us[e4 * 4 + 2], us[e4 * 4 + 3]));
+                            *hp4 = make_float4(n0.x, n0.y, n1.x, n1.y);
+                        }
+                        if (own && c >= 1) {
+                            *reinterpret_cast<uint4 *>(sH + sw128_chunk(m, col0 / 8)) =
+                                make_uint4(hb[0], hb[1], hb[2], hb[3]);
+                            *reinterpret_cast<uint4 *>(sH + sw128_chunk(m, col0 / 8 + 1)) =
+                                make_uint4(hb[4], hb[5], hb[6], hb[7]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            mbar_arrive(&misc->u_free[s]);
+            if (c >= 1) mbar_arrive(&misc->u_free[s ^ 1]);
+            if (!own) {
+                // state-only chunk: U_c has been read (u_full), so the stage is free
+                mbar_arrive(&misc->stage_empty[st]);
                 continue;
             }
-            float sv[32];
-            tmem_ld32(tmem + t_lane + kColS + jb * 32, sv);
-            tmem_wait_ld();
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-                const int j = jb * 32 + u;
-                const float p = (j <= tid) ? sv[u] * exp2f(acs2 - misc->acs2[j]) : 0.0f;
-                sv[u] = p;
-                rowsum += p;
+            mbar_arrive(&misc->hs_full[s]);
+
+            // ---- epilogue: y = Y [+ D v], bf16, 16-byte stores straight to HBM
+            bad = !mbar_wait_abortable(&misc->y_full[s], ko & 1, abort_flag);
+            if (named_bar_any(bar_id, kGroupThreads, bad)) {
+                if (wt == 0) raise_timeout(misc, status, 36 + s);
+                break;
             }
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-                *reinterpret_cast<uint4 *>(pblk + sw128_chunk(tid, (jb & 1) * 4 + q4)) =
-                    pack8(sv + q4 * 8);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
             tc_fence_after();
-            // Y = P V  (M = 128, N = 64, K = 128 tokens)
+            {
+                float y0[16], y1[16];
+                tmem_ld16(tmem + lane_off + kColY + s * 64 + hf * 32, y0);
+                tmem_ld16(tmem + lane_off + kColY + s * 64 + hf * 32 + 16, y1);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&misc->y_free[s]);
+                const float4 *Dh = reinterpret_cast<const float4 *>(sD);
+                uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)(row0 + c * kC + row) * kD + hf * 32);
 #pragma unroll
-            for (int ks = 0; ks < kC / 16; ++ks)
-                mma_bf16(tmem + kColY, desc_k(sbase + kOffP + (ks >> 2) * kTileBytes + (ks & 3) * 32),
-                         desc_mn(aV + ks * 2048), idesc_Y, ks > 0);
-            mma_commit(&misc->bar_mma);
-        }
-
-        // ---- normaliser: q_i . z_{c-1}, then z_c = exp(lam) z_{c-1} + sum_j w_j k_j (fp32)
-        float qz = 0.0f;
-        if (normalize) {
-            if (c > 0) {
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int ch = hf * 4 + q4;
+                    const float *yy = q4 < 2 ? (y0 + q4 * 8) : (y1 + (q4 - 2) * 8);
+                    uint32_t w[4];
+                    if (Dres) {
+                        const uint4 vv = *reinterpret_cast<const uint4 *>(sV + sw128_chunk(row, ch));
+                        const float4 d0 = Dh[2 * ch], d1 = Dh[2 * ch + 1];
+                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
+                        const float2 dd[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                                              make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float f[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(sQ + sw128_chunk(tid, ch)), f);
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = f2_to_bf2(__ffma2_rn(dd[e], bf2_to_f2(vw[e]),
+                                                        make_float2(yy[2 * e], yy[2 * e + 1])));
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) qz = fmaf(f[e], misc->z[ch * 8 + e], qz);
+                        for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(yy[2 * e], yy[2 * e + 1]);
+                    }
+                    dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
                 }
+                mbar_arrive(&misc->stage_empty[st]);  // this thread is done with the stage
             }
-            __syncthreads();
-            if (tid < kD) {
-                float s = 0.0f;
-                for (int j = 0; j < kC; ++j) {
-                    const uint16_t kb =
-                        *reinterpret_cast<const uint16_t *>(sK + sw128_offset(j, tid));
-                    s = fmaf(exp2f(lam2 - misc->acs2[j]), __uint_as_float((uint32_t)kb << 16), s);
-                }
-                misc->z[tid] = fmaf(exp2f(lam2), misc->z[tid], s);
-            }
-        }
-
-        // ---- epilogue
-        if (!mbar_wait_bounded(&misc->bar_mma, c & 1)) record_timeout(status, 3, misc);
-        tc_fence_after();
-        {
-            const float eoff = exp2f(acs2);
-            float y[64];
-            tmem_ld32(tmem + t_lane + kColY, *reinterpret_cast<float(*)[32]>(y));
-            tmem_ld32(tmem + t_lane + kColY + 32, *reinterpret_cast<float(*)[32]>(y + 32));
-            tmem_wait_ld();
-            if (c > 0) {
-                float yo[32];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tmem + t_lane + kColYoff + half * 32, yo);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) y[half * 32 + e] = fmaf(eoff, yo[e], y[half * 32 + e]);
-                }
-            }
-            if (normalize) {
-                const float inv = 1.0f / fmaf(eoff, qz, rowsum);
-#pragma unroll
-                for (int e = 0; e < 64; ++e) y[e] *= inv;
-            }
-            if (Dres) {
-                const float *Dh = Dres + h * kD;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    float f[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(sV + sw128_chunk(tid, ch)), f);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) y[ch * 8 + e] = fmaf(__ldg(Dh + ch * 8 + e), f[e], y[ch * 8 + e]);
-                }
-            }
-            // stage the bf16 row in the (now free) Q buffer and store the tile with TMA
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4 *>(sQ + sw128_chunk(tid, ch)) = pack8(y + ch * 8);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_2d(&tm_o, sQ, 0, row0 + c * kC);
-            bulk_commit_group();
         }
     }
 
-    if (tid == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------- host side
@@ -409,11 +544,27 @@ bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk) {
 
 size_t tc_order1_workspace(int, int, int, int, int) { return 0; }
 
+// Segments per head: enough CTAs to cover the SMs, as long as the extra
+// state-only work (segment r re-folds r earlier segments) stays small.
+int segments_per_head(int BH, int nc) {
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            sms = 148;
+    }
+    int R = 1;
+    while (R < 2 && BH * (R * 2) <= sms && nc >= R * 2 * 2) R *= 2;
+    return R;
+}
+
 int launch_tc_order1(const FwdArgs &a, const Plan &) {
+    if (a.normalize) return SSD_ERR_UNSUPPORTED;
     const uint64_t rows = (uint64_t)a.B * a.H * a.N;
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv;
     if (!make_tmap_rows64(&tq, a.q, rows, kC) || !make_tmap_rows64(&tk, a.k, rows, kC) ||
-        !make_tmap_rows64(&tv, a.v, rows, kC) || !make_tmap_rows64(&to, a.out, rows, kC))
+        !make_tmap_rows64(&tv, a.v, rows, kC))
         return SSD_ERR_CUDA;
     static bool attr_set = false;
     if (!attr_set) {
@@ -423,8 +574,10 @@ int launch_tc_order1(const FwdArgs &a, const Plan &) {
         attr_set = true;
     }
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
-    tc_order1_kernel<<<a.B * a.H, kThreads, kSmemBytes, a.stream>>>(
-        tq, tk, tv, to, a.dt_p, a.A_log, a.dt_bias, a.D, a.H, a.N, a.normalize, status);
+    const int BH = a.B * a.H;
+    const int R = segments_per_head(BH, a.N / kC);
+    tc_order1_kernel<<<BH * R, kThreads, kSmemBytes, a.stream>>>(
+        tq, tk, tv, static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log, a.dt_bias, a.D, a.H, a.N, BH, R, status);
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

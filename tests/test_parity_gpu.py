@@ -95,6 +95,17 @@ def test_single_chunk_and_one_head():
         assert rel_err(y, _oracle_full(x, order, order == 2)) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("n_chunks", [1, 2, 3, 4, 7, 15])
+def test_chunk_counts_and_segment_boundaries(n_chunks):
+    """Heads split into segments at chunk boundaries (odd and even split
+    points, one-chunk heads) give the same result as the oracle."""
+    x = inputs.make_inputs(1, 3, n_chunks * 128, 64, "bf16", seed=40 + n_chunks)
+    for residual in (True, False):
+        y = run_gpu(x, "bf16", 1, False, 128, D="inputs" if residual else None)
+        ref = _oracle_full(x, 1, False, D="inputs" if residual else None)
+        assert rel_err(y, ref) <= TOL["bf16"]
+
+
 def test_order1_normalised_with_positive_features():
     x = inputs.make_inputs(2, 2, 512, 64, "bf16", seed=4)
     for key in ("q", "k"):
