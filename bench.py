@@ -41,6 +41,22 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def max_over_ranks(value: float, device="cpu") -> float:
+    """The largest `value` over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_rate(units_per_rank: float, steps: int, world: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank processes `units_per_rank` per step;
+    the job's time is the slowest rank's."""
+    return world * units_per_rank * steps / (total_ms / 1e3)
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -288,11 +304,7 @@ def main():
     if world > 1:
         dist.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev_name)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev_name)
     status = ssd.ssd_status_from_workspace(ws)
 
     # end to end: pinned host inputs -> device -> ssd_fwd -> host, per step
@@ -322,11 +334,8 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev_name)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item())
-        e2e = {"value": world * w.tokens * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev_name)
+        e2e = {"value": weak_scaling_rate(w.tokens, args.steps, world, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     if world > 1:
@@ -346,7 +355,7 @@ def main():
         bound, achieved, peak, unit = "tensor", tflops, float(peaks["bf16_tflops"]), "TFLOP/s"
     line = {
         "metric": METRIC,
-        "value": world * w.tokens * args.steps / (total_ms / 1e3),
+        "value": weak_scaling_rate(w.tokens, args.steps, world, total_ms),
         "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": mean_ms,

@@ -287,6 +287,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
         "r"(v[15])
         : "memory");
 }
+// 32 lanes x 1 32-bit column.
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return __uint_as_float(r);
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr),
+                 "r"(__float_as_uint(v))
+                 : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -304,6 +315,14 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
 // Byte offset of the 16-byte chunk `ch` (elements 8ch..8ch+7) of `row`.
 __device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t ch) {
     return row * 128u + (((ch ^ (row & 7u)) & 7u) << 4);
+}
+// The same for tiles with 64-byte rows (64-byte swizzle: chunk ^= (row / 2) % 4)
+// and 32-byte rows (32-byte swizzle: chunk ^= (row / 4) % 2).
+__device__ __forceinline__ uint32_t sw64_chunk(uint32_t row, uint32_t ch) {
+    return row * 64u + (((ch ^ (row >> 1)) & 3u) << 4);
+}
+__device__ __forceinline__ uint32_t sw32_chunk(uint32_t row, uint32_t ch) {
+    return row * 32u + (((ch ^ (row >> 2)) & 1u) << 4);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -85,6 +85,8 @@ def test_path_selection(lib):
     assert path == "simt" and n == 4
     path, n = ssd.ssd_fwd_path(4, 16, 2048, 64, ssd.SSD_BF16, 1, 128)
     assert path == "tc_order1" and n == 1
+    path, n = ssd.ssd_fwd_path(4, 16, 4096, 32, ssd.SSD_BF16, 2, 64)
+    assert path == "tc_order2" and n == 1
     with pytest.raises(ValueError):
         ssd.ssd_fwd_path(1, 2, 250, 16, ssd.SSD_F32, 1, 64)
 
