@@ -33,6 +33,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "ptx.cuh"
 #include "ssd_internal.h"
 
@@ -566,12 +568,15 @@ int launch_tc_order1(const FwdArgs &a, const Plan &) {
     if (!make_tmap_rows64(&tq, a.q, rows, kC) || !make_tmap_rows64(&tk, a.k, rows, kC) ||
         !make_tmap_rows64(&tv, a.v, rows, kC))
         return SSD_ERR_CUDA;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static std::atomic<uint64_t> attr_set{0};  // one bit per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
         if (cudaFuncSetAttribute(tc_order1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kSmemBytes) != cudaSuccess)
             return SSD_ERR_CUDA;
-        attr_set = true;
+        attr_set.fetch_or(bit);
     }
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
     const int BH = a.B * a.H;

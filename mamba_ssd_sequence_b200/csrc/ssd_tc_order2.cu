@@ -1,30 +1,37 @@
 // Order-2 (2Mamba, squared scores) tensor-core path (tcgen05 + TMEM, TMA) of
-// the SSD forward operator for bf16 inputs, d_h = 32, chunk = 64.
+// the SSD forward operator for bf16 inputs, d_h in {32, 64}, chunk = 64.
 //
 // Order 2 squares the score: w_ij = (q_i . k_j)^2 2^(acs_i - acs_j), whose
 // recurrent form (2Mamba2Furious, Algorithm 6) carries the state
 // h = sum_j 2^(A_t - A_j) (k_j (x) k_j) v_j^T of d_h^2 x d_h values, plus the
-// normaliser state z = sum_j 2^(A_t - A_j) (k_j (x) k_j).  One CTA per
-// (batch, head) keeps h and z in tensor memory (fp32) and walks the chunks
-// in order.  Per chunk of C = 64 tokens:
+// normaliser state z = sum_j 2^(A_t - A_j) (k_j (x) k_j).  The state of one
+// head does not fit one SM at d_h = 64 (1 MiB), so a thread-block cluster of
+// R = d_h^2 / 512 CTAs shares a head: CTA r keeps feature rows
+// [512 r, 512 r + 512) of h and z in tensor memory (fp32) -- feature (a, b)
+// is row a d_h + b -- and the cluster walks the chunks together.  Per chunk
+// of C = 64 tokens, every CTA:
 //   acs_t = chunk-local inclusive cumsum of A dt (log2 units)   (kernel (a), fused)
 //   S     = Q K^T                                      tcgen05 (M = 64)
 //   P_ij  = S_ij^2 2^(acs_i - acs_j) [i >= j],  r_i = sum_j P_ij   CUDA cores
 //   Y     = P V                                        tcgen05
-//   then, over the state's feature rows in slabs of 128 (feature (a, b) = a d + b):
+//   over its 4 slabs of 128 feature rows:
 //     hb    = bf16(h_slab)  (the state entering the chunk); h_slab *= 2^lam
 //     Fk    = [w_j k_ja k_jb]_{j, (a,b)},  w_j = 2^(lam - acs_j)
 //     Fq    = [2^acs_i q_ia q_ib]_{i, (a,b)}
 //     h_slab += Fk^T V,   z_slab += Fk^T 1             tcgen05 (M = 128)
-//     Y     += Fq hb,     n_off += Fq zb               tcgen05 (M = 64)
-//   y_i = Y_i / (r_i + n_off_i) [+ D v_i]             epilogue
-// The (q . k)^2 of the intra-chunk part is the same inner product as
+//     T     += Fq hb,     Tn += Fq zb                  tcgen05 (M = 64)
+// The cluster then sums the partial T, Tn of its CTAs through distributed
+// shared memory: CTA r owns rows [64 r / R, 64 (r + 1) / R) of the chunk and
+// writes y_i = (Y_i + sum T_i) / (r_i + sum Tn_i) [+ D v_i].  The
+// (q . k)^2 of the intra-chunk part is the same inner product as
 // (q (x) q) . (k (x) k) of the feature form (Algorithm 5 vs Algorithm 6).
-// All exponentials are of non-positive arguments.
+// All exponentials are of non-positive arguments.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 #include "ptx.cuh"
 #include "ssd_internal.h"
@@ -34,47 +41,58 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kC = 64;                  // chunk length
-constexpr int kD = 32;                  // head dim
-constexpr int kF = kD * kD;             // feature rows of the state (1024)
-constexpr int kSlab = 128;              // feature rows per slab (one M = 128 tile)
-constexpr int kSlabs = kF / kSlab;      // 8
-constexpr int kStages = 4;
-constexpr int kThreads = 192;           // warp 0: TMA, warp 1: TMEM owner, warps 2-5: compute
-constexpr uint32_t kTile = kC * kD * 2;          // 4 KiB: 64 rows x 64 B (64-byte swizzle)
-constexpr uint32_t kStageBytes = 3 * kTile;
-
-// shared memory map (1024-aligned pieces)
-constexpr uint32_t kOffStage = 0;
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;     // 64 x 64 bf16, 128B swizzle
-constexpr uint32_t kOffFk = kOffP + 8192;                          // 2 x 16 KiB
-constexpr uint32_t kOffFq = kOffFk + 2 * 16384;                    // 2 x 16 KiB
-constexpr uint32_t kOffHb = kOffFq + 2 * 16384;                    // 2 x 128 x 64 B (64B swizzle)
-constexpr uint32_t kOffZb = kOffHb + 2 * 8192;                     // 2 x 128 x 32 B (32B swizzle)
-constexpr uint32_t kOffOnes = kOffZb + 2 * 4096;                   // 64 x 32 B (32B swizzle)
-constexpr uint32_t kOffMisc = kOffOnes + 2048;
-constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;
-
-// TMEM columns
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColH = 0;                     // 8 slabs x 32: h (M = 128)
-constexpr uint32_t kColZ = kColH + kSlabs * kD;   // 8 slabs x 16: z (column 0 used)
-constexpr uint32_t kColS = kColZ + kSlabs * 16;   // 64: S (M = 64)
-constexpr uint32_t kColY = kColS + 64;            // 32: Y (M = 64)
-constexpr uint32_t kColN = kColY + kD;            // 16: normaliser off-chunk term (M = 64)
-static_assert(kColN + 16 <= kTmemCols, "TMEM budget");
-
+constexpr int kC = 64;          // chunk length
+constexpr int kFs = 512;        // feature rows per CTA
+constexpr int kSlab = 128;      // feature rows per slab (one M = 128 tile)
+constexpr int kNs = kFs / kSlab;
+constexpr int kStages = 2;
+constexpr int kTeam = 256;      // compute threads: warps 2-9
+constexpr int kThreads = 64 + kTeam;
+constexpr uint32_t kSw128 = 2, kSw64 = 4, kSw32 = 6;  // descriptor swizzle modes
 constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+    static constexpr int R = D * D / kFs;              // CTAs per head
+    static constexpr int ROWS = kC / R;                // output rows owned per CTA
+    static constexpr uint32_t RB = D * 2;              // bytes per bf16 row of q/k/v/hb
+    static constexpr uint32_t SW = RB == 128 ? kSw128 : kSw64;
+    static constexpr uint32_t SBO = 8 * RB;            // 8-row swizzle atom
+    static constexpr uint32_t TILE = kC * RB;          // q/k/v tile
+    static constexpr uint32_t STAGE = 3 * TILE;
+    static constexpr int PR = D + 4;                   // padded row (floats) of a partial
+    // shared memory map
+    static constexpr uint32_t OFF_STAGE = 0;
+    static constexpr uint32_t OFF_P = OFF_STAGE + kStages * STAGE;       // 64 x 64 bf16
+    static constexpr uint32_t OFF_FK = OFF_P + 8192;                      // 2 x 16 KiB
+    static constexpr uint32_t OFF_FQ = OFF_FK + 2 * 16384;                // 2 x 16 KiB
+    static constexpr uint32_t OFF_HB = OFF_FQ + 2 * 16384;                // 2 x 128 rows
+    static constexpr uint32_t OFF_ZB = OFF_HB + 2 * kSlab * RB;           // 2 x 128 x 32 B
+    static constexpr uint32_t OFF_ONES = OFF_ZB + 2 * 4096;               // 64 x 32 B
+    static constexpr uint32_t OFF_PART = OFF_ONES + 2048;                 // 2 x 64 x PR fp32
+    static constexpr uint32_t OFF_RES = OFF_PART + 2 * kC * PR * 4;       // ROWS x PR fp32
+    static constexpr uint32_t OFF_MISC = (OFF_RES + ROWS * PR * 4 + 1023) / 1024 * 1024;
+    static constexpr uint32_t SMEM = OFF_MISC + 2048 + 1024;
+    // tensor memory columns
+    static constexpr uint32_t COL_H = 0;                   // kNs x D   h    (M = 128)
+    static constexpr uint32_t COL_Z = COL_H + kNs * D;     // kNs x 16  z    (M = 128)
+    static constexpr uint32_t COL_S = COL_Z + kNs * 16;    // 64: S, then Y = P V (M = 64)
+    static constexpr uint32_t COL_T = COL_S + 64;          // D: partial state readout (M = 64)
+    static constexpr uint32_t COL_TN = COL_T + D;          // 16: partial normaliser (M = 64)
+    static_assert(COL_TN + 16 <= 512, "TMEM budget");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
 
 struct Misc {
     float acs2[kC];
-    float rsum[kC];
-    float Dh[kD];
+    float rsum[2][kC];
+    float Dh[64];
     float wtot[2];
-    uint64_t stage_full[kStages];
-    uint64_t stage_empty[kStages];
-    uint64_t mma_bar;
-    uint64_t slab_bar[2];
+    uint64_t stage_full[kStages], stage_empty[kStages];
+    uint64_t s_full, p_full, y_free, chunk_done;
+    uint64_t slab_full[2], slab_done[2];
+    uint64_t ready[2], consumed[2];
+    uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -86,8 +104,14 @@ __device__ __forceinline__ float softplus_f(float x) {
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
-// swizzle modes of the tcgen05 shared-memory descriptor
-constexpr uint32_t kSw128 = 2, kSw64 = 4, kSw32 = 6;
+__device__ __forceinline__ float bf16_at(const uint8_t *p) {
+    return __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(p) << 16);
+}
+template <uint32_t RB>
+__device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t ch) {
+    if constexpr (RB == 128) return sw128_chunk(row, ch);
+    else return sw64_chunk(row, ch);
+}
 
 __device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
     if (status) {
@@ -97,26 +121,29 @@ __device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
     *reinterpret_cast<volatile int *>(&misc->abort_flag) = 1;
 }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                  const float *__restrict__ dt_p, const float *__restrict__ A_log,
                  const float *__restrict__ dt_bias, const float *__restrict__ Dres, int H, int N,
                  int normalize, DeviceStatus *status) {
+    using K = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Misc *misc = reinterpret_cast<Misc *>(smem + kOffMisc);
+    Misc *misc = reinterpret_cast<Misc *>(smem + K::OFF_MISC);
     const volatile int *abort_flag = &misc->abort_flag;
     const uint32_t sbase = smem_u32(smem);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x, h = bh % H;
+    const uint32_t rank = cluster_ctarank();
+    const int bh = blockIdx.x / K::R, h = bh % H;
     const int nc = N / kC;
     const int row0 = bh * N;
 
     if (tid == 0) {
-        if (bh == 0 && status) {
+        if (blockIdx.x == 0 && status) {
             status->code = 0;
             status->detail = 0;
         }
@@ -124,26 +151,34 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_init(&misc->stage_full[i], 1);
             mbar_init(&misc->stage_empty[i], 1);
         }
-        mbar_init(&misc->mma_bar, 1);
-        mbar_init(&misc->slab_bar[0], 1);
-        mbar_init(&misc->slab_bar[1], 1);
+        mbar_init(&misc->s_full, 1);
+        mbar_init(&misc->p_full, kTeam);
+        mbar_init(&misc->y_free, kTeam);
+        mbar_init(&misc->chunk_done, 1);
+        mbar_init(&misc->drain, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&misc->slab_full[b], kTeam);
+            mbar_init(&misc->slab_done[b], 1);
+            mbar_init(&misc->ready[b], K::R);
+            mbar_init(&misc->consumed[b], K::R);
+        }
         misc->abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&misc->tmem_base, kTmemCols);
+        tmem_alloc(&misc->tmem_base, 512);
         tmem_relinquish();
     }
-    // constant B operand [1, 0, ..., 0] per token (64 rows x 16 bf16, 32B swizzle)
+    // constant B operand: [1, 0, ..., 0] per token (64 rows x 16 bf16, 32B swizzle)
     for (int i = tid; i < kC * 2; i += kThreads) {
         const int r = i >> 1, ch = i & 1;
-        const uint32_t one = ch == 0 ? 0x3F80u : 0u;  // bf16 1.0 in the first element
-        *reinterpret_cast<uint4 *>(smem + kOffOnes + sw32_chunk(r, ch)) = make_uint4(one, 0, 0, 0);
+        *reinterpret_cast<uint4 *>(smem + K::OFF_ONES + sw32_chunk(r, ch)) =
+            make_uint4(ch == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
     }
-    if (tid < kD) misc->Dh[tid] = Dres ? Dres[h * kD + tid] : 0.0f;
+    if (tid < D) misc->Dh[tid] = Dres ? Dres[h * D + tid] : 0.0f;
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // every CTA's barriers exist before any remote arrive
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
 
@@ -153,6 +188,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
+            int issued = 0;
             for (int c = 0; c < nc; ++c) {
                 const int st = c % kStages;
                 if (c >= kStages &&
@@ -160,49 +196,122 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     raise_timeout(misc, status, 10);
                     break;
                 }
-                uint8_t *dst = smem + kOffStage + st * kStageBytes;
+                uint8_t *dst = smem + K::OFF_STAGE + st * K::STAGE;
                 const int r = row0 + c * kC;
-                mbar_arrive_expect_tx(&misc->stage_full[st], kStageBytes);
+                mbar_arrive_expect_tx(&misc->stage_full[st], K::STAGE);
                 tma_load_2d(dst, &tm_q, 0, r, &misc->stage_full[st]);
-                tma_load_2d(dst + kTile, &tm_k, 0, r, &misc->stage_full[st]);
-                tma_load_2d(dst + 2 * kTile, &tm_v, 0, r, &misc->stage_full[st]);
+                tma_load_2d(dst + K::TILE, &tm_k, 0, r, &misc->stage_full[st]);
+                tma_load_2d(dst + 2 * K::TILE, &tm_v, 0, r, &misc->stage_full[st]);
+                ++issued;
+            }
+            // copies still in flight after an abort land before the CTA exits (bounded)
+            for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+                mbar_wait_bounded(&misc->stage_full[c % kStages], (c / kStages) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idS = make_idesc_bf16(64, 64, 0, 0);
+            constexpr uint32_t idPV = make_idesc_bf16(64, D, 0, 1);
+            constexpr uint32_t idU = make_idesc_bf16(128, D, 1, 1);
+            constexpr uint32_t idZ = make_idesc_bf16(128, 16, 1, 1);
+            constexpr uint32_t idT = make_idesc_bf16(64, D, 0, 1);
+            constexpr uint32_t idTn = make_idesc_bf16(64, 16, 0, 1);
+            uint32_t slab_uses[2] = {0, 0};
+            bool ok = true;
+            for (int c = 0; ok && c < nc; ++c) {
+                const int st = c % kStages;
+                const uint32_t aQ = sbase + K::OFF_STAGE + st * K::STAGE;
+                const uint32_t aK = aQ + K::TILE, aV = aK + K::TILE;
+                if (!(ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag))) break;
+                if (c >= 1 && !(ok = mbar_wait_abortable(&misc->y_free, (c - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    mma_bf16(tmem + K::COL_S, make_sdesc(aQ + ks * 32, 16, K::SBO, K::SW),
+                             make_sdesc(aK + ks * 32, 16, K::SBO, K::SW), idS, ks > 0);
+                mma_commit(&misc->s_full);
+                if (!(ok = mbar_wait_abortable(&misc->p_full, c & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < kC / 16; ++ks)
+                    mma_bf16(tmem + K::COL_S, make_sdesc(sbase + K::OFF_P + ks * 32, 16, 1024, kSw128),
+                             make_sdesc(aV + ks * 16 * K::RB, 16, K::SBO, K::SW), idPV, ks > 0);
+                for (int sl = 0; sl < kNs; ++sl) {
+                    const int b = sl & 1;
+                    if (!(ok = mbar_wait_abortable(&misc->slab_full[b], slab_uses[b] & 1, abort_flag))) break;
+                    ++slab_uses[b];
+                    tc_fence_after();
+                    const uint32_t fkA = sbase + K::OFF_FK + b * 16384;
+                    const uint32_t fqA = sbase + K::OFF_FQ + b * 16384;
+                    // h_slab += Fk^T V  (A: features x tokens, MN-major, two 64-feature groups)
+#pragma unroll
+                    for (int ks = 0; ks < kC / 16; ++ks)
+                        mma_bf16(tmem + K::COL_H + sl * D, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
+                                 make_sdesc(aV + ks * 16 * K::RB, 16, K::SBO, K::SW), idU, (c > 0 || ks > 0));
+                    if (normalize) {
+#pragma unroll
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            mma_bf16(tmem + K::COL_Z + sl * 16, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
+                                     make_sdesc(sbase + K::OFF_ONES + ks * 512, 16, 256, kSw32), idZ,
+                                     (c > 0 || ks > 0));
+                    }
+                    if (c >= 1) {
+                        // T += Fq hb ;  Tn += Fq zb   (A: tokens x features, K-major)
+                        const uint32_t hbB = sbase + K::OFF_HB + b * kSlab * K::RB;
+                        const uint32_t zbB = sbase + K::OFF_ZB + b * 4096;
+#pragma unroll
+                        for (int ks = 0; ks < kSlab / 16; ++ks) {
+                            const uint64_t adesc =
+                                make_sdesc(fqA + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128);
+                            mma_bf16(tmem + K::COL_T, adesc, make_sdesc(hbB + ks * 16 * K::RB, 16, K::SBO, K::SW),
+                                     idT, (sl > 0 || ks > 0));
+                            if (normalize)
+                                mma_bf16(tmem + K::COL_TN, adesc, make_sdesc(zbB + ks * 512, 16, 256, kSw32), idTn,
+                                         (sl > 0 || ks > 0));
+                        }
+                    }
+                    mma_commit(&misc->slab_done[b]);
+                }
+                if (!ok) break;
+                mma_commit(&misc->chunk_done);
+            }
+            if (!ok) {
+                raise_timeout(misc, status, 20);
+                // matrix products still in flight finish before TMEM is released (bounded)
+                mma_commit(&misc->drain);
+                mbar_wait_bounded(&misc->drain, 0);
             }
         }
-    } else if (warp >= 2) {
-        // ------------------------------------------------------ compute group
-        const int ct = tid - 64;                  // 0..127
-        const int g = warp & 3;                   // TMEM lane quarter
+    } else {
+        // ------------------------------------------------------ compute team
+        const int ct = tid - 64;                    // 0..255
+        const int g = warp & 3;                     // TMEM lane quarter
+        const int hf = (warp - 2) >> 2;             // which half of the columns
         const uint32_t lane_off = (uint32_t)(g * 32) << 16;
-        const int frow = g * 32 + lane;           // feature row of a slab (M = 128 layout)
-        const int mrow = g * 16 + lane;           // chunk row in the M = 64 layout (lane < 16)
+        const int frow = g * 32 + lane;             // feature row of a slab (M = 128 layout)
+        const int mrow = g * 16 + lane;             // chunk row (M = 64 layout, lane < 16)
         const bool mrow_ok = lane < 16;
+        const bool own_row = mrow_ok && mrow / K::ROWS == (int)rank;
         const float A2 = -expf(A_log[h]) * kLog2e;
         const float bias = dt_bias[h];
         const bool elected = ct == 0;
-
-        constexpr uint32_t idS = make_idesc_bf16(64, 64, 0, 0);
-        constexpr uint32_t idPV = make_idesc_bf16(64, kD, 0, 1);
-        constexpr uint32_t idU = make_idesc_bf16(128, kD, 1, 1);
-        constexpr uint32_t idZ = make_idesc_bf16(128, 16, 1, 1);
-        constexpr uint32_t idT = make_idesc_bf16(64, kD, 0, 1);
-        constexpr uint32_t idTz = make_idesc_bf16(64, 16, 0, 1);
-
-        uint32_t mma_uses = 0, slab_uses[2] = {0, 0};
-        auto wait_mma = [&](uint64_t *bar, uint32_t uses) -> bool {
-            return mbar_wait_abortable(bar, (uses - 1) & 1, abort_flag);
-        };
+        const int tok = ct & 63, q4 = ct >> 6;      // feature generation: token, 32-feature part
+        uint32_t slab_uses[2] = {0, 0};
+        float *part0 = reinterpret_cast<float *>(smem + K::OFF_PART);
+        float *res = reinterpret_cast<float *>(smem + K::OFF_RES);
 
         float dt_next = (ct < kC && nc > 0) ? dt_p[(size_t)row0 + ct] : 0.0f;
         for (int c = 0; c < nc; ++c) {
             const int st = c % kStages;
-            uint8_t *sQ = smem + kOffStage + st * kStageBytes;
-            uint8_t *sK = sQ + kTile;
-            uint8_t *sV = sK + kTile;
-            const uint32_t aQ = smem_u32(sQ), aK = aQ + kTile, aV = aK + kTile;
+            uint8_t *sQ = smem + K::OFF_STAGE + st * K::STAGE;
+            uint8_t *sK = sQ + K::TILE;
+            uint8_t *sV = sK + K::TILE;
             const float dtv = dt_next;
             if (ct < kC && c + 1 < nc) dt_next = dt_p[(size_t)row0 + (size_t)(c + 1) * kC + ct];
 
-            // ---- decay (tokens 0..63 on threads 0..63: warps 2 and 3)
+            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
+            // ---- decay (tokens 0..63 on threads 0..63)
             float a = 0.0f;
             if (ct < kC) {
                 a = A2 * softplus_f(dtv + bias);
@@ -213,258 +322,257 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 if (lane == 31) misc->wtot[ct >> 5] = a;
             }
-            named_bar_sync(1, 128);
+            if (named_bar_any(1, kTeam, bad)) {
+                if (elected) raise_timeout(misc, status, 30);
+                break;
+            }
             if (ct >= 32 && ct < kC) a += misc->wtot[0];
             if (ct < kC) misc->acs2[ct] = a;
             const float lam2 = misc->wtot[0] + misc->wtot[1];
 
-            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
-            if (named_bar_any(1, 128, bad)) {
-                if (elected) raise_timeout(misc, status, 30);
-                break;
-            }
-            // ---- S = Q K^T
-            if (elected) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks)
-                    mma_bf16(tmem + kColS, make_sdesc(aQ + ks * 32, 16, 512, kSw64),
-                             make_sdesc(aK + ks * 32, 16, 512, kSw64), idS, ks > 0);
-                mma_commit(&misc->mma_bar);
-            }
-            ++mma_uses;
-            bad = !wait_mma(&misc->mma_bar, mma_uses);
-            if (named_bar_any(1, 128, bad)) {
+            // ---- P = S^2 2^(acs_i - acs_j) [i >= j]: row mrow, columns [32 hf, 32 hf + 32)
+            bad = !mbar_wait_abortable(&misc->s_full, c & 1, abort_flag);
+            if (named_bar_any(1, kTeam, bad)) {  // also publishes acs2[]
                 if (elected) raise_timeout(misc, status, 31);
                 break;
             }
             tc_fence_after();
-
-            // ---- P = S^2 2^(acs_i - acs_j) [i >= j] (rows of the M = 64 layout), row sums
             {
                 float sv[32];
-                float rs = 0.0f;
-                const float ai = misc->acs2[mrow & 63];
+                tmem_ld32(tmem + lane_off + K::COL_S + hf * 32, sv);
+                tmem_wait_ld();
+                if (own_row) {  // rows of other CTAs are never read back from Y
+                    const float ai = misc->acs2[mrow];
+                    float rs = 0.0f;
+                    uint32_t pk[16];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(tmem + lane_off + kColS + half * 32, sv);
-                    tmem_wait_ld();
-                    if (mrow_ok) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const int j = half * 32 + e;
-                            float p0 = sv[e] * sv[e] * ex2_approx(ai - misc->acs2[j]);
-                            float p1 = sv[e + 1] * sv[e + 1] * ex2_approx(ai - misc->acs2[j + 1]);
-                            if (j > mrow) p0 = 0.0f;
-                            if (j + 1 > mrow) p1 = 0.0f;
-                            rs += p0 + p1;
-                            pk[e >> 1] = pack_bf16x2(p0, p1);
-                        }
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4)
-                            *reinterpret_cast<uint4 *>(smem + kOffP + sw128_chunk(mrow, half * 4 + q4)) =
-                                make_uint4(pk[q4 * 4], pk[q4 * 4 + 1], pk[q4 * 4 + 2], pk[q4 * 4 + 3]);
+                    for (int e = 0; e < 32; e += 2) {
+                        const int j = hf * 32 + e;
+                        float p0 = sv[e] * sv[e] * ex2_approx(ai - misc->acs2[j]);
+                        float p1 = sv[e + 1] * sv[e + 1] * ex2_approx(ai - misc->acs2[j + 1]);
+                        if (j > mrow) p0 = 0.0f;
+                        if (j + 1 > mrow) p1 = 0.0f;
+                        rs += p0 + p1;
+                        pk[e >> 1] = pack_bf16x2(p0, p1);
                     }
-                }
-                if (mrow_ok) misc->rsum[mrow] = rs;
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(1, 128);
-            // ---- Y = P V
-            if (elected) {
-                tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_bf16(tmem + kColY, make_sdesc(sbase + kOffP + ks * 32, 16, 1024, kSw128),
-                             make_sdesc(aV + ks * 1024, 16, 512, kSw64), idPV, ks > 0);
+                    for (int k4 = 0; k4 < 4; ++k4)
+                        *reinterpret_cast<uint4 *>(smem + K::OFF_P + sw128_chunk(mrow, hf * 4 + k4)) =
+                            make_uint4(pk[k4 * 4], pk[k4 * 4 + 1], pk[k4 * 4 + 2], pk[k4 * 4 + 3]);
+                    misc->rsum[hf][mrow] = rs;
+                }
             }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            mbar_arrive(&misc->p_full);
 
             // ---- state slabs
-            const float acs_tok = misc->acs2[ct & 63];        // token of this thread in F*
-            const float wk = ex2_approx(lam2 - acs_tok);       // w_j for F_k
-            const float sq = ex2_approx(acs_tok);              // 2^acs_i for F_q
-            const float dec = ex2_approx(lam2);                // decay of the whole chunk
-            const int tok = ct & 63, blk = ct >> 6;
-            float kr[kD], qr[kD];                              // this token's k and q rows
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                const uint4 ku = *reinterpret_cast<const uint4 *>(sK + sw64_chunk(tok, ch));
-                const uint4 qu = *reinterpret_cast<const uint4 *>(sQ + sw64_chunk(tok, ch));
-                const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 kf = bf2_to_f2(kw[e]), qf = bf2_to_f2(qw[e]);
-                    kr[ch * 8 + 2 * e] = kf.x;
-                    kr[ch * 8 + 2 * e + 1] = kf.y;
-                    qr[ch * 8 + 2 * e] = qf.x;
-                    qr[ch * 8 + 2 * e + 1] = qf.y;
-                }
-            }
-            for (int sl = 0; sl < kSlabs; ++sl) {
+            const float acs_tok = misc->acs2[tok];
+            const float wk = ex2_approx(lam2 - acs_tok);   // w_j for F_k
+            const float sqs = ex2_approx(acs_tok);         // 2^acs_i for F_q
+            const float dec = ex2_approx(lam2);            // decay over the whole chunk
+            for (int sl = 0; sl < kNs; ++sl) {
                 const int b = sl & 1;
                 if (slab_uses[b] > 0) {
-                    bad = !wait_mma(&misc->slab_bar[b], slab_uses[b]);
-                    if (named_bar_any(1, 128, bad)) {
+                    bad = !mbar_wait_abortable(&misc->slab_done[b], (slab_uses[b] - 1) & 1, abort_flag);
+                    if (named_bar_any(1, kTeam, bad)) {
                         if (elected) raise_timeout(misc, status, 32);
                         goto done;
                     }
                     tc_fence_after();
                 }
-                // h_{c-1} of this slab to bf16 (64B-swizzled rows), then h *= 2^lam; same for z
-                {
-                    float hv[32];
-                    tmem_ld32(tmem + lane_off + kColH + sl * kD, hv);
-                    float zv = normalize ? tmem_ld1(tmem + lane_off + kColZ + sl * 16) : 0.0f;
+                // h_{c-1} of this slab -> bf16, then h *= 2^lam (columns [hf D/2, hf D/2 + D/2));
+                // z likewise (column 0, half 0 only)
+                if (c >= 1) {
+                    constexpr int HC = D / 2;
+                    float hv[HC];
+                    const uint32_t ta = tmem + lane_off + K::COL_H + sl * D + hf * HC;
+                    if constexpr (HC == 32) tmem_ld32(ta, hv);
+                    else tmem_ld16(ta, hv);
+                    const float zv = (normalize && hf == 0) ? tmem_ld1(tmem + lane_off + K::COL_Z + sl * 16) : 0.0f;
                     tmem_wait_ld();
-                    if (c >= 1) {
-                        uint8_t *hb = smem + kOffHb + b * 8192;
+                    uint8_t *hb = smem + K::OFF_HB + b * kSlab * K::RB;
 #pragma unroll
-                        for (int ch = 0; ch < 4; ++ch)
-                            *reinterpret_cast<uint4 *>(hb + sw64_chunk(frow, ch)) =
-                                make_uint4(pack_bf16x2(hv[ch * 8], hv[ch * 8 + 1]),
-                                           pack_bf16x2(hv[ch * 8 + 2], hv[ch * 8 + 3]),
-                                           pack_bf16x2(hv[ch * 8 + 4], hv[ch * 8 + 5]),
-                                           pack_bf16x2(hv[ch * 8 + 6], hv[ch * 8 + 7]));
-                        if (normalize) {
-                            uint8_t *zb = smem + kOffZb + b * 4096;
-                            *reinterpret_cast<uint4 *>(zb + sw32_chunk(frow, 0)) =
-                                make_uint4(pack_bf16x2(zv, 0.0f), 0u, 0u, 0u);
-                            *reinterpret_cast<uint4 *>(zb + sw32_chunk(frow, 1)) = make_uint4(0u, 0u, 0u, 0u);
-                        }
-                        const float2 d2 = make_float2(dec, dec);
+                    for (int ch = 0; ch < HC / 8; ++ch)
+                        *reinterpret_cast<uint4 *>(hb + swz<K::RB>(frow, hf * (HC / 8) + ch)) =
+                            make_uint4(pack_bf16x2(hv[ch * 8], hv[ch * 8 + 1]),
+                                       pack_bf16x2(hv[ch * 8 + 2], hv[ch * 8 + 3]),
+                                       pack_bf16x2(hv[ch * 8 + 4], hv[ch * 8 + 5]),
+                                       pack_bf16x2(hv[ch * 8 + 6], hv[ch * 8 + 7]));
+                    const float2 d2 = make_float2(dec, dec);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float2 r2 = __fmul2_rn(make_float2(hv[e], hv[e + 1]), d2);
-                            hv[e] = r2.x;
-                            hv[e + 1] = r2.y;
-                        }
-                        tmem_st32(tmem + lane_off + kColH + sl * kD, hv);
-                        if (normalize) tmem_st1(tmem + lane_off + kColZ + sl * 16, zv * dec);
+                    for (int e = 0; e < HC; e += 2) {
+                        const float2 r2 = __fmul2_rn(make_float2(hv[e], hv[e + 1]), d2);
+                        hv[e] = r2.x;
+                        hv[e + 1] = r2.y;
+                    }
+                    if constexpr (HC == 32) tmem_st32(ta, hv);
+                    else tmem_st16(ta, hv);
+                    if (normalize && hf == 0) {
+                        uint8_t *zb = smem + K::OFF_ZB + b * 4096;
+                        *reinterpret_cast<uint4 *>(zb + sw32_chunk(frow, 0)) =
+                            make_uint4(pack_bf16x2(zv, 0.0f), 0u, 0u, 0u);
+                        *reinterpret_cast<uint4 *>(zb + sw32_chunk(frow, 1)) = make_uint4(0u, 0u, 0u, 0u);
+                        tmem_st1(tmem + lane_off + K::COL_Z + sl * 16, zv * dec);
                     }
                 }
-                // F_k and F_q: this thread writes token `tok`, 64-feature block `blk`
-                // (features (a, b) with a = 4 sl + 2 blk + {0, 1}, b = 0..31)
+                // features: token `tok`, slab-local features [32 q4, 32 q4 + 32)
                 {
-                    const int a0 = sl * 4 + blk * 2;
-                    uint8_t *fk = smem + kOffFk + b * 16384 + blk * 8192;
-                    uint8_t *fq = smem + kOffFq + b * 16384 + blk * 8192;
+                    const int fl0 = q4 * 32;
+                    const int a = (int)(rank * kFs + sl * kSlab + fl0) / D;  // first index of the pair
+                    const int b0 = (rank * kFs + sl * kSlab + fl0) % D;
+                    const float ka = bf16_at(sK + swz<K::RB>(tok, a >> 3) + (a & 7) * 2);
+                    const float qa = bf16_at(sQ + swz<K::RB>(tok, a >> 3) + (a & 7) * 2);
+                    const float2 sk2 = make_float2(wk * ka, wk * ka), sq2 = make_float2(sqs * qa, sqs * qa);
+                    uint8_t *fk = smem + K::OFF_FK + b * 16384 + (fl0 >> 6) * 8192;
+                    uint8_t *fq = smem + K::OFF_FQ + b * 16384 + (fl0 >> 6) * 8192;
 #pragma unroll
-                    for (int aa = 0; aa < 2; ++aa) {
-                        const int ai = a0 + aa;  // k_{j,a} and q_{i,a} read back from the tiles
-                        const uint32_t eo = sw64_chunk(tok, ai >> 3) + (ai & 7) * 2;
-                        const float ka = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(sK + eo) << 16);
-                        const float qa = __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(sQ + eo) << 16);
-                        const float sk = wk * ka, sqq = sq * qa;
-                        const float2 sk2 = make_float2(sk, sk), sq2 = make_float2(sqq, sqq);
+                    for (int ch = 0; ch < 4; ++ch) {
+                        const int bb = b0 + ch * 8;
+                        const uint4 ku = *reinterpret_cast<const uint4 *>(sK + swz<K::RB>(tok, bb >> 3));
+                        const uint4 qu = *reinterpret_cast<const uint4 *>(sQ + swz<K::RB>(tok, bb >> 3));
+                        const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
+                        uint32_t ok4[4], oq4[4];
 #pragma unroll
-                        for (int ch = 0; ch < 4; ++ch) {
-                            uint32_t wk4[4], wq4[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int bb = ch * 8 + 2 * e;
-                                const float2 kv = __fmul2_rn(make_float2(kr[bb], kr[bb + 1]), sk2);
-                                const float2 qv = __fmul2_rn(make_float2(qr[bb], qr[bb + 1]), sq2);
-                                wk4[e] = pack_bf16x2(kv.x, kv.y);
-                                wq4[e] = pack_bf16x2(qv.x, qv.y);
-                            }
-                            const int cidx = aa * 4 + ch;  // 16B chunk in the 128B row
-                            *reinterpret_cast<uint4 *>(fk + sw128_chunk(tok, cidx)) =
-                                make_uint4(wk4[0], wk4[1], wk4[2], wk4[3]);
-                            *reinterpret_cast<uint4 *>(fq + sw128_chunk(tok, cidx)) =
-                                make_uint4(wq4[0], wq4[1], wq4[2], wq4[3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 kv = __fmul2_rn(bf2_to_f2(kw[e]), sk2);
+                            const float2 qv = __fmul2_rn(bf2_to_f2(qw[e]), sq2);
+                            ok4[e] = pack_bf16x2(kv.x, kv.y);
+                            oq4[e] = pack_bf16x2(qv.x, qv.y);
                         }
+                        const int cidx = ((fl0 & 63) >> 3) + ch;  // 16B chunk in the 128B feature row
+                        *reinterpret_cast<uint4 *>(fk + sw128_chunk(tok, cidx)) =
+                            make_uint4(ok4[0], ok4[1], ok4[2], ok4[3]);
+                        *reinterpret_cast<uint4 *>(fq + sw128_chunk(tok, cidx)) =
+                            make_uint4(oq4[0], oq4[1], oq4[2], oq4[3]);
                     }
                 }
                 tmem_wait_st();
-                fence_proxy_async_smem();
                 tc_fence_before();
-                named_bar_sync(1, 128);
-                if (elected) {
-                    tc_fence_after();
-                    const uint32_t fkA = sbase + kOffFk + b * 16384;
-                    const uint32_t fqA = sbase + kOffFq + b * 16384;
-                    // h_slab += Fk^T V  (A: features x tokens, MN-major, two 64-feature groups)
-#pragma unroll
-                    for (int ks = 0; ks < kC / 16; ++ks)
-                        mma_bf16(tmem + kColH + sl * kD, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
-                                 make_sdesc(aV + ks * 1024, 16, 512, kSw64), idU, (c > 0 || ks > 0));
-                    if (normalize) {
-#pragma unroll
-                        for (int ks = 0; ks < kC / 16; ++ks)
-                            mma_bf16(tmem + kColZ + sl * 16, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
-                                     make_sdesc(sbase + kOffOnes + ks * 512, 16, 256, kSw32), idZ,
-                                     (c > 0 || ks > 0));
-                    }
-                    if (c >= 1) {
-                        // Y += Fq hb ;  n_off += Fq zb   (A: tokens x features, K-major)
-                        const uint32_t hbB = sbase + kOffHb + b * 8192;
-                        const uint32_t zbB = sbase + kOffZb + b * 4096;
-#pragma unroll
-                        for (int ks = 0; ks < kSlab / 16; ++ks) {
-                            const uint64_t adesc =
-                                make_sdesc(fqA + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128);
-                            mma_bf16(tmem + kColY, adesc, make_sdesc(hbB + ks * 1024, 16, 512, kSw64), idT, 1);
-                            if (normalize)
-                                mma_bf16(tmem + kColN, adesc, make_sdesc(zbB + ks * 512, 16, 256, kSw32), idTz,
-                                         (sl > 0 || ks > 0));
-                        }
-                    }
-                    mma_commit(&misc->slab_bar[b]);
-                }
+                fence_proxy_async_smem();
+                mbar_arrive(&misc->slab_full[b]);
                 ++slab_uses[b];
             }
-            // ---- all MMAs of the chunk done
-            if (elected) mma_commit(&misc->mma_bar);
-            ++mma_uses;
-            bad = !wait_mma(&misc->mma_bar, mma_uses);
-            if (named_bar_any(1, 128, bad)) {
+
+            // ---- this CTA's partial (plus Y and r on its own rows) into part[c & 1]
+            bad = !mbar_wait_abortable(&misc->chunk_done, c & 1, abort_flag);
+            bad = bad || (c >= 2 && !mbar_wait_cluster(&misc->consumed[c & 1], ((c >> 1) - 1) & 1, abort_flag));
+            if (named_bar_any(1, kTeam, bad)) {
                 if (elected) raise_timeout(misc, status, 33);
                 break;
             }
             tc_fence_after();
-
-            // ---- epilogue: y = Y / (r + n_off) [+ D v], bf16 stores (rows of the M = 64 layout)
             {
-                float yv[32];
-                tmem_ld32(tmem + lane_off + kColY, yv);
-                const float noff = (normalize && c >= 1) ? tmem_ld1(tmem + lane_off + kColN) : 0.0f;
+                constexpr int HC = D / 2;
+                float tv[HC], yv[HC];
+                const uint32_t tt = tmem + lane_off + K::COL_T + hf * HC;
+                const uint32_t ty = tmem + lane_off + K::COL_S + hf * HC;
+                if constexpr (HC == 32) {
+                    tmem_ld32(tt, tv);
+                    tmem_ld32(ty, yv);
+                } else {
+                    tmem_ld16(tt, tv);
+                    tmem_ld16(ty, yv);
+                }
+                const float tn = (normalize && hf == 0) ? tmem_ld1(tmem + lane_off + K::COL_TN) : 0.0f;
                 tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&misc->y_free);
                 if (mrow_ok) {
-                    const float inv = normalize ? 1.0f / (misc->rsum[mrow] + noff) : 1.0f;
-                    uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)(row0 + c * kC + mrow) * kD);
+                    float *prow = part0 + (c & 1) * kC * K::PR + mrow * K::PR;
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const uint4 vu = *reinterpret_cast<const uint4 *>(sV + sw64_chunk(mrow, ch));
-                        const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
-                        uint32_t w[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int cc = ch * 8 + 2 * e;
-                            float y0 = yv[cc] * inv, y1 = yv[cc + 1] * inv;
-                            if (Dres) {
-                                const float2 vf = bf2_to_f2(vw[e]);
-                                y0 = fmaf(misc->Dh[cc], vf.x, y0);
-                                y1 = fmaf(misc->Dh[cc + 1], vf.y, y1);
-                            }
-                            w[e] = pack_bf16x2(y0, y1);
+                    for (int e = 0; e < HC; e += 4) {
+                        float4 v = c >= 1 ? make_float4(tv[e], tv[e + 1], tv[e + 2], tv[e + 3])
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (own_row) {
+                            v.x += yv[e];
+                            v.y += yv[e + 1];
+                            v.z += yv[e + 2];
+                            v.w += yv[e + 3];
                         }
-                        dst[ch] = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<float4 *>(prow + hf * HC + e) = v;
+                    }
+                    if (hf == 0)
+                        prow[D] = (c >= 1 ? tn : 0.0f) +
+                                  (own_row ? misc->rsum[0][mrow] + misc->rsum[1][mrow] : 0.0f);
+                }
+            }
+            named_bar_sync(1, kTeam);
+            if (elected) {
+                fence_acq_rel_cluster();
+                const uint32_t rdy = smem_u32(&misc->ready[c & 1]);
+                for (int r2 = 0; r2 < K::R; ++r2) mbar_arrive_cluster(mapa_shared(rdy, r2));
+            }
+
+            // ---- own rows: sum the R partials (distributed shared memory), epilogue
+            bad = !mbar_wait_cluster(&misc->ready[c & 1], (c >> 1) & 1, abort_flag);
+            if (named_bar_any(1, kTeam, bad)) {
+                if (elected) raise_timeout(misc, status, 34);
+                break;
+            }
+            {
+                constexpr int NV = D / 4 + 1;  // float4 groups of a row, plus the normaliser
+                const uint32_t pb = smem_u32(part0 + (c & 1) * kC * K::PR);
+                for (int it = ct; it < K::ROWS * NV; it += kTeam) {
+                    const int rr = it / NV, v = it % NV;
+                    const int row = rank * K::ROWS + rr;
+                    const uint32_t off = (uint32_t)(row * K::PR + (v < D / 4 ? v * 4 : D)) * 4u;
+                    if (v < D / 4) {
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int r2 = 0; r2 < K::R; ++r2) {
+                            const float4 x = ld_dsmem_f4(mapa_shared(pb + off, r2));
+                            acc.x += x.x;
+                            acc.y += x.y;
+                            acc.z += x.z;
+                            acc.w += x.w;
+                        }
+                        *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc;
+                    } else {
+                        float acc = 0.0f;
+                        for (int r2 = 0; r2 < K::R; ++r2) acc += ld_dsmem_f1(mapa_shared(pb + off, r2));
+                        res[rr * K::PR + D] = acc;
                     }
                 }
             }
-            tc_fence_before();
-            named_bar_sync(1, 128);
+            named_bar_sync(1, kTeam);
+            if (elected) {
+                fence_acq_rel_cluster();
+                const uint32_t cns = smem_u32(&misc->consumed[c & 1]);
+                for (int r2 = 0; r2 < K::R; ++r2) mbar_arrive_cluster(mapa_shared(cns, r2));
+            }
+            for (int it = ct; it < K::ROWS * (D / 8); it += kTeam) {
+                const int rr = it / (D / 8), ch = it % (D / 8);
+                const int row = rank * K::ROWS + rr;
+                const float *rrow = res + rr * K::PR;
+                const float inv = normalize ? 1.0f / rrow[D] : 1.0f;
+                const uint4 vu = *reinterpret_cast<const uint4 *>(sV + swz<K::RB>(row, ch));
+                const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int cc = ch * 8 + 2 * e;
+                    float y0 = rrow[cc] * inv, y1 = rrow[cc + 1] * inv;
+                    if (Dres) {
+                        const float2 vf = bf2_to_f2(vw[e]);
+                        y0 = fmaf(misc->Dh[cc], vf.x, y0);
+                        y1 = fmaf(misc->Dh[cc + 1], vf.y, y1);
+                    }
+                    w[e] = pack_bf16x2(y0, y1);
+                }
+                *reinterpret_cast<uint4 *>(out + (size_t)(row0 + c * kC + row) * D + ch * 8) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            named_bar_sync(1, kTeam);
             if (elected) mbar_arrive(&misc->stage_empty[st]);
         }
     done:;
     }
 
+    __syncwarp();
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // no CTA leaves while another may still read its shared memory
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------- host side
@@ -481,46 +589,68 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-// [rows, 32] bf16 row-major tensor, boxes of 64 rows, 64-byte swizzle.
-bool make_tmap_rows32(CUtensorMap *m, const void *base, uint64_t rows) {
+// [rows, d] bf16 row-major tensor, boxes of 64 rows, swizzle = row bytes.
+bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, int d) {
     auto enc = get_encode_fn();
     if (!enc) return false;
-    cuuint64_t dims[2] = {kD, rows};
-    cuuint64_t strides[1] = {kD * 2};
-    cuuint32_t box[2] = {kD, kC};
+    cuuint64_t dims[2] = {(cuuint64_t)d, rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {(cuuint32_t)d, kC};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     d == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+template <int D>
+int launch_d(const FwdArgs &a) {
+    using K = Cfg<D>;
+    const uint64_t rows = (uint64_t)a.B * a.H * a.N;
+    CUtensorMap tq, tk, tv;
+    if (!make_tmap(&tq, a.q, rows, D) || !make_tmap(&tk, a.k, rows, D) || !make_tmap(&tv, a.v, rows, D))
+        return SSD_ERR_CUDA;
+    static std::atomic<uint64_t> attr_set{0};  // one bit per device
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_set.load() & bit)) {
+        if (cudaFuncSetAttribute(tc_order2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)K::SMEM) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        attr_set.fetch_or(bit);
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.B * a.H * K::R);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = K::SMEM;
+    cfg.stream = a.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = K::R;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_order2_kernel<D>, tq, tk, tv,
+                                       static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log,
+                                       a.dt_bias, a.D, a.H, a.N, a.normalize, status);
+    return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
 }  // namespace
 
 bool tc_order2_supports(int B, int H, int N, int d, int dtype, int chunk) {
-    return dtype == SSD_BF16 && d == kD && chunk == kC && (long long)B * H * N < (1ll << 31);
+    return dtype == SSD_BF16 && (d == 32 || d == 64) && chunk == kC &&
+           (long long)B * H * N < (1ll << 31);
 }
 
 size_t tc_order2_workspace(int, int, int, int, int) { return 0; }
 
 int launch_tc_order2(const FwdArgs &a, const Plan &) {
-    const uint64_t rows = (uint64_t)a.B * a.H * a.N;
-    CUtensorMap tq, tk, tv;
-    if (!make_tmap_rows32(&tq, a.q, rows) || !make_tmap_rows32(&tk, a.k, rows) ||
-        !make_tmap_rows32(&tv, a.v, rows))
-        return SSD_ERR_CUDA;
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(tc_order2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytes) != cudaSuccess)
-            return SSD_ERR_CUDA;
-        attr_set = true;
-    }
-    DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
-    tc_order2_kernel<<<a.B * a.H, kThreads, kSmemBytes, a.stream>>>(
-        tq, tk, tv, static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log, a.dt_bias, a.D, a.H,
-        a.N, a.normalize, status);
-    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+    return a.d == 64 ? launch_d<64>(a) : launch_d<32>(a);
 }
 
 }  // namespace ssd
