@@ -182,9 +182,9 @@ const char *ssd_status_str(int status);
 /*
  * Which kernel sequence ssd_fwd() runs for these arguments: 0 = the general
  * SIMT path (any supported shape, fp32 or bf16), 1 = the order-1 tcgen05
- * path that walks each head's chunks in order, 2 = the order-2 tcgen05 path,
- * 3 = the chunk-parallel order-1 tcgen05 path (chunk states, state passing,
- * chunk outputs); -1 when the arguments are invalid.
+ * path (chunk states, state passing, chunk outputs: three launches),
+ * 2 = the order-2 tcgen05 path (one launch); -1 when the arguments are
+ * invalid.
  * *n_launches (may be NULL) receives the number of kernels one call launches.
  */
 int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,

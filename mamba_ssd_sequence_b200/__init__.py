@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libssd.so")
 
 SSD_F32 = 0
 SSD_BF16 = 1
-PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2", 3: "tc_chunked"}
+PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2"}
 
 _lib = None
 

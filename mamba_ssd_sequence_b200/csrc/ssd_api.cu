@@ -35,15 +35,10 @@ bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, 
                Plan *plan) {
     if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
     Plan p{};
-    if (order == 1 && !normalize && tc_chunked_supports(B, H, N, d, dtype, chunk)) {
-        p.path = PATH_TC_CHUNKED;
-        p.n_launches = 3;
-        tc_chunked_layout(B, H, N, chunk, &p);
-    } else if (order == 1 && !normalize && tc_order1_supports(B, H, N, d, dtype, chunk)) {
+    if (order == 1 && !normalize && tc_order1_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER1;
-        p.n_launches = 1;
-        p.acs_off = p.lam_off = p.state_off = kStatusBytes;
-        p.total = kStatusBytes + tc_order1_workspace(B, H, N, d, chunk);
+        p.n_launches = 3;
+        tc_order1_layout(B, H, N, chunk, &p);
     } else if (order == 2 && tc_order2_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER2;
         p.n_launches = 1;
@@ -101,7 +96,6 @@ int ssd_fwd(const void *q, const void *k, const void *v, const float *dt_p,
     switch (p.path) {
     case PATH_TC_ORDER1: return launch_tc_order1(a, p);
     case PATH_TC_ORDER2: return launch_tc_order2(a, p);
-    case PATH_TC_CHUNKED: return launch_tc_chunked(a, p);
     default: return launch_simt(a, p);
     }
 }

@@ -33,7 +33,7 @@ constexpr size_t kStatusBytes = 256;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-enum Path { PATH_SIMT = 0, PATH_TC_ORDER1 = 1, PATH_TC_ORDER2 = 2, PATH_TC_CHUNKED = 3 };
+enum Path { PATH_SIMT = 0, PATH_TC_ORDER1 = 1, PATH_TC_ORDER2 = 2 };
 
 // Workspace plan for one call: which path runs and where its buffers sit.
 struct Plan {
@@ -48,15 +48,12 @@ bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, 
 
 // Path launchers (each returns an ssd_status).
 int launch_simt(const FwdArgs &a, const Plan &p);
-int launch_tc_order1(const FwdArgs &a, const Plan &p);
 int launch_tc_order2(const FwdArgs &a, const Plan &p);
-bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);
 bool tc_order2_supports(int B, int H, int N, int d, int dtype, int chunk);
-size_t tc_order1_workspace(int B, int H, int N, int d, int chunk);
 size_t tc_order2_workspace(int B, int H, int N, int d, int chunk);
-int launch_tc_chunked(const FwdArgs &a, const Plan &p);
-bool tc_chunked_supports(int B, int H, int N, int d, int dtype, int chunk);
-void tc_chunked_layout(int B, int H, int N, int chunk, Plan *p);
+int launch_tc_order1(const FwdArgs &a, const Plan &p);
+bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);
+void tc_order1_layout(int B, int H, int N, int chunk, Plan *p);
 
 // Kernel (a): chunk-local inclusive cumsum of A*dt and the chunk totals.
 // When `status` is non-NULL, block (0,0) thread 0 clears it.

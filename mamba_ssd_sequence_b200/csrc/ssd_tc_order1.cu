@@ -1,33 +1,24 @@
-// Order-1 tensor-core path (tcgen05 + TMEM, TMA) of the SSD forward operator
-// for bf16 inputs, d_h = 64, chunk = 128, no normaliser.
+// Chunk-parallel order-1 tensor-core path of the SSD forward operator for
+// bf16 inputs, d_h = 64, chunk C in {128, 256}, no normaliser.
 //
-// Each (batch, head) is split into R segments of whole chunks; one CTA per
-// segment.  A CTA first folds the chunks before its segment into the carried
-// state (K and V only, no output), then produces its own chunks; so it never
-// waits for another CTA, and the state it carries never leaves the SM.  Per
-// chunk c (2Mamba2Furious, Algorithms 1, 3, 4 and 6, evaluated in the
-// chunked state-passing form of the semiseparable mask):
-//   acs_t = chunk-local inclusive cumsum of A*dt (log2 units)  (kernel (a), fused)
-//   S     = Q K^T                                  tcgen05, fp32 in TMEM
-//   P_ij  = S_ij 2^(acs_i - acs_j) [i >= j]        CUDA cores, bf16 back into TMEM
-//   U_c   = K'^T V,   K'_j = 2^(lam_c - acs_j) k_j  tcgen05 (the chunk's own state term)
-//   h_c   = 2^(lam_c) h_{c-1} + U_c                 CUDA cores, fp32
-//   Y     = P V + Q' h_{c-1},  Q'_i = 2^(acs_i) q_i  tcgen05 (P from TMEM)
-//   y_i   = Y_i [+ D v_i]                           epilogue, 16-byte stores
-//
-// Warp roles (608 threads): warp 0 issues TMA loads into a 3-stage ring;
-// warps 1 and 2 each issue the MMAs of one compute group in a fixed order
-// (blocking, bounded waits: no polling); warps 3-10 and 11-18 are two compute
-// groups that take even and odd chunks (ping-pong), so one group's
-// exponentials overlap the other's MMAs and epilogue.  In a group the two
-// warps that share a TMEM lane quarter split each row's columns.  Each group
-// keeps its own copy of the carried state and advances it two chunks at a
-// time, h_{c-1} = 2^(lam_{c-1}) h_{c-2} + U_{c-1}, where U_{c-1} is the other
-// group's chunk term read from TMEM: the only cross-group dependency is an
-// MMA result, never a chain of group-to-group hand-offs.  All exponentials
-// are of non-positive arguments (chunk-local differences).  Every wait is
-// bounded; a timeout sets SSD_ERR_TIMEOUT in the workspace status and all
-// roles leave their loops.
+// The chunked form of 2Mamba2Furious (thelatestinai.com summary page,
+// Algorithms 3-5) splits the masked product into work that is independent per
+// chunk and one short recurrence over chunk states.  Three launches:
+//   (1) chunk_state_kernel, one CTA per chunk c of a head:
+//         acs_t = chunk-local inclusive cumsum of A dt (log2 units), lam = acs_{C-1}
+//         U_c   = sum_j 2^(lam - acs_j) k_j v_j^T          (tcgen05, M = N = 64, K = C)
+//   (2) state_pass_kernel: h_{-1} = 0, hin_c = bf16(h_{c-1}),
+//         h_c = 2^lam_c h_{c-1} + U_c                      (fp32, elementwise over the 64 x 64 state)
+//   (3) chunk_scan_kernel, persistent, one 128-row output tile per step:
+//         S = Q K^T over the keys of the chunk up to the tile's last row   (tcgen05)
+//         P_ij = S_ij 2^(acs_i - acs_j) [j <= i]           (CUDA cores)
+//         Y = P V,  Z = Q hin                               (tcgen05)
+//         y_i = Y_i + 2^acs_i Z_i [+ D v_i]
+// The decay of an off-diagonal 32 x 32 block of P is factorised through the
+// block's last key r: 2^(acs_i - acs_j) = 2^(acs_i - acs_r) 2^(acs_r - acs_j),
+// both factors <= 1 because acs falls along the chunk, so one exp2 per row and
+// per column replaces one per element; diagonal blocks take the exact
+// per-element exp2.  Every wait is bounded; a timeout sets the status word.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -43,471 +34,731 @@ namespace {
 
 using namespace ptx;
 
-constexpr int kC = 128;             // chunk length = rows of every tile
-constexpr int kD = 64;              // head dim
-constexpr int kStages = 3;          // TMA ring depth
-constexpr int kGroupThreads = 256;  // one compute group: 8 warps, 2 per TMEM lane quarter
-constexpr int kFirstGroupWarp = 3;
-constexpr int kThreads = 32 * kFirstGroupWarp + 2 * kGroupThreads;
-constexpr uint32_t kTileBytes = kC * kD * 2;  // 16 KiB bf16 tile
-constexpr uint32_t kStageBytes = 3 * kTileBytes;
-
-constexpr uint32_t kHRow = kD + 4;                               // padded fp32 row of h
-constexpr uint32_t kOffStage = 0;                                // kStages x {Q, K, V}
-constexpr uint32_t kOffHs = kOffStage + kStages * kStageBytes;   // 2 x h_{c-1} bf16 (64 x 64)
-constexpr uint32_t kOffH32 = kOffHs + 2 * kD * kD * 2;           // 2 x own state h (fp32)
-constexpr uint32_t kOffDres = kOffH32 + 2 * kD * kHRow * 4;      // D of this head (fp32)
-constexpr uint32_t kOffMisc = kOffDres + kD * 4;
-constexpr uint32_t kSmemBytes = kOffMisc + 2048 + 1024;          // misc + alignment slack
-
-// TMEM columns
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;     // 2 x 128: S (fp32), then P (bf16 pairs) at [32, 96)
-constexpr uint32_t kColP = 32;    // offset of P inside an S slot
-constexpr uint32_t kColY = 256;   // 2 x 64: Y
-constexpr uint32_t kColU = 384;   // 2 x 64: U (M = 64 layout, rows at lanes 32g + 0..15)
-
+constexpr int kD = 64;
+constexpr uint32_t kRowB = 128;         // bytes per bf16 row of 64
+constexpr uint32_t kBox = 128 * kRowB;  // one TMA box: 128 rows, 16 KiB
+constexpr uint32_t kHinBytes = 64 * kRowB;
 constexpr float kLog2e = 1.4426950408889634f;
-
-struct Misc {
-    float acs2[2][kC];
-    float wtot[2][4];
-    float lam_red[2][4];
-    uint64_t stage_full[kStages];
-    uint64_t stage_empty[kStages];
-    uint64_t s_full[2], kp_full[2], p_full[2], u_full[2], u_free[2], hs_full[2], y_full[2],
-        y_free[2];
-    uint32_t tmem_base;
-    int abort_flag;
-};
-static_assert(sizeof(Misc) <= 2048, "misc block");
 
 __device__ __forceinline__ float softplus_f(float x) {
     return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
-__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) { return make_sdesc(saddr, 16, 1024); }
-__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) {
-    return make_sdesc(saddr, kTileBytes, 1024);
-}
-// bf16 pair (low, high) -> float2
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
-__device__ __forceinline__ uint32_t f2_to_bf2(float2 v) { return pack_bf16x2(v.x, v.y); }
+__device__ __forceinline__ uint64_t desc_k(uint32_t saddr) { return make_sdesc(saddr, 16, 1024); }
+__device__ __forceinline__ uint64_t desc_mn(uint32_t saddr) { return make_sdesc(saddr, 8192, 1024); }
 
-// Scales columns [32 hf, 32 hf + 32) of row `row` of a 128B-swizzled bf16 tile.
-__device__ __forceinline__ void scale_half_row_inplace(uint8_t *tile, int row, int hf, float s) {
-    const float2 s2 = make_float2(s, s);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 *p = reinterpret_cast<uint4 *>(tile + sw128_chunk(row, hf * 4 + q));
-        uint4 u = *p;
-        u.x = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.x), s2));
-        u.y = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.y), s2));
-        u.z = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.z), s2));
-        u.w = f2_to_bf2(__fmul2_rn(bf2_to_f2(u.w), s2));
-        *p = u;
-    }
-}
-
-// P for 16 columns (tokens j0 .. j0+15, all inside column block jb) of this
-// thread's row, from the S values `sv` already loaded; writes 8 packed bf16
-// columns of TMEM at column j0 / 2.  Blocks entirely above the diagonal
-// (jb > g) are written as zeros.
-__device__ __forceinline__ void build_p16(uint32_t tP, int j0, int jb, int g, int row, float acs2,
-                                          const float *acs_row, const float (&sv)[16]) {
-    uint32_t pk[8];
-    if (jb > g) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pk[e] = 0u;
-    } else {
-        const float2 ai = make_float2(acs2, acs2);
-        const float4 *ac = reinterpret_cast<const float4 *>(acs_row + j0);
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const float4 aj = ac[q4];
-            const float2 d0 = __fadd2_rn(ai, make_float2(-aj.x, -aj.y));
-            const float2 d1 = __fadd2_rn(ai, make_float2(-aj.z, -aj.w));
-            float2 p0 = __fmul2_rn(make_float2(sv[q4 * 4], sv[q4 * 4 + 1]),
-                                   make_float2(ex2_approx(d0.x), ex2_approx(d0.y)));
-            float2 p1 = __fmul2_rn(make_float2(sv[q4 * 4 + 2], sv[q4 * 4 + 3]),
-                                   make_float2(ex2_approx(d1.x), ex2_approx(d1.y)));
-            if (jb == g) {  // the diagonal block: keep j <= i
-                const int j = j0 + q4 * 4;
-                if (j > row) p0.x = 0.0f;
-                if (j + 1 > row) p0.y = 0.0f;
-                if (j + 2 > row) p1.x = 0.0f;
-                if (j + 3 > row) p1.y = 0.0f;
-            }
-            pk[q4 * 2] = f2_to_bf2(p0);
-            pk[q4 * 2 + 1] = f2_to_bf2(p1);
-        }
-    }
-    tmem_st8(tP + j0 / 2, pk);
-}
-
-__device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
+__device__ void set_timeout(DeviceStatus *status, int where, int *abort_flag) {
     if (status) {
         atomicCAS(&status->code, 0, (int)SSD_ERR_TIMEOUT);
         atomicCAS(&status->detail, 0, where);
     }
-    *reinterpret_cast<volatile int *>(&misc->abort_flag) = 1;
+    if (abort_flag) *reinterpret_cast<volatile int *>(abort_flag) = 1;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-tc_order1_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
-                 const float *__restrict__ dt_p, const float *__restrict__ A_log,
-                 const float *__restrict__ dt_bias, const float *__restrict__ Dres, int H, int N,
-                 int BH, int R, DeviceStatus *status) {
+// =====================================================================
+// (1) chunk states: persistent, warp-specialised
+//   warp 0: TMA producer (ring of K, V chunk tiles)
+//   warp 1: MMA issuer (U_c^T = V^T K' into the owning group's TMEM accumulator)
+//   NG compute groups of 4 warps taking chunks round-robin: decay scan, K'
+//   scaling in place, U epilogue.  While one group waits for its product the
+//   others work, which hides most of each chunk's latency chain.
+// U is stored transposed, U^T[n][k] (value index n, feature index k), which
+// is the K-major layout the output kernel's MMA takes for the state.
+// =====================================================================
+constexpr int kStateGroup = 128;
+
+template <int C>
+struct StateCfg {
+    static constexpr int NG = C == 128 ? 4 : 2;
+    static constexpr int THREADS = 64 + NG * kStateGroup;
+    static constexpr int STAGES = C == 128 ? 6 : 3;
+    static constexpr uint32_t STAGE = 2 * C * kRowB;  // K then V
+    static constexpr uint32_t MISC_OFF = STAGES * STAGE;
+    static constexpr uint32_t MISC_BYTES = 4 * NG * C + 1024;
+    static constexpr uint32_t SMEM = MISC_OFF + MISC_BYTES + 1024;
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int C>
+struct StateMisc {
+    static constexpr int NG = StateCfg<C>::NG;
+    float wk[NG][C];  // per group: 2^(lam - acs_j) per key
+    float wtot[NG][4];
+    uint64_t stage_full[StateCfg<C>::STAGES], stage_empty[StateCfg<C>::STAGES];
+    uint64_t kp_full[NG], u_full[NG], u_free[NG];
+    uint64_t drain;
+    uint32_t tmem;
+    int abort_flag;
+};
+static_assert(sizeof(StateMisc<128>) <= StateCfg<128>::MISC_BYTES, "misc block");
+static_assert(sizeof(StateMisc<256>) <= StateCfg<256>::MISC_BYTES, "misc block");
+
+template <int C>
+__global__ void __launch_bounds__(StateCfg<C>::THREADS, 1)
+chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const float *__restrict__ dt_p, const float *__restrict__ A_log,
+                   const float *__restrict__ dt_bias, int H, int N, int n_chunks, float *__restrict__ acs_out,
+                   float *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status) {
+    using K = StateCfg<C>;
+    constexpr int NG = K::NG;
+    constexpr int KP = C / 128;  // keys per thread in the decay scan
+    pdl_launch_dependents();  // the state pass waits for this grid before it reads anything
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Misc *misc = reinterpret_cast<Misc *>(smem + kOffMisc);
+    StateMisc<C> *misc = reinterpret_cast<StateMisc<C> *>(smem + K::MISC_OFF);
     const volatile int *abort_flag = &misc->abort_flag;
-
+    const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x % BH, seg = blockIdx.x / BH, h = bh % H;
-    const int nc = N / kC;
-    const int row0 = bh * N;
-    // This CTA produces the outputs of chunks [c_begin, c_end) of its head.
-    // Chunks [0, c_begin) are only folded into the carried state (K and V
-    // are read, no output), so the CTA starts its own segment from the exact
-    // state without waiting for another CTA.
-    const int c_begin = (seg * nc) / R, c_end = ((seg + 1) * nc) / R;
-    // index of own chunk c among the own chunks of its parity (phases of the
-    // barriers that only own chunks use)
-    auto own_idx = [&](int c) { return (c - (c_begin + ((c ^ c_begin) & 1))) >> 1; };
+    const int nc = N / C;
 
     if (tid == 0) {
         if (blockIdx.x == 0 && status) {
             status->code = 0;
             status->detail = 0;
         }
-        for (int i = 0; i < kStages; ++i) {
+        for (int i = 0; i < K::STAGES; ++i) {
             mbar_init(&misc->stage_full[i], 1);
-            mbar_init(&misc->stage_empty[i], kGroupThreads);
+            mbar_init(&misc->stage_empty[i], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&misc->s_full[s], 1);
-            mbar_init(&misc->kp_full[s], kGroupThreads);
-            mbar_init(&misc->p_full[s], kGroupThreads);
-            mbar_init(&misc->u_full[s], 1);
-            mbar_init(&misc->u_free[s], 2 * kGroupThreads);
-            mbar_init(&misc->hs_full[s], kGroupThreads);
-            mbar_init(&misc->y_full[s], 1);
-            mbar_init(&misc->y_free[s], kGroupThreads);
+        for (int b = 0; b < NG; ++b) {
+            mbar_init(&misc->kp_full[b], kStateGroup);
+            mbar_init(&misc->u_full[b], 1);
+            mbar_init(&misc->u_free[b], kStateGroup);
         }
+        mbar_init(&misc->drain, 1);
         misc->abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&misc->tmem_base, kTmemCols);
+        tmem_alloc(&misc->tmem, 64 * NG);
         tmem_relinquish();
-    }
-    {
-        float *sD = reinterpret_cast<float *>(smem + kOffDres);
-        float *sH32 = reinterpret_cast<float *>(smem + kOffH32);
-        for (int i = tid; i < kD; i += kThreads) sD[i] = Dres ? Dres[h * kD + i] : 0.0f;
-        for (int i = tid; i < 2 * kD * (int)kHRow; i += kThreads) sH32[i] = 0.0f;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = misc->tmem_base;
+    const uint32_t tmem = misc->tmem;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_k);
+            prefetch_tmap(&tm_v);
+            int i = 0;
+            for (int t = blockIdx.x; t < n_chunks; t += gridDim.x, ++i) {
+                const int st = i % K::STAGES;
+                if (i >= K::STAGES &&
+                    !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag)) {
+                    set_timeout(status, 100, &misc->abort_flag);
+                    break;
+                }
+                const int row = t * C;  // chunks are contiguous row blocks of [B H N, d]
+                uint8_t *sp = smem + st * K::STAGE;
+                mbar_arrive_expect_tx(&misc->stage_full[st], K::STAGE);
+#pragma unroll
+                for (int b = 0; b < C / 128; ++b) {
+                    tma_load_2d(sp + b * kBox, &tm_k, 0, row + 128 * b, &misc->stage_full[st]);
+                    tma_load_2d(sp + C * kRowB + b * kBox, &tm_v, 0, row + 128 * b, &misc->stage_full[st]);
+                }
+            }
+            for (int j = i > K::STAGES ? i - K::STAGES : 0; j < i; ++j)
+                mbar_wait_bounded(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idU = make_idesc_bf16(64, 64, 1, 1);
+            bool ok = true;
+            int i = 0;
+            for (int t = blockIdx.x; t < n_chunks; t += gridDim.x, ++i) {
+                const int st = i % K::STAGES, ub = i % NG, use = i / NG;
+                if (!(ok = mbar_wait_abortable(&misc->kp_full[ub], use & 1, abort_flag))) break;
+                if (use >= 1 && !(ok = mbar_wait_abortable(&misc->u_free[ub], (use - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+                const uint32_t sp = sbase + st * K::STAGE;
+                // D[n][k] = sum_j v_jn k'_jk: A = V (MN-major), B = K' (MN-major)
+#pragma unroll
+                for (int ks = 0; ks < C / 16; ++ks)
+                    mma_bf16(tmem + 64 * ub, desc_mn(sp + C * kRowB + ks * 2048), desc_mn(sp + ks * 2048), idU,
+                             ks > 0);
+                mma_commit(&misc->u_full[ub]);
+                mma_commit(&misc->stage_empty[st]);
+            }
+            if (!ok) {
+                set_timeout(status, 101, &misc->abort_flag);
+                mma_commit(&misc->drain);
+                mbar_wait_bounded(&misc->drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ compute groups
+        const int gi = (warp - 2) >> 2;      // group: chunks i with i % NG == gi
+        const int gt = (tid - 64) & 127;     // thread in the group
+        const int gw = gt >> 5;              // warp in the group
+        const int g = warp & 3;              // TMEM lane quarter
+        const uint32_t lane_off = (uint32_t)(g * 32) << 16;
+        const int bar = 1 + gi;
+        bool failed = false;
+
+        struct Raw {
+            float dt[KP], alog, bias;
+        };
+        auto fetch = [&](int t) -> Raw {
+            Raw x;
+#pragma unroll
+            for (int e = 0; e < KP; ++e) x.dt[e] = 0.0f;
+            x.alog = x.bias = 0.0f;
+            if (t >= n_chunks) return x;
+            const int h = (t / nc) % H;
+            x.alog = __ldg(A_log + h);
+            x.bias = __ldg(dt_bias + h);
+#pragma unroll
+            for (int e = 0; e < KP; ++e) x.dt[e] = __ldg(dt_p + (size_t)t * C + KP * gt + e);
+            return x;
+        };
+
+        int i = gi;
+        Raw raw_next = fetch(blockIdx.x + gi * gridDim.x);
+        for (int t = blockIdx.x + gi * gridDim.x; t < n_chunks; t += NG * gridDim.x, i += NG) {
+            const int st = i % K::STAGES, use = i / NG;
+            const Raw raw = raw_next;
+            raw_next = fetch(t + NG * gridDim.x);
+            // ---- decay: inclusive scan of A dt over the chunk (log2 units)
+            const float A2 = -expf(raw.alog) * kLog2e;
+            float a[KP];
+            float run = 0.0f;
+#pragma unroll
+            for (int e = 0; e < KP; ++e) {
+                run += A2 * softplus_f(raw.dt[e] + raw.bias);
+                a[e] = run;
+            }
+            float incl = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            if (lane == 31) misc->wtot[gi][gw] = incl;
+            named_bar_sync(bar, kStateGroup);
+            float pre = incl - run, lam = 0.0f;
+#pragma unroll
+            for (int ww = 0; ww < 4; ++ww) {
+                const float x = misc->wtot[gi][ww];
+                if (ww < gw) pre += x;
+                lam += x;
+            }
+#pragma unroll
+            for (int e = 0; e < KP; ++e) {
+                const float acs = pre + a[e];
+                acs_out[(size_t)t * C + KP * gt + e] = acs;
+                misc->wk[gi][KP * gt + e] = ex2_approx(lam - acs);
+            }
+            if (gt == 0) lam_out[t] = lam;
+            // ---- K'_j = 2^(lam - acs_j) k_j in place: eight lanes per 128-byte row
+            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (i / K::STAGES) & 1, abort_flag);
+            if (named_bar_any(bar, kStateGroup, bad)) {  // also publishes wk[]
+                failed = true;
+                break;
+            }
+            uint8_t *sk = smem + st * K::STAGE;
+#pragma unroll 4
+            for (int it = 0; it < C / 16; ++it) {
+                const int j = it * 16 + (gt >> 3);
+                const float wj = misc->wk[gi][j];
+                const float2 w2 = make_float2(wj, wj);
+                uint4 *pp = reinterpret_cast<uint4 *>(sk + j * kRowB) + (gt & 7);
+                const uint4 x = *pp;
+                uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __fmul2_rn(bf2_to_f2(wv[q]), w2);
+                    wv[q] = pack_bf16x2(f.x, f.y);
+                }
+                *pp = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&misc->kp_full[gi]);
+            // ---- U^T epilogue: rows 16 g + lane (lanes 0-15) of the M = 64 accumulator
+            bad = !mbar_wait_abortable(&misc->u_full[gi], use & 1, abort_flag);
+            if (named_bar_any(bar, kStateGroup, bad)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            float v0[32], v1[32];
+            tmem_ld32(tmem + lane_off + 64 * gi, v0);
+            tmem_ld32(tmem + lane_off + 64 * gi + 32, v1);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&misc->u_free[gi]);
+            if (lane < 16) {
+                float4 *dst = reinterpret_cast<float4 *>(Ut + ((size_t)t * 64 + g * 16 + lane) * 64);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) dst[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    dst[8 + q] = make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
+            }
+        }
+        if (failed && gt == 0) set_timeout(status, 102, &misc->abort_flag);
+    }
+
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 64 * NG);
+}
+
+// =====================================================================
+// (2) state passing: one thread per 4 state entries of a head
+// =====================================================================
+__global__ void __launch_bounds__(256)
+state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __nv_bfloat16 *__restrict__ hin,
+                  int nc) {
+    pdl_launch_dependents();  // the chunk scan waits for this grid before it reads hin
+    pdl_wait();               // U and lam of the chunk-state kernel
+    const int bh = blockIdx.x;
+    const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // 4 consecutive entries of the 64 x 64 state
+    const float4 *u = reinterpret_cast<const float4 *>(U + (size_t)bh * nc * 4096 + e);
+    uint2 *out = reinterpret_cast<uint2 *>(hin + (size_t)bh * nc * 4096 + e);
+    const float *lm = lam + (size_t)bh * nc;
+    float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
+    // eight chunks' inputs are in flight before the dependent updates run
+    for (int c0 = 0; c0 < nc; c0 += 8) {
+        float4 ub[8];
+        float fb[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (c0 + j < nc) {
+                ub[j] = __ldg(u + (size_t)(c0 + j) * 1024);
+                fb[j] = __ldg(lm + c0 + j);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (c0 + j < nc) {
+                const float f = ex2_approx(fb[j]);
+                out[(size_t)(c0 + j) * 1024] = make_uint2(pack_bf16x2(hs.x, hs.y), pack_bf16x2(hs.z, hs.w));
+                hs.x = fmaf(f, hs.x, ub[j].x);
+                hs.y = fmaf(f, hs.y, ub[j].y);
+                hs.z = fmaf(f, hs.z, ub[j].z);
+                hs.w = fmaf(f, hs.w, ub[j].w);
+            }
+        }
+    }
+}
+
+// =====================================================================
+// (3) chunk scan: persistent, warp-specialised
+//   warp 0: TMA producer.
+//   warp 1: MMA issuer.  It polls its barriers and issues whichever product
+//     is ready: S' = Q [K ; hin^T]^T (scores and the state readout Z = Q hin
+//     in one N = 192 product), or Y = P V with P read from TMEM.
+//   NG compute groups of 8 warps (two for C = 128, one for C = 256) taking
+//     tiles round-robin: P from S (written back to TMEM as bf16), then the
+//     epilogue of the same tile.
+// Keeping P in TMEM and reading Q once for both S and Z roughly halves the
+// shared-memory operand traffic of the tensor core, which bounds this kernel.
+// =====================================================================
+template <int C>
+struct ScanCfg {
+    static constexpr int NG = C == 128 ? 2 : 1;      // compute groups
+    static constexpr int THREADS = 64 + 256 * NG;
+    static constexpr int NKB = C / 128;              // 128-key blocks per chunk
+    static constexpr int NRB = C / 128;              // 128-row tiles per chunk
+    static constexpr int NSB = C == 128 ? 2 : 1;     // S' buffers in TMEM
+    static constexpr int STAGES = C == 128 ? 3 : 2;
+    // Per stage: Q | K slots (NKB boxes) | hin^T (64 rows) | V slots (NKB boxes).
+    // The last K slot is followed directly by hin^T, so [K ; hin^T] is one
+    // B operand of 192 rows.  A tile with nkb key blocks puts key block kb in
+    // K slot NKB - nkb + kb.
+    static constexpr uint32_t Q_OFF = 0;
+    static constexpr uint32_t K_OFF = kBox;
+    static constexpr uint32_t H_OFF = K_OFF + NKB * kBox;
+    static constexpr uint32_t V_OFF = H_OFF + kHinBytes;
+    static constexpr uint32_t STAGE = V_OFF + NKB * kBox;
+    static constexpr uint32_t MISC_OFF = STAGES * STAGE;
+    static constexpr uint32_t MISC_BYTES = 20 * NG * C + 1024;
+    static constexpr uint32_t SMEM = MISC_OFF + MISC_BYTES + 1024;
+    // TMEM: C = 128: S' buffers at 0 and 192 (keys at +0, Z at +128);
+    //       C = 256: keys k at 128 (2 - nkb) + k, Z at 256.  Y buffers at 384, 448.
+    static constexpr uint32_t COL_Y = 384;
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(STAGE % 1024 == 0, "stage alignment");
+};
+
+// Per group, two alternating tile slots: a thread may write its group's next
+// tile's entries while a slower one still reads the current tile's.
+template <int C>
+struct ScanMisc {
+    static constexpr int NG = ScanCfg<C>::NG;
+    float acs[NG][2][C];
+    float colf[NG][2][C];   // 2^(acs_r - acs_j), r the last key of j's 32-key block
+    float dres[NG][2][64];  // D of the tile's head
+    uint64_t stage_full[ScanCfg<C>::STAGES], stage_empty[ScanCfg<C>::STAGES];
+    uint64_t s_full[ScanCfg<C>::NSB], p_full[NG][ScanCfg<C>::NKB], y_full[2], ep_done[2];
+    uint64_t drain;
+    uint32_t tmem;
+    int abort_flag;
+};
+static_assert(sizeof(ScanMisc<128>) <= ScanCfg<128>::MISC_BYTES, "misc block");
+static_assert(sizeof(ScanMisc<256>) <= ScanCfg<256>::MISC_BYTES, "misc block");
+
+struct TileIdx {
+    int bh, c, rb;
+};
+template <int C>
+__device__ __forceinline__ TileIdx tile_idx(int t, int nc) {
+    constexpr int NRB = ScanCfg<C>::NRB;
+    TileIdx x;
+    x.rb = t % NRB;
+    x.c = (t / NRB) % nc;
+    x.bh = t / (NRB * nc);
+    return x;
+}
+// TMEM column of key 0 of a tile's scores, and of its state readout Z
+template <int C>
+__device__ __forceinline__ uint32_t key_col(int sb, int nkb) {
+    return C == 128 ? (uint32_t)sb * 192u : 128u * (uint32_t)(2 - nkb);
+}
+template <int C>
+__device__ __forceinline__ uint32_t z_col(int sb) {
+    return C == 128 ? (uint32_t)sb * 192u + 128u : 256u;
+}
+
+template <int C>
+__global__ void __launch_bounds__(ScanCfg<C>::THREADS, 1)
+chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
+                  const __nv_bfloat16 *__restrict__ vglob, __nv_bfloat16 *__restrict__ out,
+                  const float *__restrict__ acs_in, const float *__restrict__ Dres, int H, int N,
+                  int n_tiles, DeviceStatus *status) {
+    using K = ScanCfg<C>;
+    constexpr int NG = K::NG;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    ScanMisc<C> *misc = reinterpret_cast<ScanMisc<C> *>(smem + K::MISC_OFF);
+    const volatile int *abort_flag = &misc->abort_flag;
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nc = N / C;
+    // number of tiles this CTA processes
+    const int my_tiles = (int)blockIdx.x < n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+
+    if (tid == 0) {
+        for (int i = 0; i < K::STAGES; ++i) {
+            mbar_init(&misc->stage_full[i], 1);
+            mbar_init(&misc->stage_empty[i], 1);
+        }
+        for (int i = 0; i < K::NSB; ++i) mbar_init(&misc->s_full[i], 1);
+        for (int gi = 0; gi < NG; ++gi)
+            for (int kb = 0; kb < K::NKB; ++kb) mbar_init(&misc->p_full[gi][kb], 256);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&misc->y_full[i], 1);
+            mbar_init(&misc->ep_done[i], 256);
+        }
+        mbar_init(&misc->drain, 1);
+        misc->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&misc->tmem, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc->tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            for (int c = 0; c < c_end; ++c) {
-                const int st = c % kStages;
-                if (c >= kStages &&
-                    !mbar_wait_abortable(&misc->stage_empty[st], ((c / kStages) - 1) & 1, abort_flag)) {
-                    raise_timeout(misc, status, 10);
+            prefetch_tmap(&tm_h);
+            pdl_wait();  // hin (state pass) and everything before it are visible
+            int i = 0;
+            for (; i < my_tiles; ++i) {
+                const int t = blockIdx.x + i * gridDim.x;
+                const int st = i % K::STAGES;
+                if (i >= K::STAGES &&
+                    !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag)) {
+                    set_timeout(status, 110, &misc->abort_flag);
                     break;
                 }
-                uint8_t *dst = smem + kOffStage + st * kStageBytes;
-                const int r = row0 + c * kC;
-                const bool own = c >= c_begin;
-                mbar_arrive_expect_tx(&misc->stage_full[st], own ? kStageBytes : 2 * kTileBytes);
-                if (own) tma_load_2d(dst, &tm_q, 0, r, &misc->stage_full[st]);
-                tma_load_2d(dst + kTileBytes, &tm_k, 0, r, &misc->stage_full[st]);
-                tma_load_2d(dst + 2 * kTileBytes, &tm_v, 0, r, &misc->stage_full[st]);
+                const TileIdx x = tile_idx<C>(t, nc);
+                const int nkb = x.rb + 1;
+                const int crow = x.bh * N + x.c * C;
+                uint8_t *sp = smem + st * K::STAGE;
+                mbar_arrive_expect_tx(&misc->stage_full[st], kBox + kHinBytes + 2 * nkb * kBox);
+                tma_load_2d(sp + K::Q_OFF, &tm_q, 0, crow + 128 * x.rb, &misc->stage_full[st]);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    tma_load_2d(sp + K::K_OFF + (K::NKB - nkb + kb) * kBox, &tm_k, 0, crow + 128 * kb,
+                                &misc->stage_full[st]);
+                    tma_load_2d(sp + K::V_OFF + kb * kBox, &tm_v, 0, crow + 128 * kb, &misc->stage_full[st]);
+                }
+                tma_load_2d(sp + K::H_OFF, &tm_h, 0, (x.bh * nc + x.c) * 64, &misc->stage_full[st]);
             }
+            // copies still in flight after an abort land before the CTA exits (bounded)
+            for (int j = i > K::STAGES ? i - K::STAGES : 0; j < i; ++j)
+                mbar_wait_bounded(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1);
         }
-    } else if (warp < 3) {
-        // ------------------------------------------------------ MMA issuers
-        // Warp 1 issues every MMA of group 0's chunks, warp 2 of group 1's, in
-        // chunk order: S, U, P V, Q' h.  Same-thread issue order keeps the
-        // slot reuse of S / P, Y and h_{c-1} in order; U slots are shared with
-        // the other group and are guarded by u_free.
-        const int s = warp - 1;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_S = make_idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t idesc_Y = make_idesc_bf16(128, 64, 0, 1);
-            constexpr uint32_t idesc_U = make_idesc_bf16(64, 64, 1, 1);
-            const uint32_t sbase = smem_u32(smem);
+            constexpr uint32_t idS128 = make_idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t idS192 = make_idesc_bf16(128, 192, 0, 0);
+            constexpr uint32_t idO = make_idesc_bf16(128, 64, 0, 1);
+            uint32_t np[NG][K::NKB];
+            for (int gi = 0; gi < NG; ++gi)
+                for (int kb = 0; kb < K::NKB; ++kb) np[gi][kb] = 0;
+            int next_s = 0, next_pv = 0, pv_kb = 0;
             bool ok = true;
-            for (int c = s; ok && c < c_end; c += 2) {
-                const int k = c >> 1, st = c % kStages;
-                const bool own = c >= c_begin;
-                const int ko = own ? own_idx(c) : 0;
-                const uint32_t aQ = sbase + kOffStage + st * kStageBytes;
-                const uint32_t aK = aQ + kTileBytes, aV = aK + kTileBytes;
-                if (own) {  // S = Q K^T
-                    if (!(ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag)))
+            uint64_t idle_since = globaltimer_ns();
+            uint32_t spins = 0;
+            while (next_pv < my_tiles) {
+                bool progress = false;
+                // ---- Y = P V for tile next_pv, one 128-key block at a time
+                if (next_pv < next_s) {
+                    const int i = next_pv, gi = i % NG, tb = i & 1, st = i % K::STAGES;
+                    const TileIdx x = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
+                    const int nkb = x.rb + 1;
+                    if (mbar_test(&misc->p_full[gi][pv_kb], np[gi][pv_kb] & 1)) {
+                        ++np[gi][pv_kb];
+                        tc_fence_after();
+                        const uint32_t sp = sbase + st * K::STAGE;
+                        const uint32_t pcol = key_col<C>(i % K::NSB, nkb) + 128 * pv_kb;
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            mma_bf16_ts(tmem + K::COL_Y + tb * 64, tmem + pcol + 64 * (ks >> 2) + 8 * (ks & 3),
+                                        desc_mn(sp + K::V_OFF + pv_kb * kBox + ks * 2048), idO,
+                                        (pv_kb > 0 || ks > 0));
+                        if (++pv_kb == nkb) {
+                            mma_commit(&misc->y_full[tb]);
+                            mma_commit(&misc->stage_empty[st]);
+                            ++next_pv;
+                            pv_kb = 0;
+                        }
+                        progress = true;
+                    }
+                }
+                // ---- S' for tile next_s (its TMEM buffer is free once tile next_s - NSB is done)
+                if (next_s < my_tiles) {
+                    const int j = next_s, st = j % K::STAGES;
+                    const int jp = j - K::NSB;  // previous user of the S' buffer
+                    const bool buf_free = jp < 0 || mbar_test(&misc->ep_done[jp & 1], (jp >> 1) & 1);
+                    if (buf_free && mbar_test(&misc->stage_full[st], (j / K::STAGES) & 1)) {
+                        tc_fence_after();
+                        const TileIdx x = tile_idx<C>(blockIdx.x + j * gridDim.x, nc);
+                        const int nkb = x.rb + 1;
+                        const int sb = j % K::NSB;
+                        const uint32_t sp = sbase + st * K::STAGE;
+                        const uint32_t kc = key_col<C>(sb, nkb);
+                        if (nkb == 2) {
+                            // keys [0, 128) of a 256-key row block: plain scores from K slot 0
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16(tmem + kc, desc_k(sp + K::Q_OFF + ks * 32), desc_k(sp + K::K_OFF + ks * 32),
+                                         idS128, ks > 0);
+                        }
+                        // last key block and the state readout: B = [K slot NKB - 1 ; hin^T]
+                        const uint32_t kl = sp + K::K_OFF + (K::NKB - 1) * kBox;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16(tmem + kc + 128 * (nkb - 1), desc_k(sp + K::Q_OFF + ks * 32), desc_k(kl + ks * 32),
+                                     idS192, ks > 0);
+                        mma_commit(&misc->s_full[sb]);
+                        ++next_s;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    idle_since = 0;
+                    spins = 0;
+                } else if ((++spins & 255u) == 0) {
+                    const uint64_t now = globaltimer_ns();
+                    if (idle_since == 0) idle_since = now;
+                    if (*abort_flag || now - idle_since > 1000000000ull) {
+                        ok = false;
                         break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks)
-                        mma_bf16(tmem + kColS + s * 128, desc_k(aQ + ks * 32), desc_k(aK + ks * 32),
-                                 idesc_S, ks > 0);
-                    mma_commit(&misc->s_full[s]);
+                    }
                 }
-                // U_c = K'^T V   (M = 64, N = 64, K = 128 tokens; K' and V MN-major)
-                if (!(ok = mbar_wait_abortable(&misc->kp_full[s], k & 1, abort_flag))) break;
-                if (c >= 2 && !(ok = mbar_wait_abortable(&misc->u_free[s], (k - 1) & 1, abort_flag)))
-                    break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_bf16(tmem + kColU + s * 64, desc_mn(aK + ks * 2048), desc_mn(aV + ks * 2048),
-                             idesc_U, ks > 0);
-                mma_commit(&misc->u_full[s]);
-                if (!own) continue;
-                // Y = P V   (A = P from TMEM, 8 packed columns per 16 tokens)
-                if (!(ok = mbar_wait_abortable(&misc->p_full[s], ko & 1, abort_flag))) break;
-                if (ko >= 1 && !(ok = mbar_wait_abortable(&misc->y_free[s], (ko - 1) & 1, abort_flag)))
-                    break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_bf16_ts(tmem + kColY + s * 64, tmem + kColS + s * 128 + kColP + ks * 8,
-                                desc_mn(aV + ks * 2048), idesc_Y, ks > 0);
-                // Y += Q' h_{c-1}
-                if (!(ok = mbar_wait_abortable(&misc->hs_full[s], ko & 1, abort_flag))) break;
-                tc_fence_after();
-                if (c >= 1) {
-                    const uint32_t aH = sbase + kOffHs + s * (kD * kD * 2);
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks)
-                        mma_bf16(tmem + kColY + s * 64, desc_k(aQ + ks * 32), desc_mn(aH + ks * 2048),
-                                 idesc_Y, 1);
-                }
-                mma_commit(&misc->y_full[s]);
             }
-            if (!ok) raise_timeout(misc, status, 20 + s);
+            if (!ok) {
+                set_timeout(status, 120, &misc->abort_flag);
+                // products still in flight finish before TMEM is released (bounded)
+                mma_commit(&misc->drain);
+                mbar_wait_bounded(&misc->drain, 0);
+            }
         }
-    } else if (warp >= kFirstGroupWarp) {
-        // ------------------------------------------------------ compute groups
-        const int s = (warp - kFirstGroupWarp) >> 3;  // 0: even chunks, 1: odd chunks
-        const int wi = (warp - kFirstGroupWarp) & 7;  // warp inside the group
-        const int g = warp & 3;                       // TMEM lane quarter = row block
-        const int hf = wi >> 2;                       // which half of each row's columns
-        const int row = g * 32 + lane;                // chunk row owned (shared by the halves)
-        const int wt = wi * 32 + lane;                // 0..255 inside the group
-        const int bar_id = 1 + s;                     // group barrier
+    } else {
+        // ------------------------------------------------------------ compute groups
+        const int gi = (warp - 2) >> 3;    // group: tiles i with i % NG == gi
+        const int ct = (tid - 64) & 255;   // thread in the group; key ct of the tile
+        const int gw = ct >> 5;            // warp in the group
+        const int g = warp & 3;            // TMEM lane quarter
+        const int hf = gw >> 2;            // half of the columns
         const uint32_t lane_off = (uint32_t)(g * 32) << 16;
-        const float A2 = -expf(A_log[h]) * kLog2e;
-        const float bias = dt_bias[h];
-        // own carried state h_{c-2}, fp32 in shared memory (row m = 16g + lane)
-        float *hown = reinterpret_cast<float *>(smem + kOffH32) + s * kD * kHRow;
-        const float *sD = reinterpret_cast<const float *>(smem + kOffDres);
-        // half 0 scans this chunk's decay; half 1 sums the previous chunk's
-        // (the other group's), so each loads one dt per chunk, one ahead
-        const int dt_off = hf == 0 ? 0 : -1;
-        float dt_next = (s + dt_off >= 0 && s + dt_off < c_end)
-                            ? dt_p[(size_t)row0 + (s + dt_off) * kC + row] : 0.0f;
+        const int r = g * 32 + lane;       // row of the 128-row tile
+        const int bar = 1 + gi;
 
-        for (int c = s; c < c_end; c += 2) {
-            const int k = c >> 1, st = c % kStages;
-            const bool own = c >= c_begin;  // produce outputs (else: state only)
-            const int ko = own ? own_idx(c) : 0;
-            uint8_t *sQ = smem + kOffStage + st * kStageBytes;
-            uint8_t *sK = sQ + kTileBytes;
-            uint8_t *sV = sK + kTileBytes;
-            const float dtv = dt_next;
-            const int cn = c + 2 + dt_off;
-            if (cn < c_end) dt_next = dt_p[(size_t)row0 + (size_t)cn * kC + row];
+        // Raw inputs of a tile, fetched one tile ahead: acs of key ct and four entries of D.
+        struct Raw {
+            float acs;
+            float4 d;
+        };
+        auto fetch = [&](int i) -> Raw {
+            Raw x{0.0f, make_float4(0.f, 0.f, 0.f, 0.f)};
+            if (i >= my_tiles) return x;
+            const TileIdx ti = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
+            if (ct < 128 * (ti.rb + 1)) x.acs = __ldg(acs_in + (size_t)ti.bh * N + (size_t)ti.c * C + ct);
+            if (Dres && ct < 16) x.d = __ldg(reinterpret_cast<const float4 *>(Dres + (ti.bh % H) * kD) + ct);
+            return x;
+        };
 
-            // ---- decay: scan of this chunk (half 0), total of chunk c-1 (half 1)
-            float a = (hf == 0 || c >= 1) ? A2 * softplus_f(dtv + bias) : 0.0f;
-            if (hf == 0) {
+        bool failed = false;
+        pdl_wait();  // acs (chunk-state kernel) is visible
+        Raw raw_next = fetch(gi);
+        for (int i = gi; i < my_tiles; i += NG) {
+            const TileIdx x = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
+            const int nkb = x.rb + 1;
+            const int sb = i % K::NSB, tb = i & 1, slot = (i / NG) & 1;
+            const Raw raw = raw_next;
+            raw_next = fetch(i + NG);
+            const int ir = 128 * x.rb + r;  // chunk-local row
+            const size_t grow = (size_t)x.bh * N + (size_t)x.c * C + ir;
+            uint4 vr[4];
+            if (Dres) {
+                const uint4 *vp = reinterpret_cast<const uint4 *>(vglob + grow * kD + hf * 32);
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, a, o);
-                    if (lane >= o) a += y;
-                }
-                if (lane == 31) misc->wtot[s][g] = a;
-            } else {
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-                if (lane == 0) misc->lam_red[s][g] = a;
+                for (int q = 0; q < 4; ++q) vr[q] = __ldg(vp + q);
+                if (ct < 16) *reinterpret_cast<float4 *>(&misc->dres[gi][slot][4 * ct]) = raw.d;
             }
-            named_bar_sync(bar_id, kGroupThreads);
-            const float lam2 = misc->wtot[s][0] + misc->wtot[s][1] + misc->wtot[s][2] + misc->wtot[s][3];
-            const float lam2_prev = misc->lam_red[s][0] + misc->lam_red[s][1] + misc->lam_red[s][2] +
-                                    misc->lam_red[s][3];
-            if (hf == 0) {
-                for (int w = 0; w < g; ++w) a += misc->wtot[s][w];
-                misc->acs2[s][row] = a;
+            // chunk-local cumulative decay of key ct, and its factor to the end of its 32-key block
+            const float aref = __shfl_sync(0xffffffffu, raw.acs, 31);
+            if (ct < C) {
+                misc->acs[gi][slot][ct] = raw.acs;
+                misc->colf[gi][slot][ct] = ex2_approx(aref - raw.acs);
             }
-
-            // ---- wait for this chunk's tiles and for S = Q K^T (after which Q and K
-            //      may be rewritten in place)
-            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
-            bad = bad || (own && !mbar_wait_abortable(&misc->s_full[s], ko & 1, abort_flag));
-            if (named_bar_any(bar_id, kGroupThreads, bad)) {
-                if (wt == 0) raise_timeout(misc, status, 32 + s);
+            // ---- S of this tile
+            bool bad = !mbar_wait_abortable(&misc->s_full[sb], (i / K::NSB) & 1, abort_flag);
+            if (named_bar_any(bar, 256, bad)) {  // also publishes acs[], colf[], dres[]
+                failed = true;
                 break;
             }
             tc_fence_after();
-            const float acs2 = misc->acs2[s][row];
-
-            // ---- K'_j = 2^(lam - acs_j) k_j, in place in the stage's K tile (half row)
-            scale_half_row_inplace(sK, row, hf, ex2_approx(lam2 - acs2));
-            fence_proxy_async_smem();
-            mbar_arrive(&misc->kp_full[s]);
-
-            if (own) {
-                // ---- P = S (.) 2^(acs_i - acs_j) [i >= j] -> bf16 pairs back into TMEM,
-                // at columns [32, 96) of the S slot (token j at 32 + j / 2).  Half 0
-                // covers tokens 0-63 and writes columns 32-63, which only it reads
-                // (S columns 0-63); half 1 covers tokens 64-127 and writes 64-95
-                // (inside its S columns 64-127).  The 16-token pieces go in an
-                // order in which every write lands on S values already consumed.
-                const uint32_t tS = tmem + lane_off + kColS + s * 128;
-#pragma unroll 1
-                for (int t = 0; t < 4; ++t) {
-                    // half 0: tokens 48, 32, 16, 0; half 1: 64, 80, 96, 112
-                    const int j0 = hf == 0 ? 48 - 16 * t : 64 + 16 * t;
-                    const int jb = j0 >> 5;
-                    float sv[16];
-                    if (jb <= g) {
-                        tmem_ld16(tS + j0, sv);
+            const float *acs = misc->acs[gi][slot];
+            const float ai = acs[ir];
+            const int W32 = 4 * x.rb + g;  // 32-row block of this warp, chunk-local
+            const uint32_t kc = key_col<C>(sb, nkb);
+            for (int kb = 0; kb < nkb; ++kb) {
+                // this warp reads S columns [64 hf, 64 hf + 64) of the key block and
+                // writes their bf16 P over the first 32 of them (in order, so
+                // nothing is overwritten before this warp has read it)
+                const uint32_t cb = tmem + lane_off + kc + 128 * kb + 64 * hf;
+#pragma unroll
+                for (int pc = 0; pc < 2; ++pc) {
+                    const int q = 2 * hf + pc;   // 32-key piece of the 128-key block
+                    const int P32 = 4 * kb + q;  // chunk-local 32-key block
+                    const int k0 = 32 * P32;
+                    uint32_t pk[16];
+                    if (P32 > W32) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[e] = 0u;
+                    } else {
+                        float sv[32];
+                        tmem_ld32(cb + 32 * pc, sv);
                         tmem_wait_ld();
+                        if (P32 < W32) {
+                            const float rowf = ex2_approx(ai - acs[k0 + 31]);
+                            const float2 rf2 = make_float2(rowf, rowf);
+                            const float4 *cf = reinterpret_cast<const float4 *>(&misc->colf[gi][slot][k0]);
+#pragma unroll
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 c4 = cf[e4];
+                                const float2 p0 = __fmul2_rn(
+                                    __fmul2_rn(make_float2(sv[4 * e4], sv[4 * e4 + 1]), make_float2(c4.x, c4.y)), rf2);
+                                const float2 p1 = __fmul2_rn(
+                                    __fmul2_rn(make_float2(sv[4 * e4 + 2], sv[4 * e4 + 3]), make_float2(c4.z, c4.w)),
+                                    rf2);
+                                pk[2 * e4] = pack_bf16x2(p0.x, p0.y);
+                                pk[2 * e4 + 1] = pack_bf16x2(p1.x, p1.y);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) {
+                                const int j = k0 + e;
+                                float p0 = sv[e] * ex2_approx(ai - acs[j]);
+                                float p1 = sv[e + 1] * ex2_approx(ai - acs[j + 1]);
+                                if (j > ir) p0 = 0.0f;
+                                if (j + 1 > ir) p1 = 0.0f;
+                                pk[e >> 1] = pack_bf16x2(p0, p1);
+                            }
+                        }
                     }
-                    build_p16(tS + kColP, j0, jb, g, row, acs2, misc->acs2[s], sv);
+                    tmem_st16(cb + 16 * pc, pk);
                 }
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&misc->p_full[s]);
-
-                // ---- Q'_i = 2^(acs_i) q_i, in place (the S MMA of this chunk is done)
-                scale_half_row_inplace(sQ, row, hf, ex2_approx(acs2));
+                mbar_arrive(&misc->p_full[gi][kb]);
             }
-
-            // ---- carried state: h_{c-1} (bf16, for Y) and own h_c; this warp does
-            //      columns [32 hf, 32 hf + 32) of rows m = 16g + lane (lane < 16)
-            bad = (c >= 1) && !mbar_wait_abortable(&misc->u_full[s ^ 1], ((c - 1) >> 1) & 1, abort_flag);
-            bad = bad || !mbar_wait_abortable(&misc->u_full[s], k & 1, abort_flag);
-            if (named_bar_any(bar_id, kGroupThreads, bad)) {
-                if (wt == 0) raise_timeout(misc, status, 34 + s);
+            // ---- epilogue: y = Y + 2^acs_i Z [+ D v], columns [32 hf, 32 hf + 32)
+            bad = !mbar_wait_abortable(&misc->y_full[tb], (i >> 1) & 1, abort_flag);
+            if (named_bar_any(bar, 256, bad)) {
+                failed = true;
                 break;
             }
             tc_fence_after();
-            {
-                const float dp = ex2_approx(lam2_prev), dc = ex2_approx(lam2);
-                const float2 dprev = make_float2(dp, dp), dcur = make_float2(dc, dc);
-                const uint32_t tUo = tmem + lane_off + kColU + (s ^ 1) * 64 + hf * 32;
-                const uint32_t tUs = tmem + lane_off + kColU + s * 64 + hf * 32;
-                uint8_t *sH = smem + kOffHs + s * (kD * kD * 2);
-                const int m = g * 16 + lane;  // state row (valid for lane < 16)
+            const float e = ex2_approx(ai);
+            const float *dh = &misc->dres[gi][slot][hf * 32];
+            uint4 *op = reinterpret_cast<uint4 *>(out + grow * kD + hf * 32);
+            const uint32_t zc = tmem + lane_off + z_col<C>(sb) + 32 * hf;
+            const uint32_t yc = tmem + lane_off + K::COL_Y + 64 * tb + 32 * hf;
 #pragma unroll
-                for (int qt = 0; qt < 2; ++qt) {
-                    float uo[16], us[16];
-                    if (c >= 1) tmem_ld16(tUo + qt * 16, uo);
-                    tmem_ld16(tUs + qt * 16, us);
-                    tmem_wait_ld();
-                    if (lane < 16) {
-                        const int col0 = hf * 32 + qt * 16;
-                        uint32_t hb[8];
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            float4 *hp4 = reinterpret_cast<float4 *>(hown + m * kHRow + col0 + e4 * 4);
-                            const float4 hv = *hp4;
-                            float2 h0 = make_float2(0.0f, 0.0f), h1 = h0;
-                            if (c >= 1) {
-                                h0 = __ffma2_rn(dprev, make_float2(hv.x, hv.y),
-                                                make_float2(uo[e4 * 4], uo[e4 * 4 + 1]));
-                                h1 = __ffma2_rn(dprev, make_float2(hv.z, hv.w),
-                                                make_float2(uo[e4 * 4 + 2], uo[e4 * 4 + 3]));
-                            }
-                            hb[e4 * 2] = f2_to_bf2(h0);
-                            hb[e4 * 2 + 1] = f2_to_bf2(h1);
-                            const float2 n0 = __ffma2_rn(dcur, h0, make_float2(us[e4 * 4], us[e4 * 4 + 1]));
-                            const float2 n1 = __ffma2_rn(dcur, h1, make_float2(us[e4 * 4 + 2], us[e4 * 4 + 3]));
-                            *hp4 = make_float4(n0.x, n0.y, n1.x, n1.y);
-                        }
-                        if (own && c >= 1) {
-                            *reinterpret_cast<uint4 *>(sH + sw128_chunk(m, col0 / 8)) =
-                                make_uint4(hb[0], hb[1], hb[2], hb[3]);
-                            *reinterpret_cast<uint4 *>(sH + sw128_chunk(m, col0 / 8 + 1)) =
-                                make_uint4(hb[4], hb[5], hb[6], hb[7]);
-                        }
-                    }
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            mbar_arrive(&misc->u_free[s]);
-            if (c >= 1) mbar_arrive(&misc->u_free[s ^ 1]);
-            if (!own) {
-                // state-only chunk: U_c has been read (u_full), so the stage is free
-                mbar_arrive(&misc->stage_empty[st]);
-                continue;
-            }
-            mbar_arrive(&misc->hs_full[s]);
-
-            // ---- epilogue: y = Y [+ D v], bf16, 16-byte stores straight to HBM
-            bad = !mbar_wait_abortable(&misc->y_full[s], ko & 1, abort_flag);
-            if (named_bar_any(bar_id, kGroupThreads, bad)) {
-                if (wt == 0) raise_timeout(misc, status, 36 + s);
-                break;
-            }
-            tc_fence_after();
-            {
-                float y0[16], y1[16];
-                tmem_ld16(tmem + lane_off + kColY + s * 64 + hf * 32, y0);
-                tmem_ld16(tmem + lane_off + kColY + s * 64 + hf * 32 + 16, y1);
+            for (int half = 0; half < 2; ++half) {
+                float yv[16], zv[16];
+                tmem_ld16(yc + 16 * half, yv);
+                tmem_ld16(zc + 16 * half, zv);
                 tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&misc->y_free[s]);
-                const float4 *Dh = reinterpret_cast<const float4 *>(sD);
-                uint4 *dst = reinterpret_cast<uint4 *>(out + (size_t)(row0 + c * kC + row) * kD + hf * 32);
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int ch = hf * 4 + q4;
-                    const float *yy = q4 < 2 ? (y0 + q4 * 8) : (y1 + (q4 - 2) * 8);
-                    uint32_t w[4];
-                    if (Dres) {
-                        const uint4 vv = *reinterpret_cast<const uint4 *>(sV + sw128_chunk(row, ch));
-                        const float4 d0 = Dh[2 * ch], d1 = Dh[2 * ch + 1];
-                        const uint32_t vw[4] = {vv.x, vv.y, vv.z, vv.w};
-                        const float2 dd[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
-                                              make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = f2_to_bf2(__ffma2_rn(dd[e], bf2_to_f2(vw[e]),
-                                                        make_float2(yy[2 * e], yy[2 * e + 1])));
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) w[e] = pack_bf16x2(yy[2 * e], yy[2 * e + 1]);
-                    }
-                    dst[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+                if (half == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&misc->ep_done[tb]);
                 }
-                mbar_arrive(&misc->stage_empty[st]);  // this thread is done with the stage
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int q = 2 * half + q2;
+                    uint32_t wv[4];
+                    const uint32_t vw[4] = {vr[q].x, vr[q].y, vr[q].z, vr[q].w};
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const int cl = q2 * 8 + 2 * pp;  // column within the half
+                        float y0 = fmaf(e, zv[cl], yv[cl]);
+                        float y1 = fmaf(e, zv[cl + 1], yv[cl + 1]);
+                        if (Dres) {
+                            const float2 vf = bf2_to_f2(vw[pp]);
+                            y0 = fmaf(dh[16 * half + cl], vf.x, y0);
+                            y1 = fmaf(dh[16 * half + cl + 1], vf.y, y1);
+                        }
+                        wv[pp] = pack_bf16x2(y0, y1);
+                    }
+                    op[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                }
             }
         }
+        if (failed && ct == 0) set_timeout(status, 130, &misc->abort_flag);
     }
 
+    __syncwarp();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------- host side
@@ -524,66 +775,115 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     return fn;
 }
 
-// [rows, 64] bf16 row-major tensor, boxes of box_rows x 64, 128-byte swizzle.
-bool make_tmap_rows64(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
+// [rows, 64] bf16 row-major tensor read in boxes of `box_rows` rows, 128-byte swizzle.
+bool make_tmap64(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
     auto enc = get_encode_fn();
     if (!enc) return false;
     cuuint64_t dims[2] = {64, rows};
     cuuint64_t strides[1] = {64 * 2};
     cuuint32_t box[2] = {64, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// Sets the dynamic shared-memory limit of `fn` once per device.
+template <typename F>
+bool smem_attr_once(F fn, int bytes, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load() & bit) return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    done.fetch_or(bit);
+    return true;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return n;
+}
+
+template <int C>
+int launch_c(const FwdArgs &a, const Plan &p) {
+    using K = ScanCfg<C>;
+    const int BH = a.B * a.H, nc = a.N / C;
+    const uint64_t rows = (uint64_t)BH * a.N;
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    DeviceStatus *status = reinterpret_cast<DeviceStatus *>(ws);
+    float *lam = reinterpret_cast<float *>(ws + p.lam_off);
+    float *acs = reinterpret_cast<float *>(ws + p.acs_off);
+    float *U = reinterpret_cast<float *>(ws + p.state_off);
+    __nv_bfloat16 *hin = reinterpret_cast<__nv_bfloat16 *>(ws + p.aux_off);
+    CUtensorMap tq, tk, tv, th;
+    if (!make_tmap64(&tq, a.q, rows, 128) || !make_tmap64(&tk, a.k, rows, 128) ||
+        !make_tmap64(&tv, a.v, rows, 128) || !make_tmap64(&th, hin, (uint64_t)BH * nc * 64, 64))
+        return SSD_ERR_CUDA;
+    static std::atomic<uint64_t> attr1{0}, attr3{0};
+    if (!smem_attr_once(chunk_state_kernel<C>, (int)StateCfg<C>::SMEM, attr1) ||
+        !smem_attr_once(chunk_scan_kernel<C>, (int)K::SMEM, attr3))
+        return SSD_ERR_CUDA;
+    const int sms = num_sms();
+    if (sms <= 0) return SSD_ERR_CUDA;
+
+    const int n_chunks = BH * nc;
+    chunk_state_kernel<C><<<n_chunks < sms ? n_chunks : sms, StateCfg<C>::THREADS, StateCfg<C>::SMEM, a.stream>>>(
+        tk, tv, a.dt_p, a.A_log, a.dt_bias, a.H, a.N, n_chunks, acs, U, lam, status);
+    // The state pass and the chunk scan are launched as programmatic dependents:
+    // their CTAs may start while the previous kernel drains, and each waits
+    // (griddepcontrol.wait) before it reads that kernel's results.
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3(BH, 4);
+    c2.blockDim = dim3(256);
+    c2.stream = a.stream;
+    c2.attrs = pdl;
+    c2.numAttrs = 1;
+    if (cudaLaunchKernelEx(&c2, state_pass_kernel, (const float *)U, (const float *)lam, hin, nc) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    const int n_tiles = BH * nc * K::NRB;
+    const int grid = n_tiles < sms ? n_tiles : sms;
+    cudaLaunchConfig_t c3 = {};
+    c3.gridDim = dim3(grid);
+    c3.blockDim = dim3(K::THREADS);
+    c3.dynamicSmemBytes = K::SMEM;
+    c3.stream = a.stream;
+    c3.attrs = pdl;
+    c3.numAttrs = 1;
+    if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, static_cast<const __nv_bfloat16 *>(a.v),
+                           static_cast<__nv_bfloat16 *>(a.out), (const float *)acs, a.D, a.H, a.N, n_tiles,
+                           status) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
 }  // namespace
 
 bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk) {
-    return dtype == SSD_BF16 && d == kD && chunk == kC && (long long)B * H * N < (1ll << 31);
+    return dtype == SSD_BF16 && d == kD && (chunk == 128 || chunk == 256) && (long long)B * H * N < (1ll << 31);
 }
 
-size_t tc_order1_workspace(int, int, int, int, int) { return 0; }
-
-// Segments per head: enough CTAs to cover the SMs, as long as the extra
-// state-only work (segment r re-folds r earlier segments) stays small.
-int segments_per_head(int BH, int nc) {
-    static int sms = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-            sms = 148;
-    }
-    int R = 1;
-    while (R < 2 && BH * (R * 2) <= sms && nc >= R * 2 * 2) R *= 2;
-    return R;
+// lam (n_chunks floats), acs (B H N floats), U (n_chunks x 64 x 64 fp32),
+// hin (n_chunks x 64 x 64 bf16)
+void tc_order1_layout(int B, int H, int N, int chunk, Plan *p) {
+    const size_t n = (size_t)B * H * (N / chunk);
+    p->lam_off = kStatusBytes;
+    p->acs_off = align_up(p->lam_off + n * sizeof(float), 256);
+    p->state_off = align_up(p->acs_off + (size_t)B * H * N * sizeof(float), 256);
+    p->aux_off = align_up(p->state_off + n * 4096 * sizeof(float), 256);
+    p->total = align_up(p->aux_off + n * 4096 * 2, 256);
 }
 
-int launch_tc_order1(const FwdArgs &a, const Plan &) {
-    if (a.normalize) return SSD_ERR_UNSUPPORTED;
-    const uint64_t rows = (uint64_t)a.B * a.H * a.N;
-    CUtensorMap tq, tk, tv;
-    if (!make_tmap_rows64(&tq, a.q, rows, kC) || !make_tmap_rows64(&tk, a.k, rows, kC) ||
-        !make_tmap_rows64(&tv, a.v, rows, kC))
-        return SSD_ERR_CUDA;
-    static std::atomic<uint64_t> attr_set{0};  // one bit per device
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
-    const uint64_t bit = 1ull << (dev & 63);
-    if (!(attr_set.load() & bit)) {
-        if (cudaFuncSetAttribute(tc_order1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kSmemBytes) != cudaSuccess)
-            return SSD_ERR_CUDA;
-        attr_set.fetch_or(bit);
-    }
-    DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
-    const int BH = a.B * a.H;
-    const int R = segments_per_head(BH, a.N / kC);
-    tc_order1_kernel<<<BH * R, kThreads, kSmemBytes, a.stream>>>(
-        tq, tk, tv, static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log, a.dt_bias, a.D, a.H, a.N, BH, R, status);
-    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+int launch_tc_order1(const FwdArgs &a, const Plan &p) {
+    if (a.normalize || a.order != 1) return SSD_ERR_UNSUPPORTED;
+    return a.chunk == 256 ? launch_c<256>(a, p) : launch_c<128>(a, p);
 }
 
 }  // namespace ssd

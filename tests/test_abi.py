@@ -84,9 +84,9 @@ def test_path_selection(lib):
     path, n = ssd.ssd_fwd_path(1, 2, 256, 16, ssd.SSD_F32, 1, 64)
     assert path == "simt" and n == 4
     path, n = ssd.ssd_fwd_path(4, 16, 2048, 64, ssd.SSD_BF16, 1, 128)
-    assert path == "tc_chunked" and n == 3
+    assert path == "tc_order1" and n == 3
     path, n = ssd.ssd_fwd_path(1, 32, 65536, 64, ssd.SSD_BF16, 1, 256)
-    assert path == "tc_chunked" and n == 3
+    assert path == "tc_order1" and n == 3
     path, n = ssd.ssd_fwd_path(1, 4, 1024, 64, ssd.SSD_BF16, 1, 64)
     assert path == "simt" and n == 4
     path, n = ssd.ssd_fwd_path(4, 16, 4096, 32, ssd.SSD_BF16, 2, 64)
