@@ -51,15 +51,17 @@ def _load():
     lib.oracle_mask.restype = ctypes.c_double
     lib.oracle_feature.argtypes = [_f64p, ctypes.c_int, ctypes.c_int, _f64p]
     lib.oracle_feature.restype = ctypes.c_int
-    lib.oracle_log_decay.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
+    lib.oracle_log_decay.argtypes = [_f32p, _f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_int, _f64p]
     lib.oracle_log_decay.restype = None
     lib.oracle_ssd_quadratic.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
+                                         _f32p, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, _i32p, ctypes.c_int,
                                          _f64p, _f64p]
     lib.oracle_ssd_quadratic.restype = ctypes.c_int
     lib.oracle_ssd_recurrent.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
+                                         _f32p, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
     lib.oracle_ssd_recurrent.restype = ctypes.c_int
@@ -104,28 +106,36 @@ def feature(x: np.ndarray, order: int) -> np.ndarray:
     return out
 
 
-def log_decay(dt_p, A_log, dt_bias) -> np.ndarray:
-    """A^CS = cumsum(-exp(A_log) * softplus(dt_p + dt_bias)) per (b, h), inclusive.
-
-    dt_p is [B, H, N]; returns float64 [B, H, N] (Algorithm 3, last line)."""
-    dt_p = _f32(dt_p)
-    B, H, N = dt_p.shape
-    A_log = _f32(A_log)
-    dt_bias = _f32(dt_bias)
+def log_decay(dt_p, A_log, dt_bias, log_decay_in=None) -> np.ndarray:
+    """A^CS = cumsum(-exp(A_log) * softplus(dt_p + dt_bias)) per (b, h), inclusive
+    (Algorithm 3, last line), or cumsum(log_decay_in) when that [B, H, N] array
+    is given (Algorithm 4).  Returns float64 [B, H, N]."""
+    ld = None if log_decay_in is None else _f32(log_decay_in)
+    dt_p = None if dt_p is None else _f32(dt_p)
+    B, H, N = (ld if ld is not None else dt_p).shape
+    A_log = None if A_log is None else _f32(A_log)
+    dt_bias = None if dt_bias is None else _f32(dt_bias)
     out = np.zeros((B, H, N), dtype=np.float64)
     _load().oracle_log_decay(_ptr(dt_p, _f32p), _ptr(A_log, _f32p), _ptr(dt_bias, _f32p),
-                             B, H, N, _ptr(out, _f64p))
+                             _ptr(ld, _f32p), B, H, N, _ptr(out, _f64p))
     return out
 
 
+def _opt(a):
+    return None if a is None else _f32(a)
+
+
 def ssd_quadratic(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
-                  rows: Optional[Sequence[int]] = None, return_norm: bool = False):
+                  rows: Optional[Sequence[int]] = None, return_norm: bool = False,
+                  log_decay=None, value_dt: bool = False):
     """Masked-matrix form of the operator (Algorithms 1 and 5), in float64.
 
-    Returns y as [B, H, len(rows) or N, d] (and the row sums N_i when
-    ``return_norm``)."""
-    q, k, v, dt_p = _f32(q), _f32(k), _f32(v), _f32(dt_p)
-    A_log, dt_bias = _f32(A_log), _f32(dt_bias)
+    ``log_decay`` ([B, H, N], optional) replaces A dt by a given per-token
+    log-decay (Algorithm 4); ``value_dt`` contracts with V (.) dt instead of V
+    (Algorithm 4, V_dt).  Returns y as [B, H, len(rows) or N, d] (and the row
+    sums N_i when ``return_norm``)."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    dt_p, A_log, dt_bias, ld = _opt(dt_p), _opt(A_log), _opt(dt_bias), _opt(log_decay)
     Dv = None if D is None else _f32(D)
     B, H, N, d = q.shape
     if rows is None:
@@ -138,8 +148,8 @@ def ssd_quadratic(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
     norm = np.zeros((B, H, n_rows), dtype=np.float64)
     rc = _load().oracle_ssd_quadratic(
         _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(dt_p, _f32p),
-        _ptr(A_log, _f32p), _ptr(dt_bias, _f32p), _ptr(Dv, _f32p),
-        B, H, N, d, int(order), int(bool(normalize)),
+        _ptr(A_log, _f32p), _ptr(dt_bias, _f32p), _ptr(Dv, _f32p), _ptr(ld, _f32p),
+        int(bool(value_dt)), B, H, N, d, int(order), int(bool(normalize)),
         _ptr(r_arr, _i32p), n_rows, _ptr(out, _f64p), _ptr(norm, _f64p))
     if rc != 0:
         raise ValueError("oracle_ssd_quadratic rejected its arguments")
@@ -147,13 +157,15 @@ def ssd_quadratic(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
 
 
 def ssd_recurrent(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
-                  return_norm: bool = False, return_state: bool = False):
+                  return_norm: bool = False, return_state: bool = False,
+                  log_decay=None, value_dt: bool = False):
     """Token-by-token recurrent form (Algorithm 6), in float64.
 
-    Returns y [B, H, N, d]; optionally the row sums [B, H, N] and the final
-    states H_up [B, H, d^order, d] and H_dn [B, H, d^order]."""
-    q, k, v, dt_p = _f32(q), _f32(k), _f32(v), _f32(dt_p)
-    A_log, dt_bias = _f32(A_log), _f32(dt_bias)
+    ``log_decay`` and ``value_dt`` as in ssd_quadratic.  Returns y
+    [B, H, N, d]; optionally the row sums [B, H, N] and the final states
+    H_up [B, H, d^order, d] and H_dn [B, H, d^order]."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    dt_p, A_log, dt_bias, ld = _opt(dt_p), _opt(A_log), _opt(dt_bias), _opt(log_decay)
     Dv = None if D is None else _f32(D)
     B, H, N, d = q.shape
     Dphi = d ** order
@@ -163,8 +175,8 @@ def ssd_recurrent(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
     zst = np.zeros((B, H, Dphi), dtype=np.float64) if return_state else None
     rc = _load().oracle_ssd_recurrent(
         _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(dt_p, _f32p),
-        _ptr(A_log, _f32p), _ptr(dt_bias, _f32p), _ptr(Dv, _f32p),
-        B, H, N, d, int(order), int(bool(normalize)),
+        _ptr(A_log, _f32p), _ptr(dt_bias, _f32p), _ptr(Dv, _f32p), _ptr(ld, _f32p),
+        int(bool(value_dt)), B, H, N, d, int(order), int(bool(normalize)),
         _ptr(out, _f64p), _ptr(norm, _f64p), _ptr(st, _f64p), _ptr(zst, _f64p))
     if rc != 0:
         raise ValueError("oracle_ssd_recurrent rejected its arguments")

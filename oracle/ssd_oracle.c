@@ -21,17 +21,25 @@
  *   - Algorithm 6 (2Mamba inference): H_up_t = a_t H_up_{t-1} + phi(k_t)^T v_t,
  *       H_dn_t = a_t H_dn_{t-1} + phi(k_t), phi(x) = x (x) x for order 2.
  *
+ *   - Algorithm 4 (Mamba-2S): A = -softplus(h W_A) given per token (the
+ *       "log_decay" input here), A^CS = cumsum(A), and the value
+ *       discretisation V_dt = V (.) dt with dt = softplus(h W_dt) (the
+ *       "value_dt" switch, with dt = softplus(dt_P + dt_bias)).
+ *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - the cumulative sum is inclusive and starts at zero for every (b, h);
- *   - the contraction uses raw V (no V * dt);
+ *   - the contraction uses raw V unless value_dt is set (then V_dt);
+ *   - the normaliser sums the masked score matrix only (it does not see dt);
  *   - the D residual is added after normalisation, to raw V;
  *   - the normaliser divides by the exact row sum, with no epsilon;
  *   - the Algorithm 6 output line is cut off on the page; the plain reading
  *     y_t = phi(q_t)^T H_up_t (divided by phi(q_t) . H_dn_t when normalising)
  *     is used.
  *
- * Layouts: q, k, v, out are [B, H, N, d] row-major; dt_p is [B, H, N];
- * A_log and dt_bias are [H]; D is [H*d] or NULL.
+ * Layouts: q, k, v, out are [B, H, N, d] row-major; dt_p and log_decay are
+ * [B, H, N]; A_log and dt_bias are [H]; D is [H*d] or NULL.  Pointers that an
+ * option does not use may be NULL: A_log when log_decay is given; dt_p and
+ * dt_bias when log_decay is given and value_dt is off.
  */
 #include <math.h>
 #include <stdint.h>
@@ -49,31 +57,44 @@ double oracle_softplus(double x)
     return (x > 0.0 ? x : 0.0) + log1p(exp(-ax));
 }
 
-/* Per-token log-decay a_t = A_h * dt_t and its inclusive cumulative sum
+/* Per-token log-decay a_t and its inclusive cumulative sum
  * A^CS_t = sum_{tau <= t} a_tau for one (b, h) row of length N.
  * Algorithm 3: A = -exp(A_log), dt = softplus(dt_P + dt_bias),
- * A^CS = cumsum(A (.) dt). */
+ * a_t = A * dt_t.  Algorithm 4: a_t is given directly (ld_row != NULL). */
 static void log_decay_row(const float *dt_p_row, double A_log_h, double dt_bias_h,
-                          int N, double *acs_row)
+                          const float *ld_row, int N, double *acs_row)
 {
-    double A = -exp(A_log_h);
     double run = 0.0;
     for (int t = 0; t < N; ++t) {
-        double dt = oracle_softplus((double)dt_p_row[t] + dt_bias_h);
-        run += A * dt;
+        if (ld_row) {
+            run += (double)ld_row[t];
+        } else {
+            double dt = oracle_softplus((double)dt_p_row[t] + dt_bias_h);
+            run += -exp(A_log_h) * dt;
+        }
         acs_row[t] = run;
     }
 }
 
-/* A^CS for every (b, h): out is [B, H, N]. */
+/* A^CS for every (b, h): out is [B, H, N].  log_decay ([B, H, N], may be
+ * NULL) replaces A * dt when given; A_log, dt_p and dt_bias are then unused. */
 void oracle_log_decay(const float *dt_p, const float *A_log, const float *dt_bias,
-                      int B, int H, int N, double *acs)
+                      const float *log_decay, int B, int H, int N, double *acs)
 {
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H; ++h) {
             size_t off = ((size_t)b * H + h) * (size_t)N;
-            log_decay_row(dt_p + off, A_log[h], dt_bias[h], N, acs + off);
+            log_decay_row(log_decay ? NULL : dt_p + off, log_decay ? 0.0 : A_log[h],
+                          log_decay ? 0.0 : dt_bias[h], log_decay ? log_decay + off : NULL, N,
+                          acs + off);
         }
+}
+
+/* Value factor of token t: dt_t = softplus(dt_P + dt_bias) when value_dt
+ * (Algorithm 4, V_dt = V (.) dt), else 1. */
+static double value_factor(const float *dt_p, const float *dt_bias, int value_dt, size_t tok, int h)
+{
+    return value_dt ? oracle_softplus((double)dt_p[tok] + (double)dt_bias[h]) : 1.0;
 }
 
 /* Mask entry A^M_ij * M_ij (Algorithm 4): exp(A^CS_i - A^CS_j) when i >= j,
@@ -101,7 +122,8 @@ int oracle_feature(const double *x, int d, int order, double *out)
 /* Quadratic (masked-matrix) form, Algorithm 1 / Algorithm 5, evaluated for a
  * chosen set of rows.  For every (b, h) and every listed row i:
  *     s_ij = q_i . k_j,   w_ij = s_ij^order * A^M_ij * M_ij,
- *     y_i  = sum_j w_ij v_j,   N_i = sum_j w_ij,
+ *     y_i  = sum_j w_ij f_j v_j,   N_i = sum_j w_ij,
+ * with f_j = dt_j under value_dt and 1 otherwise,
  *     y_i /= N_i when normalise != 0,   y_ic += D[h*d + c] * v_ic when D.
  * rows: n_rows row indices (each in [0, N)), or NULL for all N rows.
  * out: [B, H, n_rows, d] (n_rows = N when rows is NULL).
@@ -109,8 +131,8 @@ int oracle_feature(const double *x, int d, int order, double *out)
  * Returns 0, or -1 on a bad argument. */
 int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
                          const float *dt_p, const float *A_log, const float *dt_bias,
-                         const float *D, int B, int H, int N, int d,
-                         int order, int normalise,
+                         const float *D, const float *log_decay, int value_dt,
+                         int B, int H, int N, int d, int order, int normalise,
                          const int *rows, int n_rows,
                          double *out, double *norm_out)
 {
@@ -123,7 +145,7 @@ int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
     int BH = B * H;
     double *acs = (double *)malloc(sizeof(double) * (size_t)BH * (size_t)(N > 0 ? N : 1));
     if (!acs) return -1;
-    oracle_log_decay(dt_p, A_log, dt_bias, B, H, N, acs);
+    oracle_log_decay(dt_p, A_log, dt_bias, log_decay, B, H, N, acs);
 
     long long total = (long long)BH * n_rows;
 #pragma omp parallel for schedule(dynamic, 4)
@@ -145,7 +167,8 @@ int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
             for (int c = 0; c < d; ++c) s += (double)qi[c] * (double)kj[c];
             double score = (order == 1) ? s : s * s;
             double w = score * oracle_mask(acs_row, i, j);
-            for (int c = 0; c < d; ++c) yi[c] += w * (double)vj[c];
+            double wv = w * value_factor(dt_p, dt_bias, value_dt, base + j, h);
+            for (int c = 0; c < d; ++c) yi[c] += wv * (double)vj[c];
             ni += w;
         }
         if (normalise)
@@ -161,8 +184,9 @@ int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
 }
 
 /* Token-by-token recurrent form, Algorithm 6, with the multiplicative decay
- * a_t = exp(A_h * dt_t) of Algorithm 3:
- *     H_up_t = a_t H_up_{t-1} + phi(k_t) v_t^T     (D_phi x d)
+ * a_t = exp(A_h * dt_t) of Algorithm 3 (or exp(log_decay_t), Algorithm 4):
+ *     H_up_t = a_t H_up_{t-1} + phi(k_t) (f_t v_t)^T     (D_phi x d),
+ *     f_t = dt_t under value_dt, else 1
  *     H_dn_t = a_t H_dn_{t-1} + phi(k_t)           (D_phi)
  *     y_t = phi(q_t)^T H_up_t,  N_t = phi(q_t) . H_dn_t,
  * then y_t /= N_t when normalising and y_tc += D[h*d+c] v_tc when D.
@@ -172,8 +196,8 @@ int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
  * Returns 0, or -1 on a bad argument / allocation failure. */
 int oracle_ssd_recurrent(const float *q, const float *k, const float *v,
                          const float *dt_p, const float *A_log, const float *dt_bias,
-                         const float *D, int B, int H, int N, int d,
-                         int order, int normalise,
+                         const float *D, const float *log_decay, int value_dt,
+                         int B, int H, int N, int d, int order, int normalise,
                          double *out, double *norm_out,
                          double *state_out, double *zstate_out)
 {
@@ -198,11 +222,16 @@ int oracle_ssd_recurrent(const float *q, const float *k, const float *v,
             free(Hup); free(Hdn); free(fq); free(fk); free(xq); free(xk);
             continue;
         }
-        double A = -exp((double)A_log[h]);
         size_t base = (size_t)bh * N;
         for (int t = 0; t < N; ++t) {
-            double dt = oracle_softplus((double)dt_p[base + t] + (double)dt_bias[h]);
-            double a = exp(A * dt);
+            double a;
+            if (log_decay) {
+                a = exp((double)log_decay[base + t]);
+            } else {
+                double dt = oracle_softplus((double)dt_p[base + t] + (double)dt_bias[h]);
+                a = exp(-exp((double)A_log[h]) * dt);
+            }
+            double f = value_factor(dt_p, dt_bias, value_dt, base + t, h);
             const float *qt = q + (base + t) * d;
             const float *kt = k + (base + t) * d;
             const float *vt = v + (base + t) * d;
@@ -211,7 +240,7 @@ int oracle_ssd_recurrent(const float *q, const float *k, const float *v,
             oracle_feature(xk, d, order, fk);
             for (int m = 0; m < Dphi; ++m) {
                 double *row = Hup + (size_t)m * d;
-                for (int c = 0; c < d; ++c) row[c] = a * row[c] + fk[m] * (double)vt[c];
+                for (int c = 0; c < d; ++c) row[c] = a * row[c] + fk[m] * f * (double)vt[c];
                 Hdn[m] = a * Hdn[m] + fk[m];
             }
             double *yt = out + (base + t) * d;

@@ -295,3 +295,95 @@ def test_recurrent_final_state_matches_definition():
             zref += w * fk
         np.testing.assert_allclose(st[0, 0], ref, rtol=1e-12, atol=1e-14)
         np.testing.assert_allclose(zst[0, 0], zref, rtol=1e-12, atol=1e-14)
+
+
+# ------------------------------------------- Mamba-2S options (Algorithm 4)
+def test_hand_mamba2s_log_decay_value_dt(golden):
+    """Given per-token log-decays and value discretisation V (.) dt
+    (Algorithm 4), on a 3-token case worked out by hand."""
+    c = golden["mamba2s-log-decay-value-dt"]
+    B, H, N, d = c["B"], c["H"], c["N"], c["d"]
+    q = np.asarray(c["q"], np.float32).reshape(B, H, N, d)
+    k = np.asarray(c["k"], np.float32).reshape(B, H, N, d)
+    v = np.asarray(c["v"], np.float32).reshape(B, H, N, d)
+    ld = np.asarray(c["log_decay"], np.float32).reshape(B, H, N)
+    dt_p = np.asarray(c["dt_p"], np.float32).reshape(B, H, N)
+    dt_bias = np.asarray(c["dt_bias"], np.float32)
+    Dres = np.asarray(c["D"], np.float32)
+    acs = oracle.log_decay(None, None, None, log_decay_in=ld)[0, 0]
+    np.testing.assert_allclose(acs, c["acs"], rtol=1e-7)  # the inputs are float32
+    for e in c["expect"]:
+        D = Dres if e["residual"] else None
+        for form in (oracle.ssd_quadratic, oracle.ssd_recurrent):
+            y, n = form(q, k, v, dt_p if e["value_dt"] else None, None,
+                        dt_bias if e["value_dt"] else None, D, e["order"], e["normalize"],
+                        return_norm=True, log_decay=ld, value_dt=e["value_dt"])
+            np.testing.assert_allclose(y[0, 0], e["y"], rtol=3e-7, err_msg=f"{form.__name__} {e}")
+            if "norm" in e:
+                np.testing.assert_allclose(n[0, 0], e["norm"], rtol=3e-7)
+
+
+def _small(seed, B=2, H=2, N=19, d=3):
+    x = inputs.make_inputs(B, H, N, d, "f32", seed=seed, residual=True)
+    return x
+
+
+@pytest.mark.parametrize("order", [1, 2])
+def test_log_decay_input_matches_a_dt(order):
+    """Passing a_t = -exp(A_log) softplus(dt_p + dt_bias) as the log-decay
+    input reproduces the Algorithm 3 parameterisation."""
+    x = _small(3)
+    dt = np.log1p(np.exp(-np.abs(x["dt_p"].astype(np.float64) + x["dt_bias"][None, :, None]))) + \
+        np.maximum(x["dt_p"].astype(np.float64) + x["dt_bias"][None, :, None], 0.0)
+    ld = (-np.exp(x["A_log"].astype(np.float64))[None, :, None] * dt).astype(np.float32)
+    for norm in (False, True):
+        ref = oracle.ssd_quadratic(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"],
+                                   order, norm)
+        got = oracle.ssd_quadratic(x["q"], x["k"], x["v"], None, None, None, x["D"], order, norm,
+                                   log_decay=ld)
+        np.testing.assert_allclose(got, ref, rtol=2e-5, atol=1e-6)
+
+
+@pytest.mark.parametrize("order", [1, 2])
+def test_value_dt_is_prescaled_values(order):
+    """value_dt equals the plain operator on V pre-scaled by dt per token
+    (the caller-side form of Algorithm 4's V_dt); the normaliser and the
+    residual (here off) do not see dt."""
+    x = _small(4)
+    z = x["dt_p"].astype(np.float64) + x["dt_bias"][None, :, None]
+    dt = np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+    v_dt = (x["v"].astype(np.float64) * dt[..., None]).astype(np.float32)
+    for norm in (False, True):
+        got, n_got = oracle.ssd_quadratic(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], None,
+                                          order, norm, value_dt=True, return_norm=True)
+        ref, n_ref = oracle.ssd_quadratic(x["q"], x["k"], v_dt, x["dt_p"], x["A_log"], x["dt_bias"], None,
+                                          order, norm, return_norm=True)
+        np.testing.assert_allclose(got, ref, rtol=2e-6, atol=1e-7)
+        np.testing.assert_allclose(n_got, n_ref, rtol=1e-14)
+
+
+@pytest.mark.parametrize("order,norm", [(1, False), (2, True), (2, False)])
+def test_options_quadratic_equals_recurrent(order, norm):
+    """Algorithm 5 and Algorithm 6 agree with both options on."""
+    x = _small(5, N=23)
+    rng = np.random.default_rng(11)
+    ld = (-rng.uniform(0.0, 0.7, size=x["dt_p"].shape)).astype(np.float32)
+    kw = dict(log_decay=ld, value_dt=True)
+    a = oracle.ssd_quadratic(x["q"], x["k"], x["v"], x["dt_p"], None, x["dt_bias"], x["D"], order, norm, **kw)
+    b = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], None, x["dt_bias"], x["D"], order, norm, **kw)
+    np.testing.assert_allclose(a, b, rtol=1e-11, atol=1e-12)
+
+
+def test_zero_log_decay_value_dt_prefix_sums():
+    """With a zero log-decay the mask is all ones below the diagonal, so the
+    operator is causal linear attention over V (.) dt: prefix sums."""
+    x = _small(6, B=1, H=1, N=17, d=4)
+    ld = np.zeros_like(x["dt_p"])
+    y = oracle.ssd_quadratic(x["q"], x["k"], x["v"], x["dt_p"], None, x["dt_bias"], None, 1, False,
+                             log_decay=ld, value_dt=True)[0, 0]
+    z = x["dt_p"][0, 0].astype(np.float64) + float(x["dt_bias"][0])
+    dt = np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+    kv = np.einsum("nc,ne->nce", x["k"][0, 0].astype(np.float64), x["v"][0, 0].astype(np.float64) * dt[:, None])
+    S = np.cumsum(kv, axis=0)
+    ref = np.einsum("nc,nce->ne", x["q"][0, 0].astype(np.float64), S)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
