@@ -62,15 +62,25 @@ typedef enum {
     SSD_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssd_workspace_bytes() */
     SSD_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed */
     SSD_ERR_TIMEOUT = 9,     /* a device-side wait ran out (read back from the workspace) */
-    SSD_ERR_UNSUPPORTED = 10 /* a valid combination this build has no kernel for */
+    SSD_ERR_UNSUPPORTED = 10, /* a valid combination this build has no kernel for */
+    SSD_ERR_FLAGS = 11       /* unknown bits in the flags of ssd_fwd_ex() */
 } ssd_status;
+
+/* Option bits of ssd_fwd_ex(). */
+typedef enum {
+    /* Value discretisation (2Mamba2Furious, Algorithm 4: V_dt = V (.) dt):
+     * the contraction uses v_t * dt_t, dt_t = softplus(dt_p[t] + dt_bias[h]).
+     * The row normaliser and the D residual still use the raw scores and the
+     * raw v. */
+    SSD_VALUE_DT = 1
+} ssd_flags;
 
 /* Element type of q, k, v and out. */
 typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
 
 /*
- * Bytes of device workspace ssd_fwd() needs for this problem.  Depends only
- * on the arguments.  Returns 0 when the arguments are invalid (ssd_fwd
+ * Bytes of device workspace ssd_fwd() and ssd_fwd_ex() need for this problem
+ * (any normalize setting, any flags).  Depends only on the arguments.  Returns 0 when the arguments are invalid (ssd_fwd
  * would reject them).  Supported: B, H >= 1; N >= 1 with N % chunk == 0;
  * d_h in {16, 32, 64}; order in {1, 2}; chunk in {64, 128, 256}.
  */
@@ -100,6 +110,30 @@ int ssd_fwd(const void *q, const void *k, const void *v,
             int order, int normalize, int chunk,
             void *out, void *workspace, size_t workspace_bytes,
             void *stream);
+
+/*
+ * The operator with the Mamba-2S options of 2Mamba2Furious Algorithm 4.
+ * Same arguments and conventions as ssd_fwd(), plus:
+ *   log_decay  device, [B, H, N] fp32, or NULL.  When given, the per-token
+ *              log-decay a_t = log_decay[t] (natural log, normally <= 0, e.g.
+ *              -softplus(h W_A)) replaces A_h * dt_t, so the mask is
+ *              exp(cumsum(a)_i - cumsum(a)_j); A_log is then not read and may
+ *              be NULL.
+ *   flags      0 or SSD_VALUE_DT.  dt_p and dt_bias must be given when
+ *              log_decay is NULL or SSD_VALUE_DT is set; otherwise they may
+ *              be NULL.
+ * ssd_fwd(...) is ssd_fwd_ex(..., log_decay = NULL, flags = 0).
+ * Paths: order 1 and order-2 decay options run on the tensor-core paths; order
+ * 2 with SSD_VALUE_DT runs on the SIMT path.
+ * Errors as ssd_fwd(), plus SSD_ERR_FLAGS for unknown flag bits.
+ */
+int ssd_fwd_ex(const void *q, const void *k, const void *v,
+               const float *dt_p, const float *A_log, const float *dt_bias,
+               const float *D, const float *log_decay,
+               int B, int H, int N, int d_h, int dtype,
+               int order, int normalize, int chunk, int flags,
+               void *out, void *workspace, size_t workspace_bytes,
+               void *stream);
 
 /*
  * ssd_fwd() with the activations in HOST memory: enqueues on `stream` the

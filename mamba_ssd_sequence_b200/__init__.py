@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libssd.so")
 
 SSD_F32 = 0
 SSD_BF16 = 1
+SSD_VALUE_DT = 1  # ssd_fwd_ex flag: contract with v * dt (Algorithm 4, V_dt)
 PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2"}
 
 _lib = None
@@ -47,6 +48,8 @@ def load_library():
     lib.ssd_workspace_bytes.restype = sz
     lib.ssd_fwd.argtypes = [vp] * 7 + [ci] * 8 + [vp, vp, sz, vp]
     lib.ssd_fwd.restype = ci
+    lib.ssd_fwd_ex.argtypes = [vp] * 8 + [ci] * 9 + [vp, vp, sz, vp]
+    lib.ssd_fwd_ex.restype = ci
     lib.ssd_fwd_host.argtypes = [vp] * 7 + [ci] * 8 + [vp] + [vp] * 8 + [vp, sz, vp]
     lib.ssd_fwd_host.restype = ci
     lib.ssd_chunk_cumsum.argtypes = [vp] * 3 + [ci] * 4 + [vp, vp, vp]
@@ -119,14 +122,16 @@ def alloc_workspace(B, H, N, d_h, dtype, order, chunk, device=None):
 
 
 def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk: int,
-            out=None, workspace=None, stream=None):
-    """y = SSD forward (include/ssd.h, ssd_fwd) on CUDA tensors.
+            out=None, workspace=None, stream=None, log_decay=None, value_dt: bool = False):
+    """y = SSD forward (include/ssd.h: ssd_fwd, or ssd_fwd_ex when a Mamba-2S
+    option is used) on CUDA tensors.
 
     q, k, v: [B, H, N, d_h] float32 or bfloat16; dt_p: [B, H, N] float32;
-    A_log, dt_bias: [H] float32; D: [H*d_h] float32 or None.  Returns `out`
-    ([B, H, N, d_h], the input dtype), allocating it and the workspace with
-    torch when not given.  Asynchronous on `stream` (default: the current
-    torch stream)."""
+    A_log, dt_bias: [H] float32; D: [H*d_h] float32 or None.  log_decay:
+    [B, H, N] float32 per-token log-decay replacing A*dt (A_log may then be
+    None); value_dt: contract with v * dt.  Returns `out` ([B, H, N, d_h], the
+    input dtype), allocating it and the workspace with torch when not given.
+    Asynchronous on `stream` (default: the current torch stream)."""
     import torch
     B, H, N, d = q.shape
     dt = _dtype_code(q)
@@ -134,11 +139,20 @@ def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk
         out = torch.empty_like(q)
     if workspace is None:
         workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device)
-    rc = load_library().ssd_fwd(
-        _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
-        B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk),
-        _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
-    _check(rc, "ssd_fwd")
+    lib = load_library()
+    if log_decay is None and not value_dt:
+        rc = lib.ssd_fwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
+            B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk),
+            _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+        _check(rc, "ssd_fwd")
+    else:
+        rc = lib.ssd_fwd_ex(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
+            _ptr(log_decay), B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk),
+            SSD_VALUE_DT if value_dt else 0, _ptr(out), _ptr(workspace), workspace.numel(),
+            _stream_handle(stream))
+        _check(rc, "ssd_fwd_ex")
     return out
 
 

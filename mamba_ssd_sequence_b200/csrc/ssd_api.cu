@@ -32,14 +32,14 @@ static size_t simt_total(int B, int H, int N, int d, int order, int chunk, Plan 
 }
 
 bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
-               Plan *plan) {
+               int value_dt, Plan *plan) {
     if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
     Plan p{};
     if (order == 1 && !normalize && tc_order1_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER1;
         p.n_launches = 3;
         tc_order1_layout(B, H, N, chunk, &p);
-    } else if (order == 2 && tc_order2_supports(B, H, N, d, dtype, chunk)) {
+    } else if (order == 2 && !value_dt && tc_order2_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER2;
         p.n_launches = 1;
         p.acs_off = p.lam_off = p.state_off = kStatusBytes;
@@ -60,44 +60,65 @@ using namespace ssd;
 extern "C" {
 
 size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk) {
-    // the size covers both settings of `normalize`, which can select different paths
-    Plan p0, p1;
-    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, &p0)) return 0;
-    if (!make_plan(B, H, N, d_h, dtype, order, 1, chunk, &p1)) return 0;
-    return p0.total > p1.total ? p0.total : p1.total;
+    // the size covers every setting of `normalize` and of the flags, which can
+    // select different paths
+    size_t need = 0;
+    for (int norm = 0; norm < 2; ++norm)
+        for (int vdt = 0; vdt < 2; ++vdt) {
+            Plan p;
+            if (!make_plan(B, H, N, d_h, dtype, order, norm, chunk, vdt, &p)) return 0;
+            if (p.total > need) need = p.total;
+        }
+    return need;
 }
 
 int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
                  int *n_launches) {
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, &p)) return -1;
+    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, 0, &p)) return -1;
     if (n_launches) *n_launches = p.n_launches;
     return p.path;
+}
+
+int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,
+               const float *A_log, const float *dt_bias, const float *D, const float *log_decay,
+               int B, int H, int N, int d_h, int dtype, int order, int normalize, int chunk,
+               int flags, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
+    const int value_dt = (flags & SSD_VALUE_DT) ? 1 : 0;
+    if (!q || !k || !v || !out) return SSD_ERR_NULL;
+    const bool need_dt = !log_decay || value_dt;  // dt feeds the decay and/or the values
+    if (need_dt && (!dt_p || !dt_bias)) return SSD_ERR_NULL;
+    if (!log_decay && !A_log) return SSD_ERR_NULL;
+    int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
+    if (rc != SSD_OK) return rc;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    const void *ptrs[] = {q, k, v, out, dt_p, A_log, dt_bias, D, log_decay};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
+    Plan p;
+    if (!make_plan(B, H, N, d_h, dtype, order, normalize, chunk, value_dt, &p))
+        return SSD_ERR_UNSUPPORTED;
+    if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
+    FwdArgs a{q, k, v, need_dt ? dt_p : nullptr, log_decay ? nullptr : A_log,
+              need_dt ? dt_bias : nullptr, D, log_decay, value_dt, B, H, N, d_h, dtype, order,
+              normalize ? 1 : 0, chunk, out, workspace, workspace_bytes,
+              static_cast<cudaStream_t>(stream)};
+    switch (p.path) {
+    case PATH_TC_ORDER1: return launch_tc_order1(a, p);
+    case PATH_TC_ORDER2: return launch_tc_order2(a, p);
+    default: return launch_simt(a, p);
+    }
 }
 
 int ssd_fwd(const void *q, const void *k, const void *v, const float *dt_p,
             const float *A_log, const float *dt_bias, const float *D, int B, int H, int N,
             int d_h, int dtype, int order, int normalize, int chunk, void *out,
             void *workspace, size_t workspace_bytes, void *stream) {
-    if (!q || !k || !v || !dt_p || !A_log || !dt_bias || !out) return SSD_ERR_NULL;
-    int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
-    if (rc != SSD_OK) return rc;
-    if (!workspace) return SSD_ERR_WORKSPACE;
-    const void *ptrs[] = {q, k, v, dt_p, A_log, dt_bias, out};
-    for (const void *p : ptrs)
-        if (!aligned16(p)) return SSD_ERR_ALIGN;
-    if (D && !aligned16(D)) return SSD_ERR_ALIGN;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
-    Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, normalize, chunk, &p)) return SSD_ERR_UNSUPPORTED;
-    if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
-    FwdArgs a{q, k, v, dt_p, A_log, dt_bias, D, B, H, N, d_h, dtype, order, normalize ? 1 : 0,
-              chunk, out, workspace, workspace_bytes, static_cast<cudaStream_t>(stream)};
-    switch (p.path) {
-    case PATH_TC_ORDER1: return launch_tc_order1(a, p);
-    case PATH_TC_ORDER2: return launch_tc_order2(a, p);
-    default: return launch_simt(a, p);
-    }
+    if (!dt_p || !A_log || !dt_bias) return SSD_ERR_NULL;
+    return ssd_fwd_ex(q, k, v, dt_p, A_log, dt_bias, D, nullptr, B, H, N, d_h, dtype, order,
+                      normalize, chunk, 0, out, workspace, workspace_bytes, stream);
 }
 
 int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
@@ -141,7 +162,7 @@ int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias
     if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_CHUNK;
     if (B < 1 || H < 1 || N < 1 || N % chunk != 0 || (long long)B * H > 65535)
         return SSD_ERR_SHAPE;
-    return launch_chunk_cumsum(dt_p, A_log, dt_bias, B, H, N, chunk, acs, chunk_sum, nullptr,
+    return launch_chunk_cumsum(dt_p, A_log, dt_bias, nullptr, B, H, N, chunk, acs, chunk_sum, nullptr,
                                static_cast<cudaStream_t>(stream));
 }
 
@@ -168,6 +189,7 @@ const char *ssd_status_str(int status) {
     case SSD_ERR_CUDA: return "SSD_ERR_CUDA: CUDA runtime or launch error";
     case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT: a bounded device-side wait gave up";
     case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED: no kernel for this combination";
+    case SSD_ERR_FLAGS: return "SSD_ERR_FLAGS: unknown bits in the flags of ssd_fwd_ex";
     default: return "unknown ssd status";
     }
 }

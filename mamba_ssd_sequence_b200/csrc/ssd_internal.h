@@ -14,6 +14,8 @@ namespace ssd {
 struct FwdArgs {
     const void *q, *k, *v;
     const float *dt_p, *A_log, *dt_bias, *D;
+    const float *log_decay;  // per-token log-decay, or NULL (A * dt)
+    int value_dt;            // contract with v * dt
     int B, H, N, d, dtype, order, normalize, chunk;
     void *out;
     void *workspace;
@@ -39,12 +41,12 @@ enum Path { PATH_SIMT = 0, PATH_TC_ORDER1 = 1, PATH_TC_ORDER2 = 2 };
 struct Plan {
     int path;
     int n_launches;
-    size_t acs_off, lam_off, state_off, aux_off, total;
+    size_t acs_off, lam_off, state_off, aux_off, vfac_off, total;
 };
 
 // Fills `plan` for validated arguments; returns false if no kernel exists.
 bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
-               Plan *plan);
+               int value_dt, Plan *plan);
 
 // Path launchers (each returns an ssd_status).
 int launch_simt(const FwdArgs &a, const Plan &p);
@@ -57,8 +59,9 @@ void tc_order1_layout(int B, int H, int N, int chunk, Plan *p);
 
 // Kernel (a): chunk-local inclusive cumsum of A*dt and the chunk totals.
 // When `status` is non-NULL, block (0,0) thread 0 clears it.
+// log_decay (may be NULL) replaces A*dt by a given per-token log-decay.
 int launch_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias,
-                        int B, int H, int N, int chunk, float *acs, float *chunk_sum,
-                        DeviceStatus *status, cudaStream_t stream);
+                        const float *log_decay, int B, int H, int N, int chunk, float *acs,
+                        float *chunk_sum, DeviceStatus *status, cudaStream_t stream);
 
 }  // namespace ssd

@@ -19,6 +19,9 @@
 //                       the same for the row sum, then /row sum, + D*v.
 // phi is the identity (order 1) or the tensor square (order 2), whose inner
 // product with phi(k) is (q.k)^2.
+// Mamba-2S options (Algorithm 4): a given per-token log-decay replaces A*dt
+// in (a); with value discretisation, v_j is multiplied by dt_j in (b) and
+// (d) (not in the normaliser column, not in the D residual).
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -45,7 +48,8 @@ __device__ __forceinline__ float softplus_f(float x) {
 // grid (n_chunks, B*H), block = chunk threads (64, 128 or 256).
 __global__ void chunk_cumsum_kernel(const float *__restrict__ dt_p,
                                     const float *__restrict__ A_log,
-                                    const float *__restrict__ dt_bias, int H, int N,
+                                    const float *__restrict__ dt_bias,
+                                    const float *__restrict__ log_decay, int H, int N,
                                     int chunk, float *__restrict__ acs,
                                     float *__restrict__ chunk_sum,
                                     DeviceStatus *status) {
@@ -57,8 +61,7 @@ __global__ void chunk_cumsum_kernel(const float *__restrict__ dt_p,
         status->detail = 0;
     }
     const size_t idx = (size_t)bh * N + (size_t)c * chunk + t;
-    const float A = -expf(A_log[h]);
-    float x = A * softplus_f(dt_p[idx] + dt_bias[h]);
+    float x = log_decay ? log_decay[idx] : -expf(A_log[h]) * softplus_f(dt_p[idx] + dt_bias[h]);
     // inclusive warp scan, then add the totals of the warps before
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -83,11 +86,14 @@ constexpr int kMaxOut = 5;   // ceil(16 * 65 / 256)
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
-                   const float *__restrict__ acs, const float *__restrict__ lam, int N,
-                   int d, int order, int chunk, float *__restrict__ states) {
+                   const float *__restrict__ acs, const float *__restrict__ lam,
+                   const float *__restrict__ dt_p, const float *__restrict__ dt_bias,
+                   int value_dt, int H, int N, int d, int order, int chunk,
+                   float *__restrict__ states) {
     __shared__ float ks[kJT * 64];
     __shared__ float vs[kJT * 64];
     __shared__ float ws[kJT];
+    __shared__ float fs[kJT];  // value factor dt_j (1 without value discretisation)
     const int mt = blockIdx.x, c = blockIdx.y, bh = blockIdx.z;
     const int nc = N / chunk;
     const int Dphi = order == 1 ? d : d * d;
@@ -114,7 +120,11 @@ chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
             ks[jj * d + cc] = load_elem(k, (tok0 + j0 + jj) * d + cc);
             vs[jj * d + cc] = load_elem(v, (tok0 + j0 + jj) * d + cc);
         }
-        if (threadIdx.x < kJT) ws[threadIdx.x] = expf(lam_c - acs[tok0 + j0 + threadIdx.x]);
+        if (threadIdx.x < kJT) {
+            const size_t tj = tok0 + j0 + threadIdx.x;
+            ws[threadIdx.x] = expf(lam_c - acs[tj]);
+            fs[threadIdx.x] = value_dt ? softplus_f(dt_p[tj] + dt_bias[(bh % H)]) : 1.0f;
+        }
         __syncthreads();
 #pragma unroll
         for (int r = 0; r < kMaxOut; ++r) {
@@ -125,7 +135,7 @@ chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
             for (int jj = 0; jj < kJT; ++jj) {
                 float f = ks[jj * d + ma];
                 if (mb >= 0) f *= ks[jj * d + mb];
-                float vv = cc < d ? vs[jj * d + cc] : 1.0f;
+                float vv = cc < d ? vs[jj * d + cc] * fs[jj] : 1.0f;
                 s = fmaf(ws[jj] * f, vv, s);
             }
             acc[r] = s;
@@ -163,11 +173,14 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
                     const T *__restrict__ v, const float *__restrict__ acs,
-                    const float *__restrict__ states, const float *__restrict__ D, int H,
-                    int N, int d, int order, int normalize, int chunk, T *__restrict__ out) {
+                    const float *__restrict__ states, const float *__restrict__ D,
+                    const float *__restrict__ dt_p, const float *__restrict__ dt_bias,
+                    int value_dt, int H, int N, int d, int order, int normalize, int chunk,
+                    T *__restrict__ out) {
     __shared__ float qs[kTI * 64];
     __shared__ float ks[kJT * 64];
     __shared__ float vs[kJT * 64];
+    __shared__ float fs[kJT];  // value factor dt_j (1 without value discretisation)
     __shared__ float ps[kTI * kJT];
     __shared__ float ss[kTM2 * 65];
     __shared__ float ys[kTI * 65];
@@ -205,6 +218,8 @@ chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
             ks[jj * d + cc] = load_elem(k, (tok0 + j0 + jj) * d + cc);
             vs[jj * d + cc] = load_elem(v, (tok0 + j0 + jj) * d + cc);
         }
+        if (threadIdx.x < kJT)
+            fs[threadIdx.x] = value_dt ? softplus_f(dt_p[tok0 + j0 + threadIdx.x] + dt_bias[h]) : 1.0f;
         __syncthreads();
         for (int e = threadIdx.x; e < kTI * kJT; e += kThreads) {
             int ii = e / kJT, jj = e % kJT;
@@ -225,7 +240,7 @@ chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
             float s = acc[r];
             const int ii = oi[r], cc = oc[r];
             for (int jj = 0; jj < kJT; ++jj) {
-                float vv = cc < d ? vs[jj * d + cc] : 1.0f;
+                float vv = cc < d ? vs[jj * d + cc] * fs[jj] : 1.0f;
                 s = fmaf(ps[ii * kJT + jj], vv, s);
             }
             acc[r] = s;
@@ -283,33 +298,34 @@ int run_simt(const FwdArgs &a, const Plan &p) {
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(ws);
     const int BH = a.B * a.H, nc = a.N / a.chunk;
     const int Dphi = a.order == 1 ? a.d : a.d * a.d;
-    int rc = launch_chunk_cumsum(a.dt_p, a.A_log, a.dt_bias, a.B, a.H, a.N, a.chunk, acs, lam,
-                                 status, a.stream);
+    int rc = launch_chunk_cumsum(a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.B, a.H, a.N, a.chunk,
+                                 acs, lam, status, a.stream);
     if (rc != SSD_OK) return rc;
     const T *q = static_cast<const T *>(a.q);
     const T *k = static_cast<const T *>(a.k);
     const T *v = static_cast<const T *>(a.v);
     dim3 g1((Dphi + kStateTM - 1) / kStateTM, nc, BH);
-    chunk_state_kernel<T><<<g1, kThreads, 0, a.stream>>>(k, v, acs, lam, a.N, a.d, a.order,
+    chunk_state_kernel<T><<<g1, kThreads, 0, a.stream>>>(k, v, acs, lam, a.dt_p, a.dt_bias,
+                                                         a.value_dt, a.H, a.N, a.d, a.order,
                                                          a.chunk, states);
     const size_t elems = (size_t)Dphi * (a.d + 1);
     dim3 g2((unsigned)((elems + 255) / 256), BH);
     state_scan_kernel<<<g2, 256, 0, a.stream>>>(states, lam, nc, elems, BH);
     dim3 g3(a.chunk / kTI, nc, BH);
     chunk_output_kernel<T><<<g3, kThreads, 0, a.stream>>>(
-        q, k, v, acs, states, a.D, a.H, a.N, a.d, a.order, a.normalize, a.chunk,
-        static_cast<T *>(a.out));
+        q, k, v, acs, states, a.D, a.dt_p, a.dt_bias, a.value_dt, a.H, a.N, a.d, a.order,
+        a.normalize, a.chunk, static_cast<T *>(a.out));
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
 }  // namespace
 
-int launch_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias, int B,
-                        int H, int N, int chunk, float *acs, float *chunk_sum,
-                        DeviceStatus *status, cudaStream_t stream) {
+int launch_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias,
+                        const float *log_decay, int B, int H, int N, int chunk, float *acs,
+                        float *chunk_sum, DeviceStatus *status, cudaStream_t stream) {
     dim3 grid(N / chunk, B * H);
-    chunk_cumsum_kernel<<<grid, chunk, 0, stream>>>(dt_p, A_log, dt_bias, H, N, chunk, acs,
-                                                    chunk_sum, status);
+    chunk_cumsum_kernel<<<grid, chunk, 0, stream>>>(dt_p, A_log, dt_bias, log_decay, H, N, chunk,
+                                                    acs, chunk_sum, status);
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -19,6 +19,9 @@
 // both factors <= 1 because acs falls along the chunk, so one exp2 per row and
 // per column replaces one per element; diagonal blocks take the exact
 // per-element exp2.  Every wait is bounded; a timeout sets the status word.
+// Mamba-2S options (Algorithm 4): a given per-token log-decay replaces A dt
+// in (1); with value discretisation the factor dt_j multiplies key j's
+// weight in U (through K') and in P (through the per-key factors).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -99,7 +102,8 @@ template <int C>
 __global__ void __launch_bounds__(StateCfg<C>::THREADS, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const float *__restrict__ dt_p, const float *__restrict__ A_log,
-                   const float *__restrict__ dt_bias, int H, int N, int n_chunks, float *__restrict__ acs_out,
+                   const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int value_dt,
+                   int H, int N, int n_chunks, float *__restrict__ acs_out, float *__restrict__ vfac_out,
                    float *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status) {
     using K = StateCfg<C>;
     constexpr int NG = K::NG;
@@ -202,20 +206,25 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         const int bar = 1 + gi;
         bool failed = false;
 
+        // raw inputs of a chunk, fetched one chunk ahead: dt projections (when
+        // dt is used), given log-decays (when given), A_log and dt_bias
         struct Raw {
-            float dt[KP], alog, bias;
+            float dt[KP], ld[KP], alog, bias;
         };
         auto fetch = [&](int t) -> Raw {
             Raw x;
 #pragma unroll
-            for (int e = 0; e < KP; ++e) x.dt[e] = 0.0f;
+            for (int e = 0; e < KP; ++e) x.dt[e] = x.ld[e] = 0.0f;
             x.alog = x.bias = 0.0f;
             if (t >= n_chunks) return x;
             const int h = (t / nc) % H;
-            x.alog = __ldg(A_log + h);
-            x.bias = __ldg(dt_bias + h);
+            if (A_log) x.alog = __ldg(A_log + h);
+            if (dt_bias) x.bias = __ldg(dt_bias + h);
 #pragma unroll
-            for (int e = 0; e < KP; ++e) x.dt[e] = __ldg(dt_p + (size_t)t * C + KP * gt + e);
+            for (int e = 0; e < KP; ++e) {
+                if (dt_p) x.dt[e] = __ldg(dt_p + (size_t)t * C + KP * gt + e);
+                if (log_decay) x.ld[e] = __ldg(log_decay + (size_t)t * C + KP * gt + e);
+            }
             return x;
         };
 
@@ -227,12 +236,14 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             raw_next = fetch(t + NG * gridDim.x);
             // ---- decay: inclusive scan of A dt over the chunk (log2 units)
             const float A2 = -expf(raw.alog) * kLog2e;
-            float a[KP];
+            float a[KP], vf[KP];
             float run = 0.0f;
 #pragma unroll
             for (int e = 0; e < KP; ++e) {
-                run += A2 * softplus_f(raw.dt[e] + raw.bias);
+                const float dt = (value_dt || !log_decay) ? softplus_f(raw.dt[e] + raw.bias) : 0.0f;
+                run += log_decay ? raw.ld[e] * kLog2e : A2 * dt;
                 a[e] = run;
+                vf[e] = value_dt ? dt : 1.0f;
             }
             float incl = run;
 #pragma unroll
@@ -253,7 +264,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             for (int e = 0; e < KP; ++e) {
                 const float acs = pre + a[e];
                 acs_out[(size_t)t * C + KP * gt + e] = acs;
-                misc->wk[gi][KP * gt + e] = ex2_approx(lam - acs);
+                if (value_dt) vfac_out[(size_t)t * C + KP * gt + e] = vf[e];
+                misc->wk[gi][KP * gt + e] = ex2_approx(lam - acs) * vf[e];
             }
             if (gt == 0) lam_out[t] = lam;
             // ---- K'_j = 2^(lam - acs_j) k_j in place: eight lanes per 128-byte row
@@ -382,7 +394,7 @@ struct ScanCfg {
     static constexpr uint32_t V_OFF = H_OFF + kHinBytes;
     static constexpr uint32_t STAGE = V_OFF + NKB * kBox;
     static constexpr uint32_t MISC_OFF = STAGES * STAGE;
-    static constexpr uint32_t MISC_BYTES = 20 * NG * C + 1024;
+    static constexpr uint32_t MISC_BYTES = 28 * NG * C + 1024;
     static constexpr uint32_t SMEM = MISC_OFF + MISC_BYTES + 1024;
     // TMEM: C = 128: S' buffers at 0 and 192 (keys at +0, Z at +128);
     //       C = 256: keys k at 128 (2 - nkb) + k, Z at 256.  Y buffers at 384, 448.
@@ -397,7 +409,8 @@ template <int C>
 struct ScanMisc {
     static constexpr int NG = ScanCfg<C>::NG;
     float acs[NG][2][C];
-    float colf[NG][2][C];   // 2^(acs_r - acs_j), r the last key of j's 32-key block
+    float colf[NG][2][C];   // 2^(acs_r - acs_j) f_j, r the last key of j's 32-key block
+    float vf[NG][2][C];     // value factor f_j of key j (dt_j, or 1)
     float dres[NG][2][64];  // D of the tile's head
     uint64_t stage_full[ScanCfg<C>::STAGES], stage_empty[ScanCfg<C>::STAGES];
     uint64_t s_full[ScanCfg<C>::NSB], p_full[NG][ScanCfg<C>::NKB], y_full[2], ep_done[2];
@@ -435,8 +448,8 @@ __global__ void __launch_bounds__(ScanCfg<C>::THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
                   const __nv_bfloat16 *__restrict__ vglob, __nv_bfloat16 *__restrict__ out,
-                  const float *__restrict__ acs_in, const float *__restrict__ Dres, int H, int N,
-                  int n_tiles, DeviceStatus *status) {
+                  const float *__restrict__ acs_in, const float *__restrict__ vfac_in,
+                  const float *__restrict__ Dres, int H, int N, int n_tiles, DeviceStatus *status) {
     using K = ScanCfg<C>;
     constexpr int NG = K::NG;
     extern __shared__ uint8_t smem_raw[];
@@ -610,14 +623,18 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         // Raw inputs of a tile, fetched one tile ahead: acs of key ct and four entries of D.
         struct Raw {
-            float acs;
+            float acs, vf;
             float4 d;
         };
         auto fetch = [&](int i) -> Raw {
-            Raw x{0.0f, make_float4(0.f, 0.f, 0.f, 0.f)};
+            Raw x{0.0f, 1.0f, make_float4(0.f, 0.f, 0.f, 0.f)};
             if (i >= my_tiles) return x;
             const TileIdx ti = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
-            if (ct < 128 * (ti.rb + 1)) x.acs = __ldg(acs_in + (size_t)ti.bh * N + (size_t)ti.c * C + ct);
+            if (ct < 128 * (ti.rb + 1)) {
+                const size_t key = (size_t)ti.bh * N + (size_t)ti.c * C + ct;
+                x.acs = __ldg(acs_in + key);
+                if (vfac_in) x.vf = __ldg(vfac_in + key);
+            }
             if (Dres && ct < 16) x.d = __ldg(reinterpret_cast<const float4 *>(Dres + (ti.bh % H) * kD) + ct);
             return x;
         };
@@ -644,7 +661,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const float aref = __shfl_sync(0xffffffffu, raw.acs, 31);
             if (ct < C) {
                 misc->acs[gi][slot][ct] = raw.acs;
-                misc->colf[gi][slot][ct] = ex2_approx(aref - raw.acs);
+                misc->colf[gi][slot][ct] = ex2_approx(aref - raw.acs) * raw.vf;
+                misc->vf[gi][slot][ct] = raw.vf;
             }
             // ---- S of this tile
             bool bad = !mbar_wait_abortable(&misc->s_full[sb], (i / K::NSB) & 1, abort_flag);
@@ -691,11 +709,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 pk[2 * e4 + 1] = pack_bf16x2(p1.x, p1.y);
                             }
                         } else {
+                            const float *vfk = misc->vf[gi][slot];
 #pragma unroll
                             for (int e = 0; e < 32; e += 2) {
                                 const int j = k0 + e;
-                                float p0 = sv[e] * ex2_approx(ai - acs[j]);
-                                float p1 = sv[e + 1] * ex2_approx(ai - acs[j + 1]);
+                                float p0 = sv[e] * ex2_approx(ai - acs[j]) * vfk[j];
+                                float p1 = sv[e + 1] * ex2_approx(ai - acs[j + 1]) * vfk[j + 1];
                                 if (j > ir) p0 = 0.0f;
                                 if (j + 1 > ir) p1 = 0.0f;
                                 pk[e >> 1] = pack_bf16x2(p0, p1);
@@ -818,6 +837,7 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(ws);
     float *lam = reinterpret_cast<float *>(ws + p.lam_off);
     float *acs = reinterpret_cast<float *>(ws + p.acs_off);
+    float *vfac = a.value_dt ? reinterpret_cast<float *>(ws + p.vfac_off) : nullptr;
     float *U = reinterpret_cast<float *>(ws + p.state_off);
     __nv_bfloat16 *hin = reinterpret_cast<__nv_bfloat16 *>(ws + p.aux_off);
     CUtensorMap tq, tk, tv, th;
@@ -833,7 +853,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
 
     const int n_chunks = BH * nc;
     chunk_state_kernel<C><<<n_chunks < sms ? n_chunks : sms, StateCfg<C>::THREADS, StateCfg<C>::SMEM, a.stream>>>(
-        tk, tv, a.dt_p, a.A_log, a.dt_bias, a.H, a.N, n_chunks, acs, U, lam, status);
+        tk, tv, a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N, n_chunks, acs, vfac, U, lam,
+        status);
     // The state pass and the chunk scan are launched as programmatic dependents:
     // their CTAs may start while the previous kernel drains, and each waits
     // (griddepcontrol.wait) before it reads that kernel's results.
@@ -858,8 +879,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c3.attrs = pdl;
     c3.numAttrs = 1;
     if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, static_cast<const __nv_bfloat16 *>(a.v),
-                           static_cast<__nv_bfloat16 *>(a.out), (const float *)acs, a.D, a.H, a.N, n_tiles,
-                           status) != cudaSuccess)
+                           static_cast<__nv_bfloat16 *>(a.out), (const float *)acs, (const float *)vfac, a.D,
+                           a.H, a.N, n_tiles, status) != cudaSuccess)
         return SSD_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
@@ -870,13 +891,14 @@ bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk) {
     return dtype == SSD_BF16 && d == kD && (chunk == 128 || chunk == 256) && (long long)B * H * N < (1ll << 31);
 }
 
-// lam (n_chunks floats), acs (B H N floats), U (n_chunks x 64 x 64 fp32),
-// hin (n_chunks x 64 x 64 bf16)
+// lam (n_chunks floats), acs and vfac (B H N floats each), U (n_chunks x 64
+// x 64 fp32), hin (n_chunks x 64 x 64 bf16)
 void tc_order1_layout(int B, int H, int N, int chunk, Plan *p) {
     const size_t n = (size_t)B * H * (N / chunk);
     p->lam_off = kStatusBytes;
     p->acs_off = align_up(p->lam_off + n * sizeof(float), 256);
-    p->state_off = align_up(p->acs_off + (size_t)B * H * N * sizeof(float), 256);
+    p->vfac_off = align_up(p->acs_off + (size_t)B * H * N * sizeof(float), 256);
+    p->state_off = align_up(p->vfac_off + (size_t)B * H * N * sizeof(float), 256);
     p->aux_off = align_up(p->state_off + n * 4096 * sizeof(float), 256);
     p->total = align_up(p->aux_off + n * 4096 * 2, 256);
 }

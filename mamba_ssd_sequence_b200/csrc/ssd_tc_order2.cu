@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
                  const float *__restrict__ dt_p, const float *__restrict__ A_log,
-                 const float *__restrict__ dt_bias, const float *__restrict__ Dres, int H, int N,
+                 const float *__restrict__ dt_bias, const float *__restrict__ Dres,
+                 const float *__restrict__ log_decay, int H, int N,
                  int normalize, DeviceStatus *status) {
     using K = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -293,28 +294,30 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int mrow = g * 16 + lane;             // chunk row (M = 64 layout, lane < 16)
         const bool mrow_ok = lane < 16;
         const bool own_row = mrow_ok && mrow / K::ROWS == (int)rank;
-        const float A2 = -expf(A_log[h]) * kLog2e;
-        const float bias = dt_bias[h];
+        const float A2 = log_decay ? 0.0f : -expf(A_log[h]) * kLog2e;
+        const float bias = log_decay ? 0.0f : dt_bias[h];
         const bool elected = ct == 0;
         const int tok = ct & 63, q4 = ct >> 6;      // feature generation: token, 32-feature part
         uint32_t slab_uses[2] = {0, 0};
         float *part0 = reinterpret_cast<float *>(smem + K::OFF_PART);
         float *res = reinterpret_cast<float *>(smem + K::OFF_RES);
 
-        float dt_next = (ct < kC && nc > 0) ? dt_p[(size_t)row0 + ct] : 0.0f;
+        // per-token decay input: the dt projection, or the given log-decay (Algorithm 4)
+        const float *dsrc = log_decay ? log_decay : dt_p;
+        float dt_next = (ct < kC && nc > 0) ? dsrc[(size_t)row0 + ct] : 0.0f;
         for (int c = 0; c < nc; ++c) {
             const int st = c % kStages;
             uint8_t *sQ = smem + K::OFF_STAGE + st * K::STAGE;
             uint8_t *sK = sQ + K::TILE;
             uint8_t *sV = sK + K::TILE;
             const float dtv = dt_next;
-            if (ct < kC && c + 1 < nc) dt_next = dt_p[(size_t)row0 + (size_t)(c + 1) * kC + ct];
+            if (ct < kC && c + 1 < nc) dt_next = dsrc[(size_t)row0 + (size_t)(c + 1) * kC + ct];
 
             bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
             // ---- decay (tokens 0..63 on threads 0..63)
             float a = 0.0f;
             if (ct < kC) {
-                a = A2 * softplus_f(dtv + bias);
+                a = log_decay ? dtv * kLog2e : A2 * softplus_f(dtv + bias);
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float y = __shfl_up_sync(0xffffffffu, a, o);
@@ -636,7 +639,7 @@ int launch_d(const FwdArgs &a) {
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
     cudaError_t e = cudaLaunchKernelEx(&cfg, tc_order2_kernel<D>, tq, tk, tv,
                                        static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log,
-                                       a.dt_bias, a.D, a.H, a.N, a.normalize, status);
+                                       a.dt_bias, a.D, a.log_decay, a.H, a.N, a.normalize, status);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -121,3 +121,12 @@ def make_workload_inputs(w: Workload, seed: int = 0, residual: Optional[bool] = 
     """make_inputs for a named workload (residual defaults to the workload's)."""
     res = w.residual if residual is None else residual
     return make_inputs(w.B, w.H, w.N, w.d, w.dtype, seed, res)
+
+
+def make_log_decay(B: int, H: int, N: int, seed: int = 0, mean: float = -2.0) -> np.ndarray:
+    """Per-token log-decays for the Mamba-2S input form (Algorithm 4,
+    A = -softplus(h W_A)), with the projection h W_A drawn as N(mean, 1).
+    Returns float32 [B, H, N], every entry < 0 (mean -0.13 for mean = -2)."""
+    rng = np.random.Generator(np.random.PCG64(seed + 1000))
+    z = rng.standard_normal(size=(B, H, N)) + mean
+    return (-(np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z))))).astype(np.float32)

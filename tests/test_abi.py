@@ -103,3 +103,26 @@ def test_cumsum_validation(lib):
     assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 100, 64, 64, 80, None) == 2
     assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 128, 48, 64, 80, None) == 5
     assert lib.ssd_chunk_cumsum(None, 32, 48, 1, 1, 128, 64, 64, 80, None) == 1
+
+
+def _call_fwd_ex(lib, **over):
+    a = dict(q=16, k=32, v=48, dt_p=64, A_log=80, dt_bias=96, D=None, ld=None, B=1, H=2, N=256, d=16,
+             dtype=ssd.SSD_F32, order=1, normalize=0, chunk=64, flags=0, out=112, ws=256, ws_bytes=1 << 30)
+    a.update(over)
+    return lib.ssd_fwd_ex(a["q"], a["k"], a["v"], a["dt_p"], a["A_log"], a["dt_bias"], a["D"], a["ld"],
+                          a["B"], a["H"], a["N"], a["d"], a["dtype"], a["order"], a["normalize"],
+                          a["chunk"], a["flags"], a["out"], a["ws"], a["ws_bytes"], None)
+
+
+def test_fwd_ex_validation_codes(lib):
+    """ssd_fwd_ex rejects unknown flags and missing inputs of the chosen
+    decay / value form on the host (fake pointers, never dereferenced)."""
+    assert _call_fwd_ex(lib, flags=2) == 11                              # SSD_ERR_FLAGS
+    assert _call_fwd_ex(lib, flags=-1) == 11
+    assert _call_fwd_ex(lib, A_log=None) == 1                            # A*dt needs A_log
+    assert _call_fwd_ex(lib, dt_p=None) == 1                             # ... and dt_p
+    assert _call_fwd_ex(lib, ld=128, A_log=None, flags=1, dt_p=None) == 1  # V (.) dt needs dt_p
+    assert _call_fwd_ex(lib, ld=128, A_log=None, flags=1, dt_bias=None) == 1
+    assert _call_fwd_ex(lib, ld=136) == 6                                # SSD_ERR_ALIGN
+    assert _call_fwd_ex(lib, ld=128, N=250) == 2
+    assert ssd.status_str(11).startswith("SSD_ERR_FLAGS")
