@@ -55,13 +55,13 @@ def _load():
                                      ctypes.c_int, _f64p]
     lib.oracle_log_decay.restype = None
     lib.oracle_ssd_quadratic.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
-                                         _f32p, ctypes.c_int,
+                                         _f32p, ctypes.c_int, _f64p, _f64p,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, _i32p, ctypes.c_int,
                                          _f64p, _f64p]
     lib.oracle_ssd_quadratic.restype = ctypes.c_int
     lib.oracle_ssd_recurrent.argtypes = [_f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
-                                         _f32p, ctypes.c_int,
+                                         _f32p, ctypes.c_int, _f64p, _f64p,
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
     lib.oracle_ssd_recurrent.restype = ctypes.c_int
@@ -125,19 +125,34 @@ def _opt(a):
     return None if a is None else _f32(a)
 
 
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _check_state(h0, z0, B, H, d, order):
+    Dphi = d ** order
+    if h0 is not None and h0.shape != (B, H, Dphi, d):
+        raise ValueError(f"h0 must be [B, H, d^order, d] = {(B, H, Dphi, d)}")
+    if z0 is not None and z0.shape != (B, H, Dphi):
+        raise ValueError(f"z0 must be [B, H, d^order] = {(B, H, Dphi)}")
+
+
 def ssd_quadratic(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
                   rows: Optional[Sequence[int]] = None, return_norm: bool = False,
-                  log_decay=None, value_dt: bool = False):
+                  log_decay=None, value_dt: bool = False, h0=None, z0=None):
     """Masked-matrix form of the operator (Algorithms 1 and 5), in float64.
 
     ``log_decay`` ([B, H, N], optional) replaces A dt by a given per-token
     log-decay (Algorithm 4); ``value_dt`` contracts with V (.) dt instead of V
-    (Algorithm 4, V_dt).  Returns y as [B, H, len(rows) or N, d] (and the row
-    sums N_i when ``return_norm``)."""
+    (Algorithm 4, V_dt).  ``h0`` [B, H, d^order, d] and ``z0`` [B, H, d^order]
+    are the states carried into token 0 (zero when None).  Returns y as
+    [B, H, len(rows) or N, d] (and the row sums N_i when ``return_norm``)."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     dt_p, A_log, dt_bias, ld = _opt(dt_p), _opt(A_log), _opt(dt_bias), _opt(log_decay)
+    h0d, z0d = _f64(h0), _f64(z0)
     Dv = None if D is None else _f32(D)
     B, H, N, d = q.shape
+    _check_state(h0d, z0d, B, H, d, order)
     if rows is None:
         r_arr = None
         n_rows = N
@@ -149,7 +164,8 @@ def ssd_quadratic(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
     rc = _load().oracle_ssd_quadratic(
         _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(dt_p, _f32p),
         _ptr(A_log, _f32p), _ptr(dt_bias, _f32p), _ptr(Dv, _f32p), _ptr(ld, _f32p),
-        int(bool(value_dt)), B, H, N, d, int(order), int(bool(normalize)),
+        int(bool(value_dt)), _ptr(h0d, _f64p), _ptr(z0d, _f64p),
+        B, H, N, d, int(order), int(bool(normalize)),
         _ptr(r_arr, _i32p), n_rows, _ptr(out, _f64p), _ptr(norm, _f64p))
     if rc != 0:
         raise ValueError("oracle_ssd_quadratic rejected its arguments")
@@ -158,16 +174,18 @@ def ssd_quadratic(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
 
 def ssd_recurrent(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
                   return_norm: bool = False, return_state: bool = False,
-                  log_decay=None, value_dt: bool = False):
+                  log_decay=None, value_dt: bool = False, h0=None, z0=None):
     """Token-by-token recurrent form (Algorithm 6), in float64.
 
-    ``log_decay`` and ``value_dt`` as in ssd_quadratic.  Returns y
+    ``log_decay``, ``value_dt``, ``h0`` and ``z0`` as in ssd_quadratic.  Returns y
     [B, H, N, d]; optionally the row sums [B, H, N] and the final states
     H_up [B, H, d^order, d] and H_dn [B, H, d^order]."""
     q, k, v = _f32(q), _f32(k), _f32(v)
     dt_p, A_log, dt_bias, ld = _opt(dt_p), _opt(A_log), _opt(dt_bias), _opt(log_decay)
+    h0d, z0d = _f64(h0), _f64(z0)
     Dv = None if D is None else _f32(D)
     B, H, N, d = q.shape
+    _check_state(h0d, z0d, B, H, d, order)
     Dphi = d ** order
     out = np.zeros((B, H, N, d), dtype=np.float64)
     norm = np.zeros((B, H, N), dtype=np.float64)
@@ -176,7 +194,8 @@ def ssd_recurrent(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
     rc = _load().oracle_ssd_recurrent(
         _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(dt_p, _f32p),
         _ptr(A_log, _f32p), _ptr(dt_bias, _f32p), _ptr(Dv, _f32p), _ptr(ld, _f32p),
-        int(bool(value_dt)), B, H, N, d, int(order), int(bool(normalize)),
+        int(bool(value_dt)), _ptr(h0d, _f64p), _ptr(z0d, _f64p),
+        B, H, N, d, int(order), int(bool(normalize)),
         _ptr(out, _f64p), _ptr(norm, _f64p), _ptr(st, _f64p), _ptr(zst, _f64p))
     if rc != 0:
         raise ValueError("oracle_ssd_recurrent rejected its arguments")

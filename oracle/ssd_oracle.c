@@ -125,6 +125,10 @@ int oracle_feature(const double *x, int d, int order, double *out)
  *     y_i  = sum_j w_ij f_j v_j,   N_i = sum_j w_ij,
  * with f_j = dt_j under value_dt and 1 otherwise,
  *     y_i /= N_i when normalise != 0,   y_ic += D[h*d + c] * v_ic when D.
+ * With an initial state (h0 [B, H, D_phi, d], z0 [B, H, D_phi], either may be
+ * NULL for zero) the state carried into token 0 decays by exp(A^CS_i) up to
+ * token i (Algorithm 6 unrolled): y_i += exp(A^CS_i) phi(q_i)^T h0 and
+ * N_i += exp(A^CS_i) phi(q_i) . z0.
  * rows: n_rows row indices (each in [0, N)), or NULL for all N rows.
  * out: [B, H, n_rows, d] (n_rows = N when rows is NULL).
  * norm_out (may be NULL): [B, H, n_rows], the row sums N_i.
@@ -132,12 +136,13 @@ int oracle_feature(const double *x, int d, int order, double *out)
 int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
                          const float *dt_p, const float *A_log, const float *dt_bias,
                          const float *D, const float *log_decay, int value_dt,
+                         const double *h0, const double *z0,
                          int B, int H, int N, int d, int order, int normalise,
                          const int *rows, int n_rows,
                          double *out, double *norm_out)
 {
     if (order != 1 && order != 2) return -1;
-    if (B < 0 || H < 0 || N < 0 || d <= 0) return -1;
+    if (B < 0 || H < 0 || N < 0 || d <= 0 || d > 64) return -1;
     if (rows == NULL) n_rows = N;
     for (int r = 0; rows && r < n_rows; ++r)
         if (rows[r] < 0 || rows[r] >= N) return -1;
@@ -171,6 +176,20 @@ int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
             for (int c = 0; c < d; ++c) yi[c] += wv * (double)vj[c];
             ni += w;
         }
+        if (h0 || z0) {
+            int Dphi = (order == 1) ? d : d * d;
+            double e = exp(acs_row[i]);
+            double xq[64], fq[64 * 64];
+            for (int c = 0; c < d; ++c) xq[c] = qi[c];
+            oracle_feature(xq, d, order, fq);
+            for (int m = 0; m < Dphi; ++m) {
+                if (h0) {
+                    const double *row = h0 + ((size_t)bh * Dphi + m) * d;
+                    for (int c = 0; c < d; ++c) yi[c] += e * fq[m] * row[c];
+                }
+                if (z0) ni += e * fq[m] * z0[(size_t)bh * Dphi + m];
+            }
+        }
         if (normalise)
             for (int c = 0; c < d; ++c) yi[c] /= ni;
         if (D) {
@@ -190,13 +209,15 @@ int oracle_ssd_quadratic(const float *q, const float *k, const float *v,
  *     H_dn_t = a_t H_dn_{t-1} + phi(k_t)           (D_phi)
  *     y_t = phi(q_t)^T H_up_t,  N_t = phi(q_t) . H_dn_t,
  * then y_t /= N_t when normalising and y_tc += D[h*d+c] v_tc when D.
- * Both states start at zero.  out is [B, H, N, d]; norm_out may be NULL.
+ * The states start at h0 [B, H, D_phi, d] and z0 [B, H, D_phi] (zero when
+ * NULL).  out is [B, H, N, d]; norm_out may be NULL.
  * state_out (may be NULL) receives the final H_up as [B, H, D_phi, d] and
  * zstate_out (may be NULL) the final H_dn as [B, H, D_phi].
  * Returns 0, or -1 on a bad argument / allocation failure. */
 int oracle_ssd_recurrent(const float *q, const float *k, const float *v,
                          const float *dt_p, const float *A_log, const float *dt_bias,
                          const float *D, const float *log_decay, int value_dt,
+                         const double *h0, const double *z0,
                          int B, int H, int N, int d, int order, int normalise,
                          double *out, double *norm_out,
                          double *state_out, double *zstate_out)
@@ -222,6 +243,8 @@ int oracle_ssd_recurrent(const float *q, const float *k, const float *v,
             free(Hup); free(Hdn); free(fq); free(fk); free(xq); free(xk);
             continue;
         }
+        if (h0) memcpy(Hup, h0 + (size_t)bh * Dphi * d, sizeof(double) * (size_t)Dphi * d);
+        if (z0) memcpy(Hdn, z0 + (size_t)bh * Dphi, sizeof(double) * (size_t)Dphi);
         size_t base = (size_t)bh * N;
         for (int t = 0; t < N; ++t) {
             double a;

@@ -387,3 +387,58 @@ def test_zero_log_decay_value_dt_prefix_sums():
     S = np.cumsum(kv, axis=0)
     ref = np.einsum("nc,nce->ne", x["q"][0, 0].astype(np.float64), S)
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------ carried state in and out (Algorithm 6)
+def test_hand_decode_step_initial_state(golden):
+    """One recurrent step from a given state, worked out by hand."""
+    c = golden["decode-step-initial-state"]
+    arr = lambda a: np.asarray(a, np.float32).reshape(1, 1, 1, 1)
+    q, k, v = arr(c["q"]), arr(c["k"]), arr(c["v"])
+    ld = np.asarray(c["log_decay"], np.float32).reshape(1, 1, 1)
+    h0 = np.asarray(c["h0"], np.float64).reshape(1, 1, 1, 1)
+    z0 = np.asarray(c["z0"], np.float64).reshape(1, 1, 1)
+    for e in c["expect"]:
+        D = np.asarray(c["D"], np.float32) if e["residual"] else None
+        y, _, h, z = oracle.ssd_recurrent(q, k, v, None, None, None, D, e["order"], e["normalize"],
+                                          return_norm=True, return_state=True, log_decay=ld, h0=h0, z0=z0)
+        np.testing.assert_allclose(y[0, 0], e["y"], rtol=1e-7)
+        if "h" in e:
+            np.testing.assert_allclose(h[0, 0], e["h"], rtol=1e-7)
+            np.testing.assert_allclose(z[0, 0], e["z"], rtol=1e-7)
+        yq = oracle.ssd_quadratic(q, k, v, None, None, None, D, e["order"], e["normalize"],
+                                  log_decay=ld, h0=h0, z0=z0)
+        np.testing.assert_allclose(yq[0, 0], e["y"], rtol=1e-7)
+
+
+@pytest.mark.parametrize("order,norm", [(1, False), (2, True)])
+def test_split_sequence_carries_state(order, norm):
+    """Running tokens [0, n) and then [n, N) from the state the first part
+    leaves gives the same outputs as running [0, N) at once."""
+    x = _small(7, N=21)
+    n = 8
+    y_all = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"],
+                                 order, norm)
+    sl = lambda a, lo, hi: a[:, :, lo:hi]
+    y1, h, z = oracle.ssd_recurrent(sl(x["q"], 0, n), sl(x["k"], 0, n), sl(x["v"], 0, n), sl(x["dt_p"], 0, n),
+                                    x["A_log"], x["dt_bias"], x["D"], order, norm, return_state=True)
+    y2 = oracle.ssd_recurrent(sl(x["q"], n, None), sl(x["k"], n, None), sl(x["v"], n, None),
+                              sl(x["dt_p"], n, None), x["A_log"], x["dt_bias"], x["D"], order, norm, h0=h, z0=z)
+    np.testing.assert_allclose(np.concatenate([y1, y2], axis=2), y_all, rtol=1e-12, atol=1e-12)
+    # the quadratic form with the same carried state agrees with the recurrence
+    y2q = oracle.ssd_quadratic(sl(x["q"], n, None), sl(x["k"], n, None), sl(x["v"], n, None),
+                               sl(x["dt_p"], n, None), x["A_log"], x["dt_bias"], x["D"], order, norm, h0=h, z0=z)
+    np.testing.assert_allclose(y2q, y2, rtol=1e-11, atol=1e-12)
+
+
+def test_zero_decay_initial_state_prefix_sums():
+    """Zero log-decay from a given state: y_i = q_i^T (h0 + sum_{j<=i} k_j v_j^T)."""
+    x = _small(8, B=1, H=1, N=13, d=3)
+    rng = np.random.default_rng(3)
+    h0 = rng.standard_normal((1, 1, 3, 3))
+    ld = np.zeros_like(x["dt_p"])
+    y = oracle.ssd_quadratic(x["q"], x["k"], x["v"], None, None, None, None, 1, False, log_decay=ld, h0=h0)[0, 0]
+    S = h0[0, 0] + np.cumsum(np.einsum("nc,ne->nce", x["k"][0, 0].astype(np.float64),
+                                       x["v"][0, 0].astype(np.float64)), axis=0)
+    ref = np.einsum("nc,nce->ne", x["q"][0, 0].astype(np.float64), S)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
