@@ -79,12 +79,24 @@ typedef enum {
 typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
 
 /*
- * Bytes of device workspace ssd_fwd() and ssd_fwd_ex() need for this problem
- * (any normalize setting, any flags).  Depends only on the arguments.  Returns 0 when the arguments are invalid (ssd_fwd
+ * Bytes of device workspace ssd_fwd() needs for this problem (either
+ * normalize setting).  Depends only on the arguments.  Returns 0 when the arguments are invalid (ssd_fwd
  * would reject them).  Supported: B, H >= 1; N >= 1 with N % chunk == 0;
  * d_h in {16, 32, 64}; order in {1, 2}; chunk in {64, 128, 256}.
  */
 size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk);
+
+/* State arguments of ssd_fwd_state() that are in use (bit mask). */
+typedef enum { SSD_STATE_H = 1, SSD_STATE_Z = 2 } ssd_state_mask;
+
+/*
+ * Bytes of device workspace ssd_fwd_ex() / ssd_fwd_state() need: `flags` as
+ * passed to them, `state` = SSD_STATE_H if h0 or h_out is given, | SSD_STATE_Z
+ * if z0 or z_out is given (0 for ssd_fwd_ex).  Either normalize setting.
+ * 0 for invalid arguments.
+ */
+size_t ssd_workspace_bytes_ex(int B, int H, int N, int d_h, int dtype, int order, int chunk,
+                              int flags, int state);
 
 /*
  * Forward pass of the operator above.
@@ -123,6 +135,7 @@ int ssd_fwd(const void *q, const void *k, const void *v,
  *              log_decay is NULL or SSD_VALUE_DT is set; otherwise they may
  *              be NULL.
  * ssd_fwd(...) is ssd_fwd_ex(..., log_decay = NULL, flags = 0).
+ * workspace_bytes must be at least ssd_workspace_bytes_ex(..., flags, 0).
  * Paths: order 1 and order-2 decay options run on the tensor-core paths; order
  * 2 with SSD_VALUE_DT runs on the SIMT path.
  * Errors as ssd_fwd(), plus SSD_ERR_FLAGS for unknown flag bits.
@@ -209,6 +222,65 @@ int ssd_fwd_noalloc(const void *q, const void *k, const void *v,
                     int B, int H, int N, int d_h, int dtype,
                     int order, int normalize, int chunk,
                     void *out, void *stream);
+
+/*
+ * ssd_fwd_ex() with the carried state in and out (prefill before decode;
+ * 2Mamba2Furious Algorithm 6, whose state update H_t = a_t H_{t-1} +
+ * phi(k_t) v_t^T this continues).  Extra arguments, each may be NULL:
+ *   h0     device, [B, H, D_phi, d_h] fp32, the state carried into token 0
+ *          (D_phi = d_h for order 1, d_h^2 for order 2; feature (a, b) of
+ *          order 2 is row a*d_h + b).  NULL = zero.
+ *   z0     device, [B, H, D_phi] fp32, the normaliser state carried in.
+ *          NULL = zero.
+ *   h_out  device, [B, H, D_phi, d_h] fp32, receives the state after token
+ *          N-1.  May equal h0 (updated in place).
+ *   z_out  device, [B, H, D_phi] fp32, the normaliser state after token N-1.
+ *          May equal z0.
+ * With value discretisation the state accumulates phi(k) (dt v)^T; the
+ * normaliser state never sees dt.  Paths: order 1 with h0/h_out only runs on
+ * the tensor-core path; z0/z_out for order 1, and any state for order 2, run
+ * on the SIMT path.  Errors as ssd_fwd_ex().
+ */
+int ssd_fwd_state(const void *q, const void *k, const void *v,
+                  const float *dt_p, const float *A_log, const float *dt_bias,
+                  const float *D, const float *log_decay,
+                  int B, int H, int N, int d_h, int dtype,
+                  int order, int normalize, int chunk, int flags,
+                  const float *h0, const float *z0, float *h_out, float *z_out,
+                  void *out, void *workspace, size_t workspace_bytes,
+                  void *stream);
+
+/*
+ * Bytes of device workspace ssd_decode_step() needs (0 for invalid
+ * arguments: d_h in {16, 32, 64}, order in {1, 2}, B, H >= 1).
+ */
+size_t ssd_decode_workspace_bytes(int B, int H, int d_h, int order);
+
+/*
+ * One recurrent step per (b, h): the token-by-token form of 2Mamba2Furious
+ * Algorithm 6 used for generation after a prefill.
+ *   q, k, v    device, [B, H, d_h], element type `dtype`
+ *   dt_p       device, [B, H] fp32 (may be NULL when log_decay is given and
+ *              SSD_VALUE_DT is not set); A_log, dt_bias [H] fp32 as in
+ *              ssd_fwd_ex(); log_decay device [B, H] fp32 or NULL
+ *   D          device, [H*d_h] fp32, or NULL
+ *   h          device, [B, H, D_phi, d_h] fp32, updated in place:
+ *              h <- a h + phi(k) (f v)^T, a = exp(log-decay), f = dt or 1
+ *   z          device, [B, H, D_phi] fp32, updated in place when given:
+ *              z <- a z + phi(k); required when normalize != 0, may be NULL
+ *              otherwise
+ *   out        device, [B, H, d_h], element type `dtype`:
+ *              y = phi(q)^T h [/ phi(q) . z] [+ D (.) v]
+ *   workspace  device, >= ssd_decode_workspace_bytes(), 256-byte aligned
+ * The step reads and writes the whole state once (memory-bound: order 2 at
+ * d_h = 64 moves 2 MiB per head).  Two launches.  Errors as ssd_fwd_ex().
+ */
+int ssd_decode_step(const void *q, const void *k, const void *v,
+                    const float *dt_p, const float *A_log, const float *dt_bias,
+                    const float *D, const float *log_decay,
+                    int B, int H, int d_h, int dtype, int order, int normalize, int flags,
+                    float *h, float *z, void *out,
+                    void *workspace, size_t workspace_bytes, void *stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *ssd_status_str(int status);

@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libssd.so")
 SSD_F32 = 0
 SSD_BF16 = 1
 SSD_VALUE_DT = 1  # ssd_fwd_ex flag: contract with v * dt (Algorithm 4, V_dt)
+SSD_STATE_H = 1   # state-mask bits for ssd_workspace_bytes_ex
+SSD_STATE_Z = 2
 PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2"}
 
 _lib = None
@@ -50,6 +52,14 @@ def load_library():
     lib.ssd_fwd.restype = ci
     lib.ssd_fwd_ex.argtypes = [vp] * 8 + [ci] * 9 + [vp, vp, sz, vp]
     lib.ssd_fwd_ex.restype = ci
+    lib.ssd_fwd_state.argtypes = [vp] * 8 + [ci] * 9 + [vp] * 4 + [vp, vp, sz, vp]
+    lib.ssd_fwd_state.restype = ci
+    lib.ssd_workspace_bytes_ex.argtypes = [ci] * 9
+    lib.ssd_workspace_bytes_ex.restype = sz
+    lib.ssd_decode_workspace_bytes.argtypes = [ci] * 4
+    lib.ssd_decode_workspace_bytes.restype = sz
+    lib.ssd_decode_step.argtypes = [vp] * 8 + [ci] * 7 + [vp, vp, vp, vp, sz, vp]
+    lib.ssd_decode_step.restype = ci
     lib.ssd_fwd_host.argtypes = [vp] * 7 + [ci] * 8 + [vp] + [vp] * 8 + [vp, sz, vp]
     lib.ssd_fwd_host.restype = ci
     lib.ssd_chunk_cumsum.argtypes = [vp] * 3 + [ci] * 4 + [vp, vp, vp]
@@ -112,10 +122,17 @@ def ssd_fwd_path(B: int, H: int, N: int, d_h: int, dtype: int, order: int, chunk
     return PATH_NAMES[p], n.value
 
 
-def alloc_workspace(B, H, N, d_h, dtype, order, chunk, device=None):
-    """A torch uint8 device buffer of ssd_workspace_bytes() bytes."""
+def ssd_workspace_bytes_ex(B: int, H: int, N: int, d_h: int, dtype: int, order: int, chunk: int,
+                           flags: int = 0, state: int = 0) -> int:
+    """Device workspace (bytes) ssd_fwd_ex / ssd_fwd_state need for these
+    options (state: SSD_STATE_H | SSD_STATE_Z bits in use); 0 when invalid."""
+    return int(load_library().ssd_workspace_bytes_ex(B, H, N, d_h, dtype, order, chunk, flags, state))
+
+
+def alloc_workspace(B, H, N, d_h, dtype, order, chunk, device=None, flags: int = 0, state: int = 0):
+    """A torch uint8 device buffer of ssd_workspace_bytes_ex() bytes."""
     import torch
-    nbytes = ssd_workspace_bytes(B, H, N, d_h, dtype, order, chunk)
+    nbytes = ssd_workspace_bytes_ex(B, H, N, d_h, dtype, order, chunk, flags, state)
     if nbytes == 0:
         raise ValueError("invalid ssd arguments")
     return torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
@@ -137,8 +154,9 @@ def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk
     dt = _dtype_code(q)
     if out is None:
         out = torch.empty_like(q)
+    flags = SSD_VALUE_DT if value_dt else 0
     if workspace is None:
-        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device)
+        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device, flags)
     lib = load_library()
     if log_decay is None and not value_dt:
         rc = lib.ssd_fwd(
@@ -153,6 +171,61 @@ def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk
             SSD_VALUE_DT if value_dt else 0, _ptr(out), _ptr(workspace), workspace.numel(),
             _stream_handle(stream))
         _check(rc, "ssd_fwd_ex")
+    return out
+
+
+def ssd_fwd_state(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk: int,
+                  h0=None, z0=None, h_out=None, z_out=None, out=None, workspace=None, stream=None,
+                  log_decay=None, value_dt: bool = False):
+    """ssd_fwd with the carried state in and out (include/ssd.h, ssd_fwd_state).
+
+    h0 / h_out: [B, H, d_h^order, d_h] float32, z0 / z_out: [B, H, d_h^order]
+    float32 CUDA tensors or None (h_out may be h0: updated in place).
+    Returns `out`."""
+    import torch
+    B, H, N, d = q.shape
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    flags = SSD_VALUE_DT if value_dt else 0
+    state = (SSD_STATE_H if (h0 is not None or h_out is not None) else 0) | \
+        (SSD_STATE_Z if (z0 is not None or z_out is not None) else 0)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device, flags, state)
+    rc = load_library().ssd_fwd_state(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D), _ptr(log_decay),
+        B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk), flags,
+        _ptr(h0), _ptr(z0), _ptr(h_out), _ptr(z_out),
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "ssd_fwd_state")
+    return out
+
+
+def ssd_decode_workspace_bytes(B: int, H: int, d_h: int, order: int) -> int:
+    """Device workspace (bytes) ssd_decode_step needs; 0 when invalid."""
+    return int(load_library().ssd_decode_workspace_bytes(B, H, d_h, order))
+
+
+def ssd_decode_step(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, h, z=None,
+                    out=None, workspace=None, stream=None, log_decay=None, value_dt: bool = False):
+    """One recurrent step (include/ssd.h, ssd_decode_step): q, k, v [B, H, d_h];
+    dt_p / log_decay [B, H]; h [B, H, d_h^order, d_h] and z [B, H, d_h^order]
+    float32, updated in place.  Returns `out` [B, H, d_h]."""
+    import torch
+    B, H, d = q.shape
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        n = ssd_decode_workspace_bytes(B, H, d, order)
+        if n == 0:
+            raise ValueError("invalid ssd_decode_step arguments")
+        workspace = torch.empty(n, dtype=torch.uint8, device=q.device)
+    rc = load_library().ssd_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D), _ptr(log_decay),
+        B, H, d, dt, int(order), int(bool(normalize)), SSD_VALUE_DT if value_dt else 0,
+        _ptr(h), _ptr(z), _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "ssd_decode_step")
     return out
 
 

@@ -32,14 +32,15 @@ static size_t simt_total(int B, int H, int N, int d, int order, int chunk, Plan 
 }
 
 bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
-               int value_dt, Plan *plan) {
+               int value_dt, int state, Plan *plan) {
     if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
     Plan p{};
-    if (order == 1 && !normalize && tc_order1_supports(B, H, N, d, dtype, chunk)) {
+    if (order == 1 && !normalize && !(state & SSD_STATE_Z) &&
+        tc_order1_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER1;
         p.n_launches = 3;
         tc_order1_layout(B, H, N, chunk, &p);
-    } else if (order == 2 && !value_dt && tc_order2_supports(B, H, N, d, dtype, chunk)) {
+    } else if (order == 2 && !value_dt && !state && tc_order2_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER2;
         p.n_launches = 1;
         p.acs_off = p.lam_off = p.state_off = kStatusBytes;
@@ -59,31 +60,37 @@ using namespace ssd;
 
 extern "C" {
 
-size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk) {
-    // the size covers every setting of `normalize` and of the flags, which can
-    // select different paths
+size_t ssd_workspace_bytes_ex(int B, int H, int N, int d_h, int dtype, int order, int chunk,
+                              int flags, int state) {
+    if ((flags & ~SSD_VALUE_DT) != 0 || (state & ~(SSD_STATE_H | SSD_STATE_Z)) != 0) return 0;
+    // the size covers both settings of `normalize`, which can select different paths
     size_t need = 0;
-    for (int norm = 0; norm < 2; ++norm)
-        for (int vdt = 0; vdt < 2; ++vdt) {
-            Plan p;
-            if (!make_plan(B, H, N, d_h, dtype, order, norm, chunk, vdt, &p)) return 0;
-            if (p.total > need) need = p.total;
-        }
+    for (int norm = 0; norm < 2; ++norm) {
+        Plan p;
+        if (!make_plan(B, H, N, d_h, dtype, order, norm, chunk, flags & SSD_VALUE_DT, state, &p))
+            return 0;
+        if (p.total > need) need = p.total;
+    }
     return need;
+}
+
+size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk) {
+    return ssd_workspace_bytes_ex(B, H, N, d_h, dtype, order, chunk, 0, 0);
 }
 
 int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
                  int *n_launches) {
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, 0, &p)) return -1;
+    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, 0, 0, &p)) return -1;
     if (n_launches) *n_launches = p.n_launches;
     return p.path;
 }
 
-int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,
-               const float *A_log, const float *dt_bias, const float *D, const float *log_decay,
-               int B, int H, int N, int d_h, int dtype, int order, int normalize, int chunk,
-               int flags, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+int ssd_fwd_state(const void *q, const void *k, const void *v, const float *dt_p,
+                  const float *A_log, const float *dt_bias, const float *D, const float *log_decay,
+                  int B, int H, int N, int d_h, int dtype, int order, int normalize, int chunk,
+                  int flags, const float *h0, const float *z0, float *h_out, float *z_out,
+                  void *out, void *workspace, size_t workspace_bytes, void *stream) {
     if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
     const int value_dt = (flags & SSD_VALUE_DT) ? 1 : 0;
     if (!q || !k || !v || !out) return SSD_ERR_NULL;
@@ -93,23 +100,71 @@ int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,
     int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
     if (rc != SSD_OK) return rc;
     if (!workspace) return SSD_ERR_WORKSPACE;
-    const void *ptrs[] = {q, k, v, out, dt_p, A_log, dt_bias, D, log_decay};
+    const void *ptrs[] = {q, k, v, out, dt_p, A_log, dt_bias, D, log_decay, h0, z0, h_out, z_out};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return SSD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
+    const int state = ((h0 || h_out) ? SSD_STATE_H : 0) | ((z0 || z_out) ? SSD_STATE_Z : 0);
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, normalize, chunk, value_dt, &p))
+    if (!make_plan(B, H, N, d_h, dtype, order, normalize, chunk, value_dt, state, &p))
         return SSD_ERR_UNSUPPORTED;
     if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
     FwdArgs a{q, k, v, need_dt ? dt_p : nullptr, log_decay ? nullptr : A_log,
-              need_dt ? dt_bias : nullptr, D, log_decay, value_dt, B, H, N, d_h, dtype, order,
-              normalize ? 1 : 0, chunk, out, workspace, workspace_bytes,
-              static_cast<cudaStream_t>(stream)};
+              need_dt ? dt_bias : nullptr, D, log_decay, value_dt, h0, z0, h_out, z_out,
+              B, H, N, d_h, dtype, order, normalize ? 1 : 0, chunk, out, workspace,
+              workspace_bytes, static_cast<cudaStream_t>(stream)};
     switch (p.path) {
     case PATH_TC_ORDER1: return launch_tc_order1(a, p);
     case PATH_TC_ORDER2: return launch_tc_order2(a, p);
     default: return launch_simt(a, p);
     }
+}
+
+int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,
+               const float *A_log, const float *dt_bias, const float *D, const float *log_decay,
+               int B, int H, int N, int d_h, int dtype, int order, int normalize, int chunk,
+               int flags, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    return ssd_fwd_state(q, k, v, dt_p, A_log, dt_bias, D, log_decay, B, H, N, d_h, dtype, order,
+                         normalize, chunk, flags, nullptr, nullptr, nullptr, nullptr, out, workspace,
+                         workspace_bytes, stream);
+}
+
+size_t ssd_decode_workspace_bytes(int B, int H, int d_h, int order) {
+    if (B < 1 || H < 1 || (long long)B * H > 65535) return 0;
+    if ((d_h != 16 && d_h != 32 && d_h != 64) || (order != 1 && order != 2)) return 0;
+    return kStatusBytes + decode_workspace(B, H, d_h, order);
+}
+
+int ssd_decode_step(const void *q, const void *k, const void *v, const float *dt_p,
+                    const float *A_log, const float *dt_bias, const float *D,
+                    const float *log_decay, int B, int H, int d_h, int dtype, int order,
+                    int normalize, int flags, float *h, float *z, void *out, void *workspace,
+                    size_t workspace_bytes, void *stream) {
+    if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
+    const int value_dt = (flags & SSD_VALUE_DT) ? 1 : 0;
+    if (!q || !k || !v || !out || !h) return SSD_ERR_NULL;
+    if (normalize && !z) return SSD_ERR_NULL;
+    const bool need_dt = !log_decay || value_dt;
+    if (need_dt && (!dt_p || !dt_bias)) return SSD_ERR_NULL;
+    if (!log_decay && !A_log) return SSD_ERR_NULL;
+    if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_DTYPE;
+    if (order != 1 && order != 2) return SSD_ERR_ORDER;
+    const size_t need = ssd_decode_workspace_bytes(B, H, d_h, order);
+    if (need == 0) return SSD_ERR_SHAPE;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    const void *ptrs[] = {q, k, v, out, h, z, D};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return SSD_ERR_ALIGN;
+    const void *ptrs4[] = {dt_p, A_log, dt_bias, log_decay};  // per-token / per-head scalars
+    for (const void *p : ptrs4)
+        if (p && (reinterpret_cast<uintptr_t>(p) & 3u) != 0) return SSD_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
+    if (workspace_bytes < need) return SSD_ERR_WORKSPACE;
+    FwdArgs a{q, k, v, need_dt ? dt_p : nullptr, log_decay ? nullptr : A_log,
+              need_dt ? dt_bias : nullptr, D, log_decay, value_dt, nullptr, nullptr, nullptr,
+              nullptr, B, H, 1, d_h, dtype, order, normalize ? 1 : 0, 64, out, workspace,
+              workspace_bytes, static_cast<cudaStream_t>(stream)};
+    return launch_decode(a, h, z);
 }
 
 int ssd_fwd(const void *q, const void *k, const void *v, const float *dt_p,

@@ -16,6 +16,8 @@ struct FwdArgs {
     const float *dt_p, *A_log, *dt_bias, *D;
     const float *log_decay;  // per-token log-decay, or NULL (A * dt)
     int value_dt;            // contract with v * dt
+    const float *h0, *z0;    // carried state in, or NULL (zero)
+    float *h_out, *z_out;    // carried state out, or NULL
     int B, H, N, d, dtype, order, normalize, chunk;
     void *out;
     void *workspace;
@@ -45,8 +47,9 @@ struct Plan {
 };
 
 // Fills `plan` for validated arguments; returns false if no kernel exists.
+// state: SSD_STATE_H / SSD_STATE_Z bits of the state arguments in use.
 bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
-               int value_dt, Plan *plan);
+               int value_dt, int state, Plan *plan);
 
 // Path launchers (each returns an ssd_status).
 int launch_simt(const FwdArgs &a, const Plan &p);
@@ -56,6 +59,10 @@ size_t tc_order2_workspace(int B, int H, int N, int d, int chunk);
 int launch_tc_order1(const FwdArgs &a, const Plan &p);
 bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);
 void tc_order1_layout(int B, int H, int N, int chunk, Plan *p);
+
+// Decode step (ssd_decode.cu).
+size_t decode_workspace(int B, int H, int d, int order);
+int launch_decode(const FwdArgs &a, float *h, float *z);
 
 // Kernel (a): chunk-local inclusive cumsum of A*dt and the chunk totals.
 // When `status` is non-NULL, block (0,0) thread 0 clears it.

@@ -73,7 +73,8 @@ extern "C" int ssd_fwd_noalloc(const void *q, const void *k, const void *v, cons
 
     void *scratch = scratch_for_current_device();
     if (!scratch) return SSD_ERR_CUDA;
-    FwdArgs a{q, k, v, dt_p, A_log, dt_bias, D, nullptr, 0, B, H, N, d_h, dtype, order, normalize ? 1 : 0,
+    FwdArgs a{q, k, v, dt_p, A_log, dt_bias, D, nullptr, 0, nullptr, nullptr, nullptr, nullptr,
+              B, H, N, d_h, dtype, order, normalize ? 1 : 0,
               chunk, out, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream)};
     return launch_simt(a, p);
 }

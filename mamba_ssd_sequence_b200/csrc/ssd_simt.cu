@@ -149,20 +149,31 @@ chunk_state_kernel(const T *__restrict__ k, const T *__restrict__ v,
 
 // ---------------------------------------------------------------- kernel (c)
 // One thread per state element; walks the chunks in order, replacing each
-// chunk's own contribution U_c by the state entering the chunk.
+// chunk's own contribution U_c by the state entering the chunk.  Element e
+// of a state is row m = e / (d+1), column e % (d+1) (column d is the
+// normaliser state).  The scan starts from the carried state h0 / z0 (zero
+// when NULL) and leaves the state after the last chunk in h_out / z_out.
 __global__ void state_scan_kernel(float *__restrict__ states, const float *__restrict__ lam,
-                                  int nc, size_t elems_per_state, int BH) {
+                                  int nc, size_t elems_per_state, int BH, int d,
+                                  const float *__restrict__ h0, const float *__restrict__ z0,
+                                  float *__restrict__ h_out, float *__restrict__ z_out) {
     const size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int bh = blockIdx.y;
     if (e >= elems_per_state || bh >= BH) return;
+    const size_t m = e / (d + 1), col = e % (d + 1);
+    const size_t Dphi = elems_per_state / (d + 1);
     float *base = states + (size_t)bh * nc * elems_per_state + e;
     const float *lb = lam + (size_t)bh * nc;
     float h = 0.0f;
+    if (col < (size_t)d && h0) h = h0[((size_t)bh * Dphi + m) * d + col];
+    if (col == (size_t)d && z0) h = z0[(size_t)bh * Dphi + m];
     for (int c = 0; c < nc; ++c) {
         float u = base[(size_t)c * elems_per_state];
         base[(size_t)c * elems_per_state] = h;
         h = fmaf(expf(lb[c]), h, u);
     }
+    if (col < (size_t)d && h_out) h_out[((size_t)bh * Dphi + m) * d + col] = h;
+    if (col == (size_t)d && z_out) z_out[(size_t)bh * Dphi + m] = h;
 }
 
 // ---------------------------------------------------------------- kernel (d)
@@ -175,8 +186,8 @@ chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
                     const T *__restrict__ v, const float *__restrict__ acs,
                     const float *__restrict__ states, const float *__restrict__ D,
                     const float *__restrict__ dt_p, const float *__restrict__ dt_bias,
-                    int value_dt, int H, int N, int d, int order, int normalize, int chunk,
-                    T *__restrict__ out) {
+                    int value_dt, int carried, int H, int N, int d, int order, int normalize,
+                    int chunk, T *__restrict__ out) {
     __shared__ float qs[kTI * 64];
     __shared__ float ks[kJT * 64];
     __shared__ float vs[kJT * 64];
@@ -247,8 +258,9 @@ chunk_output_kernel(const T *__restrict__ q, const T *__restrict__ k,
         }
     }
 
-    // carried-state part: phi(q_i)^T S_c, scaled by exp(acs_i)
-    if (c > 0) {
+    // carried-state part: phi(q_i)^T S_c, scaled by exp(acs_i) (chunk 0 only
+    // has one when a state was carried into the sequence)
+    if (c > 0 || carried) {
         const float *S = states + ((size_t)bh * nc + c) * (size_t)Dphi * ld;
         for (int m0 = 0; m0 < Dphi; m0 += kTM2) {
             __syncthreads();
@@ -310,11 +322,12 @@ int run_simt(const FwdArgs &a, const Plan &p) {
                                                          a.chunk, states);
     const size_t elems = (size_t)Dphi * (a.d + 1);
     dim3 g2((unsigned)((elems + 255) / 256), BH);
-    state_scan_kernel<<<g2, 256, 0, a.stream>>>(states, lam, nc, elems, BH);
+    state_scan_kernel<<<g2, 256, 0, a.stream>>>(states, lam, nc, elems, BH, a.d, a.h0, a.z0, a.h_out,
+                                                a.z_out);
     dim3 g3(a.chunk / kTI, nc, BH);
     chunk_output_kernel<T><<<g3, kThreads, 0, a.stream>>>(
-        q, k, v, acs, states, a.D, a.dt_p, a.dt_bias, a.value_dt, a.H, a.N, a.d, a.order,
-        a.normalize, a.chunk, static_cast<T *>(a.out));
+        q, k, v, acs, states, a.D, a.dt_p, a.dt_bias, a.value_dt, (a.h0 || a.z0) ? 1 : 0, a.H, a.N, a.d,
+        a.order, a.normalize, a.chunk, static_cast<T *>(a.out));
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -330,7 +330,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // =====================================================================
 __global__ void __launch_bounds__(256)
 state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __nv_bfloat16 *__restrict__ hin,
-                  int nc) {
+                  int nc, const float *__restrict__ h0, float *__restrict__ h_out) {
     pdl_launch_dependents();  // the chunk scan waits for this grid before it reads hin
     pdl_wait();               // U and lam of the chunk-state kernel
     const int bh = blockIdx.x;
@@ -338,7 +338,14 @@ state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __
     const float4 *u = reinterpret_cast<const float4 *>(U + (size_t)bh * nc * 4096 + e);
     uint2 *out = reinterpret_cast<uint2 *>(hin + (size_t)bh * nc * 4096 + e);
     const float *lm = lam + (size_t)bh * nc;
+    // the state carried into the sequence (h0 is [k][n]; this thread holds
+    // entries (n, k..k+3) of the transposed state)
+    const int n_ = e / 64, k_ = e % 64;
     float4 hs = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (h0) {
+        const float *hp = h0 + (size_t)bh * 4096 + (size_t)k_ * 64 + n_;
+        hs = make_float4(hp[0], hp[64], hp[128], hp[192]);
+    }
     // eight chunks' inputs are in flight before the dependent updates run
     for (int c0 = 0; c0 < nc; c0 += 8) {
         float4 ub[8];
@@ -361,6 +368,13 @@ state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __
                 hs.w = fmaf(f, hs.w, ub[j].w);
             }
         }
+    }
+    if (h_out) {
+        float *hp = h_out + (size_t)bh * 4096 + (size_t)k_ * 64 + n_;
+        hp[0] = hs.x;
+        hp[64] = hs.y;
+        hp[128] = hs.z;
+        hp[192] = hs.w;
     }
 }
 
@@ -867,7 +881,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c2.stream = a.stream;
     c2.attrs = pdl;
     c2.numAttrs = 1;
-    if (cudaLaunchKernelEx(&c2, state_pass_kernel, (const float *)U, (const float *)lam, hin, nc) != cudaSuccess)
+    if (cudaLaunchKernelEx(&c2, state_pass_kernel, (const float *)U, (const float *)lam, hin, nc, a.h0, a.h_out) !=
+        cudaSuccess)
         return SSD_ERR_CUDA;
     const int n_tiles = BH * nc * K::NRB;
     const int grid = n_tiles < sms ? n_tiles : sms;

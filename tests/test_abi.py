@@ -126,3 +126,45 @@ def test_fwd_ex_validation_codes(lib):
     assert _call_fwd_ex(lib, ld=136) == 6                                # SSD_ERR_ALIGN
     assert _call_fwd_ex(lib, ld=128, N=250) == 2
     assert ssd.status_str(11).startswith("SSD_ERR_FLAGS")
+
+
+def test_state_and_decode_validation_codes(lib):
+    """ssd_fwd_state / ssd_decode_step reject bad arguments on the host."""
+    vp = ctypes.c_void_p
+    assert ssd.ssd_workspace_bytes_ex(1, 2, 256, 16, ssd.SSD_F32, 1, 64, 2, 0) == 0   # unknown flag
+    assert ssd.ssd_workspace_bytes_ex(1, 2, 256, 16, ssd.SSD_F32, 1, 64, 0, 4) == 0   # unknown state bit
+    assert ssd.ssd_workspace_bytes_ex(1, 2, 256, 16, ssd.SSD_F32, 1, 64, 0, 3) > 0
+    assert ssd.ssd_decode_workspace_bytes(2, 8, 64, 2) >= 2 * 8 * 64 * 65 * 4
+    assert ssd.ssd_decode_workspace_bytes(2, 8, 48, 2) == 0
+    assert ssd.ssd_decode_workspace_bytes(2, 8, 64, 3) == 0
+
+    def st(**o):
+        a = dict(q=16, k=32, v=48, dt_p=64, A_log=80, dt_bias=96, D=None, ld=None, B=1, H=2, N=256, d=16,
+                 dtype=ssd.SSD_F32, order=1, normalize=0, chunk=64, flags=0, h0=None, z0=None, ho=None,
+                 zo=None, out=112, ws=256, wsb=1 << 30)
+        a.update(o)
+        return lib.ssd_fwd_state(a["q"], a["k"], a["v"], a["dt_p"], a["A_log"], a["dt_bias"], a["D"], a["ld"],
+                                 a["B"], a["H"], a["N"], a["d"], a["dtype"], a["order"], a["normalize"],
+                                 a["chunk"], a["flags"], a["h0"], a["z0"], a["ho"], a["zo"], a["out"], a["ws"],
+                                 a["wsb"], None)
+    assert st(h0=136) == 6 and st(zo=8) == 6      # SSD_ERR_ALIGN
+    assert st(flags=4, h0=128) == 11              # SSD_ERR_FLAGS
+    assert st(q=None, h0=128) == 1
+
+    def dec(**o):
+        a = dict(q=16, k=32, v=48, dt_p=64, A_log=80, dt_bias=96, D=None, ld=None, B=1, H=2, d=16,
+                 dtype=ssd.SSD_F32, order=1, normalize=0, flags=0, h=128, z=None, out=112, ws=256, wsb=1 << 30)
+        a.update(o)
+        return lib.ssd_decode_step(a["q"], a["k"], a["v"], a["dt_p"], a["A_log"], a["dt_bias"], a["D"], a["ld"],
+                                   a["B"], a["H"], a["d"], a["dtype"], a["order"], a["normalize"], a["flags"],
+                                   a["h"], a["z"], a["out"], a["ws"], a["wsb"], None)
+    assert dec(h=None) == 1                       # the state is required
+    assert dec(normalize=1) == 1                  # ... and z when normalising
+    assert dec(A_log=None) == 1
+    assert dec(flags=2) == 11
+    assert dec(d=48) == 2
+    assert dec(order=3) == 4
+    assert dec(dtype=9) == 3
+    assert dec(h=136) == 6
+    assert dec(dt_p=66) == 6                      # per-token scalars need 4-byte alignment
+    assert dec(wsb=100) == 7
