@@ -65,6 +65,10 @@ def _load():
                                          ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, _f64p, _f64p, _f64p, _f64p]
     lib.oracle_ssd_recurrent.restype = ctypes.c_int
+    lib.oracle_silu.argtypes = [ctypes.c_double]
+    lib.oracle_silu.restype = ctypes.c_double
+    lib.oracle_conv1d.argtypes = [_f32p, _f32p, _f32p] + [ctypes.c_int] * 6 + [_f64p]
+    lib.oracle_conv1d.restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
     _lib = lib
@@ -205,3 +209,27 @@ def ssd_recurrent(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
     if return_state:
         res.extend([st, zst])
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def silu(x: float) -> float:
+    """SiLU(x) = x sigmoid(x) (Algorithm 3's sigma), in float64."""
+    return float(_load().oracle_silu(float(x)))
+
+
+def conv1d(x, w, bias=None, silu: bool = True) -> np.ndarray:
+    """Causal depthwise convolution over tokens (+ SiLU), float64.
+
+    x: [B, H, N, d]; w: [H*d, width], w[:, j] multiplies token t - j;
+    bias: [H*d] or None.  Returns [B, H, N, d]."""
+    x, w = _f32(x), _f32(w)
+    bv = None if bias is None else _f32(bias)
+    B, H, N, d = x.shape
+    width = int(w.shape[1])
+    if w.shape[0] != H * d:
+        raise ValueError("w must be [H*d, width]")
+    out = np.zeros((B, H, N, d), dtype=np.float64)
+    rc = _load().oracle_conv1d(_ptr(x, _f32p), _ptr(w, _f32p), _ptr(bv, _f32p), B, H, N, d, width,
+                               int(bool(silu)), _ptr(out, _f64p))
+    if rc != 0:
+        raise ValueError("oracle_conv1d rejected its arguments")
+    return out

@@ -296,3 +296,37 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/* SiLU(x) = x / (1 + e^-x)  (Algorithm 3, the sigma after the convolution). */
+double oracle_silu(double x)
+{
+    return x / (1.0 + exp(-x));
+}
+
+/* Causal depthwise 1-D convolution over the token axis, optionally followed by
+ * SiLU: the prologue Q, K, V = sigma(conv_1d(h W_QKV)) of Algorithm 3, and the
+ * window-2 convolution q^c_t = conv_1d(q_t, q_{t-1}) of the Algorithm 6 page.
+ * For every (b, h), token t and channel c (channel index h*d + c of the
+ * weights):
+ *     u = bias[h*d + c] + sum_{j < width} w[(h*d + c)*width + j] * x[t - j, c]
+ * with x[t < 0] = 0 (each (b, h) sequence starts from zero), out = SiLU(u) when
+ * silu != 0, else u.  x, out: [B, H, N, d]; w: [H*d, width]; bias: [H*d] or
+ * NULL.  Returns 0, or -1 on a bad argument. */
+int oracle_conv1d(const float *x, const float *w, const float *bias, int B, int H, int N, int d,
+                  int width, int silu, double *out)
+{
+    if (B < 0 || H < 0 || N < 0 || d <= 0 || width < 1) return -1;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            size_t base = ((size_t)b * H + h) * (size_t)N;
+            for (int t = 0; t < N; ++t)
+                for (int c = 0; c < d; ++c) {
+                    int ch = h * d + c;
+                    double u = bias ? (double)bias[ch] : 0.0;
+                    for (int j = 0; j < width && j <= t; ++j)
+                        u += (double)w[(size_t)ch * width + j] * (double)x[(base + t - j) * d + c];
+                    out[(base + t) * d + c] = silu ? oracle_silu(u) : u;
+                }
+        }
+    return 0;
+}

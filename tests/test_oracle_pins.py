@@ -442,3 +442,45 @@ def test_zero_decay_initial_state_prefix_sums():
                                        x["v"][0, 0].astype(np.float64)), axis=0)
     ref = np.einsum("nc,nce->ne", x["q"][0, 0].astype(np.float64), S)
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------- conv1d + SiLU prologue (Algorithms 3, 6)
+def test_silu_closed_forms():
+    assert oracle.silu(0.0) == 0.0
+    assert abs(oracle.silu(1.0) - 1.0 / (1.0 + math.exp(-1.0))) < 1e-16
+    assert abs(oracle.silu(-1.0) + math.exp(-1.0) / (1.0 + math.exp(-1.0))) < 1e-16
+    assert abs(oracle.silu(40.0) - 40.0) < 1e-12          # x sigmoid(x) -> x
+    assert abs(oracle.silu(-40.0)) < 1e-15                # -> 0
+
+
+def test_conv1d_hand_worked():
+    """Window 2 on one channel: u_t = 2 x_t - x_{t-1} + 0.5, x_{-1} = 0.
+    x = (1, 3, -2): u = (2.5, 5.5, -6.5)."""
+    x = np.asarray([1, 3, -2], np.float32).reshape(1, 1, 3, 1)
+    w = np.asarray([[2, -1]], np.float32)
+    b = np.asarray([0.5], np.float32)
+    u = oracle.conv1d(x, w, b, silu=False)[0, 0, :, 0]
+    np.testing.assert_array_equal(u, [2.5, 5.5, -6.5])
+    y = oracle.conv1d(x, w, b, silu=True)[0, 0, :, 0]
+    np.testing.assert_allclose(y, [v / (1 + math.exp(-v)) for v in (2.5, 5.5, -6.5)], rtol=1e-15)
+
+
+def test_conv1d_identity_and_shift_and_causality():
+    """w = (1, 0) is the identity; w = (0, 1) shifts by one token with a zero
+    first token; no token depends on a later one; heads never mix."""
+    x = _small(9, B=2, H=3, N=11, d=4)["q"]
+    H, d = 3, 4
+    ident = np.tile(np.asarray([[1, 0]], np.float32), (H * d, 1))
+    np.testing.assert_array_equal(oracle.conv1d(x, ident, silu=False), x.astype(np.float64))
+    shift = np.tile(np.asarray([[0, 1]], np.float32), (H * d, 1))
+    s = oracle.conv1d(x, shift, silu=False)
+    np.testing.assert_array_equal(s[:, :, 1:], x[:, :, :-1].astype(np.float64))
+    assert np.all(s[:, :, 0] == 0)
+    w = np.random.default_rng(1).standard_normal((H * d, 3)).astype(np.float32)
+    y = oracle.conv1d(x, w, silu=True)
+    x2 = x.copy()
+    x2[:, :, 7:] = 100.0                                  # change the future only
+    np.testing.assert_array_equal(oracle.conv1d(x2, w, silu=True)[:, :, :7], y[:, :, :7])
+    x3 = x.copy()
+    x3[:, 1] = 0.0                                        # another head only
+    np.testing.assert_array_equal(oracle.conv1d(x3, w, silu=True)[:, 0], y[:, 0])
