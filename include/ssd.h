@@ -282,6 +282,26 @@ int ssd_decode_step(const void *q, const void *k, const void *v,
                     float *h, float *z, void *out,
                     void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Causal depthwise convolution over tokens with optional SiLU, the prologue
+ * Q, K, V = SiLU(conv_1d(h W_QKV)) of 2Mamba2Furious Algorithm 3 and the
+ * window-2 convolution conv_1d(q_t, q_{t-1}) of its Algorithm 6 page.  Apply
+ * it to each of q, k, v before ssd_fwd (it is not fused into the operator).
+ *   x      device, [B, H, N, d_h], element type `dtype` (pre-convolution)
+ *   w      device, [H*d_h, width] fp32; w[c][j] multiplies token t - j of
+ *          channel c = h*d_h + channel (j = 0 is the current token)
+ *   bias   device, [H*d_h] fp32, or NULL
+ *   width  1..4 (the pages use 2)
+ *   silu   nonzero: out = SiLU(u) = u / (1 + e^-u), else out = u
+ *   out    device, [B, H, N, d_h], `dtype`; must not overlap x
+ * Tokens before the first of each (b, h) count as zero.  Asynchronous on
+ * `stream`.  Returns SSD_OK, SSD_ERR_NULL, SSD_ERR_DTYPE, SSD_ERR_SHAPE
+ * (sizes, width, or out overlapping x), SSD_ERR_ALIGN (x, out 16 bytes;
+ * w, bias 4 bytes) or SSD_ERR_CUDA.
+ */
+int ssd_conv1d(const void *x, const float *w, const float *bias, int B, int H, int N, int d_h,
+               int width, int silu, int dtype, void *out, void *stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *ssd_status_str(int status);
 

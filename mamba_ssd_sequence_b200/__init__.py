@@ -60,6 +60,8 @@ def load_library():
     lib.ssd_decode_workspace_bytes.restype = sz
     lib.ssd_decode_step.argtypes = [vp] * 8 + [ci] * 7 + [vp, vp, vp, vp, sz, vp]
     lib.ssd_decode_step.restype = ci
+    lib.ssd_conv1d.argtypes = [vp] * 3 + [ci] * 7 + [vp, vp]
+    lib.ssd_conv1d.restype = ci
     lib.ssd_fwd_host.argtypes = [vp] * 7 + [ci] * 8 + [vp] + [vp] * 8 + [vp, sz, vp]
     lib.ssd_fwd_host.restype = ci
     lib.ssd_chunk_cumsum.argtypes = [vp] * 3 + [ci] * 4 + [vp, vp, vp]
@@ -266,3 +268,17 @@ def ssd_status_from_workspace(workspace, stream=None) -> int:
     """Synchronise and read the device status left in the workspace."""
     return int(load_library().ssd_status_from_workspace(_ptr(workspace),
                                                         _stream_handle(stream)))
+
+
+def ssd_conv1d(x, w, bias=None, silu: bool = True, out=None, stream=None):
+    """Causal depthwise conv over tokens (+ SiLU) on a CUDA tensor
+    (include/ssd.h, ssd_conv1d): x [B, H, N, d_h]; w [H*d_h, width] float32
+    (w[:, j] multiplies token t - j); bias [H*d_h] or None.  Returns `out`."""
+    import torch
+    B, H, N, d = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    rc = load_library().ssd_conv1d(_ptr(x), _ptr(w), _ptr(bias), B, H, N, d, int(w.shape[1]),
+                                   int(bool(silu)), _dtype_code(x), _ptr(out), _stream_handle(stream))
+    _check(rc, "ssd_conv1d")
+    return out

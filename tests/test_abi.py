@@ -168,3 +168,16 @@ def test_state_and_decode_validation_codes(lib):
     assert dec(h=136) == 6
     assert dec(dt_p=66) == 6                      # per-token scalars need 4-byte alignment
     assert dec(wsb=100) == 7
+
+
+def test_conv1d_validation_codes(lib):
+    def cv(**o):
+        a = dict(x=1024, w=64, b=None, B=1, H=2, N=8, d=16, width=2, silu=1, dtype=ssd.SSD_BF16, out=4096)
+        a.update(o)
+        return lib.ssd_conv1d(a["x"], a["w"], a["b"], a["B"], a["H"], a["N"], a["d"], a["width"], a["silu"],
+                              a["dtype"], a["out"], None)
+    assert cv(x=None) == 1 and cv(w=None) == 1 and cv(out=None) == 1
+    assert cv(dtype=4) == 3
+    assert cv(width=0) == 2 and cv(width=5) == 2 and cv(d=24) == 2 and cv(N=0) == 2
+    assert cv(x=1032) == 6 and cv(w=66) == 6
+    assert cv(out=1024 + 256) == 2       # out overlaps x

@@ -1,0 +1,65 @@
+"""Parity of the conv1d + SiLU prologue (2Mamba2Furious Algorithm 3's
+Q, K, V = SiLU(conv_1d(h W_QKV)), window 2 on the Algorithm 6 page) with the
+CPU oracle, alone and followed by the operator."""
+import numpy as np
+import pytest
+
+import mamba_ssd_sequence_b200 as ssd
+import oracle
+from mamba_ssd_sequence_b200 import inputs
+from helpers import TOL, rel_err, to_device
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+def _weights(H, d, width, seed):
+    rng = np.random.default_rng(seed)
+    w = (rng.standard_normal((H * d, width)) / np.sqrt(width)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(H * d)).astype(np.float32)
+    return w, b
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("width", [1, 2, 3, 4])
+@pytest.mark.parametrize("silu,use_bias", [(True, True), (False, False), (True, False)])
+def test_conv1d_matches_oracle(dtype, width, silu, use_bias):
+    B, H, N, d = 2, 3, 77, 32
+    x = inputs.make_inputs(B, H, N, d, dtype, seed=51)
+    w, b = _weights(H, d, width, 51)
+    dev = to_device(x, dtype)
+    wd = torch.from_numpy(w).cuda()
+    bd = torch.from_numpy(b).cuda() if use_bias else None
+    y = ssd.ssd_conv1d(dev["q"], wd, bd, silu=silu)
+    torch.cuda.synchronize()
+    ref = oracle.conv1d(x["q"], w, b if use_bias else None, silu=silu)
+    got = y.float().cpu().numpy().astype(np.float64)
+    # the operator's measure, max|d| / max|ref|: an elementwise relative error
+    # is meaningless where the window's terms cancel; fp32 accumulation of a
+    # few terms, and bf16 output rounding (2^-9 relative) bound it
+    tol = 1e-5 if dtype == "f32" else 2 ** -8
+    assert rel_err(got, ref) <= tol
+
+
+def test_prologue_then_operator():
+    """conv1d + SiLU on q, k, v, then the order-1 tensor-core operator, agrees
+    with the oracle's prologue followed by the oracle's operator."""
+    B, H, N, d, chunk = 1, 2, 384, 64, 128
+    x = inputs.make_inputs(B, H, N, d, "bf16", seed=52, residual=True)
+    dev = to_device(x, "bf16")
+    conv = {}
+    ref_in = {}
+    for i, name in enumerate(("q", "k", "v")):
+        w, b = _weights(H, d, 2, 60 + i)
+        conv[name] = ssd.ssd_conv1d(dev[name], torch.from_numpy(w).cuda(), torch.from_numpy(b).cuda())
+        r = oracle.conv1d(x[name], w, b).astype(np.float32)
+        ref_in[name] = inputs.bf16_bits_to_f32(inputs.bf16_round_bits(r))  # the operator reads bf16
+    y = ssd.ssd_fwd(conv["q"], conv["k"], conv["v"], dev["dt_p"], dev["A_log"], dev["dt_bias"], dev["D"],
+                    1, False, chunk)
+    torch.cuda.synchronize()
+    ref = oracle.ssd_quadratic(ref_in["q"], ref_in["k"], ref_in["v"], x["dt_p"], x["A_log"], x["dt_bias"],
+                               x["D"], 1, False)
+    assert rel_err(y.float().cpu().numpy().astype(np.float64), ref) <= TOL["bf16"]
