@@ -101,6 +101,7 @@ static_assert(sizeof(StateMisc<256>) <= StateCfg<256>::MISC_BYTES, "misc block")
 template <int C>
 __global__ void __launch_bounds__(StateCfg<C>::THREADS, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_u,
                    const float *__restrict__ dt_p, const float *__restrict__ A_log,
                    const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int value_dt,
                    int H, int N, int n_chunks, float *__restrict__ acs_out, float *__restrict__ vfac_out,
@@ -125,7 +126,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         for (int i = 0; i < K::STAGES; ++i) {
             mbar_init(&misc->stage_full[i], 1);
-            mbar_init(&misc->stage_empty[i], 1);
+            // released by the U product (tcgen05.commit) and by the compute group
+            // once U^T, staged over K', has been stored
+            mbar_init(&misc->stage_empty[i], 2);
         }
         for (int b = 0; b < NG; ++b) {
             mbar_init(&misc->kp_full[b], kStateGroup);
@@ -150,6 +153,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         if (lane == 0) {
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_u);
             int i = 0;
             for (int t = blockIdx.x; t < n_chunks; t += gridDim.x, ++i) {
                 const int st = i % K::STAGES;
@@ -306,15 +310,29 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&misc->u_free[gi]);
+            // U^T rows n = 16 g + lane, staged over K' (read by the finished
+            // product) as two 64 x 32 fp32 boxes in the 128-byte swizzle
             if (lane < 16) {
-                float4 *dst = reinterpret_cast<float4 *>(Ut + ((size_t)t * 64 + g * 16 + lane) * 64);
+                const int n = g * 16 + lane;
 #pragma unroll
-                for (int q = 0; q < 8; ++q) dst[q] = make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    dst[8 + q] = make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
+                for (int q = 0; q < 8; ++q) {
+                    *reinterpret_cast<float4 *>(sk + sw128_chunk(n, q)) =
+                        make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
+                    *reinterpret_cast<float4 *>(sk + 8192 + sw128_chunk(n, q)) =
+                        make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(bar, kStateGroup);
+            if (gt == 0) {
+                tma_store_2d(&tm_u, sk, 0, t * 64);
+                tma_store_2d(&tm_u, sk + 8192, 32, t * 64);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                mbar_arrive(&misc->stage_empty[st]);
             }
         }
+        if (gt == 0) bulk_wait_group0();  // every U^T tile has reached global memory
         if (failed && gt == 0) set_timeout(status, 102, &misc->abort_flag);
     }
 
@@ -461,7 +479,7 @@ template <int C>
 __global__ void __launch_bounds__(ScanCfg<C>::THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
-                  const __nv_bfloat16 *__restrict__ vglob, __nv_bfloat16 *__restrict__ out,
+                  const __grid_constant__ CUtensorMap tm_out,
                   const float *__restrict__ acs_in, const float *__restrict__ vfac_in,
                   const float *__restrict__ Dres, int H, int N, int n_tiles, DeviceStatus *status) {
     using K = ScanCfg<C>;
@@ -480,7 +498,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0) {
         for (int i = 0; i < K::STAGES; ++i) {
             mbar_init(&misc->stage_full[i], 1);
-            mbar_init(&misc->stage_empty[i], 1);
+            // released by the P V product (tcgen05.commit) and by the compute
+            // group once its output tile, staged over Q, has been stored
+            mbar_init(&misc->stage_empty[i], 2);
         }
         for (int i = 0; i < K::NSB; ++i) mbar_init(&misc->s_full[i], 1);
         for (int gi = 0; gi < NG; ++gi)
@@ -509,6 +529,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_h);
+            prefetch_tmap(&tm_out);
             pdl_wait();  // hin (state pass) and everything before it are visible
             int i = 0;
             for (; i < my_tiles; ++i) {
@@ -663,14 +684,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             const Raw raw = raw_next;
             raw_next = fetch(i + NG);
             const int ir = 128 * x.rb + r;  // chunk-local row
-            const size_t grow = (size_t)x.bh * N + (size_t)x.c * C + ir;
-            uint4 vr[4];
-            if (Dres) {
-                const uint4 *vp = reinterpret_cast<const uint4 *>(vglob + grow * kD + hf * 32);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) vr[q] = __ldg(vp + q);
-                if (ct < 16) *reinterpret_cast<float4 *>(&misc->dres[gi][slot][4 * ct]) = raw.d;
-            }
+            uint8_t *sp = smem + (i % K::STAGES) * K::STAGE;
+            if (Dres && ct < 16) *reinterpret_cast<float4 *>(&misc->dres[gi][slot][4 * ct]) = raw.d;
             // chunk-local cumulative decay of key ct, and its factor to the end of its 32-key block
             const float aref = __shfl_sync(0xffffffffu, raw.acs, 31);
             if (ct < C) {
@@ -743,6 +758,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             // ---- epilogue: y = Y + 2^acs_i Z [+ D v], columns [32 hf, 32 hf + 32)
             bad = !mbar_wait_abortable(&misc->y_full[tb], (i >> 1) & 1, abort_flag);
+            // the V box is read below: observe the stage's TMA completion here too
+            // (long complete; the stage cannot be refilled before this group releases it)
+            bad = bad || !mbar_wait_abortable(&misc->stage_full[i % K::STAGES], (i / K::STAGES) & 1, abort_flag);
             if (named_bar_any(bar, 256, bad)) {
                 failed = true;
                 break;
@@ -750,7 +768,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_after();
             const float e = ex2_approx(ai);
             const float *dh = &misc->dres[gi][slot][hf * 32];
-            uint4 *op = reinterpret_cast<uint4 *>(out + grow * kD + hf * 32);
+            // residual v_i: row r of V box rb (this tile's own tokens); y is
+            // staged over Q (dead since S' completed) in the same swizzled layout
+            const uint8_t *vrow = sp + K::V_OFF + x.rb * kBox;
+            uint8_t *ytile = sp + K::Q_OFF;
             const uint32_t zc = tmem + lane_off + z_col<C>(sb) + 32 * hf;
             const uint32_t yc = tmem + lane_off + K::COL_Y + 64 * tb + 32 * hf;
 #pragma unroll
@@ -767,7 +788,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int q2 = 0; q2 < 2; ++q2) {
                     const int q = 2 * half + q2;
                     uint32_t wv[4];
-                    const uint32_t vw[4] = {vr[q].x, vr[q].y, vr[q].z, vr[q].w};
+                    uint4 vq = make_uint4(0u, 0u, 0u, 0u);
+                    if (Dres) vq = *reinterpret_cast<const uint4 *>(vrow + sw128_chunk(r, 4 * hf + q));
+                    const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w};
 #pragma unroll
                     for (int pp = 0; pp < 4; ++pp) {
                         const int cl = q2 * 8 + 2 * pp;  // column within the half
@@ -780,10 +803,21 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         }
                         wv[pp] = pack_bf16x2(y0, y1);
                     }
-                    op[q] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                    *reinterpret_cast<uint4 *>(ytile + sw128_chunk(r, 4 * hf + q)) =
+                        make_uint4(wv[0], wv[1], wv[2], wv[3]);
                 }
             }
+            // one TMA store per tile; the stage is released once it has been read
+            fence_proxy_async_smem();
+            named_bar_sync(bar, 256);
+            if (ct == 0) {
+                tma_store_2d(&tm_out, ytile, 0, x.bh * N + x.c * C + 128 * x.rb);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+                mbar_arrive(&misc->stage_empty[i % K::STAGES]);
+            }
         }
+        if (ct == 0) bulk_wait_group0();  // every output tile has reached global memory
         if (failed && ct == 0) set_timeout(status, 130, &misc->abort_flag);
     }
 
@@ -822,6 +856,21 @@ bool make_tmap64(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_r
     return r == CUDA_SUCCESS;
 }
 
+// [rows, 64] fp32 row-major tensor written in boxes of 64 rows x 32 columns,
+// 128-byte swizzle.
+bool make_tmap_f32x64(CUtensorMap *m, void *base, uint64_t rows) {
+    auto enc = get_encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {64, rows};
+    cuuint64_t strides[1] = {64 * 4};
+    cuuint32_t box[2] = {32, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Sets the dynamic shared-memory limit of `fn` once per device.
 template <typename F>
 bool smem_attr_once(F fn, int bytes, std::atomic<uint64_t> &done) {
@@ -854,10 +903,13 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     float *vfac = a.value_dt ? reinterpret_cast<float *>(ws + p.vfac_off) : nullptr;
     float *U = reinterpret_cast<float *>(ws + p.state_off);
     __nv_bfloat16 *hin = reinterpret_cast<__nv_bfloat16 *>(ws + p.aux_off);
-    CUtensorMap tq, tk, tv, th;
+    CUtensorMap tq, tk, tv, th, to;
     if (!make_tmap64(&tq, a.q, rows, 128) || !make_tmap64(&tk, a.k, rows, 128) ||
-        !make_tmap64(&tv, a.v, rows, 128) || !make_tmap64(&th, hin, (uint64_t)BH * nc * 64, 64))
+        !make_tmap64(&tv, a.v, rows, 128) || !make_tmap64(&th, hin, (uint64_t)BH * nc * 64, 64) ||
+        !make_tmap64(&to, a.out, rows, 128))
         return SSD_ERR_CUDA;
+    CUtensorMap tu;
+    if (!make_tmap_f32x64(&tu, U, (uint64_t)BH * nc * 64)) return SSD_ERR_CUDA;
     static std::atomic<uint64_t> attr1{0}, attr3{0};
     if (!smem_attr_once(chunk_state_kernel<C>, (int)StateCfg<C>::SMEM, attr1) ||
         !smem_attr_once(chunk_scan_kernel<C>, (int)K::SMEM, attr3))
@@ -867,7 +919,7 @@ int launch_c(const FwdArgs &a, const Plan &p) {
 
     const int n_chunks = BH * nc;
     chunk_state_kernel<C><<<n_chunks < sms ? n_chunks : sms, StateCfg<C>::THREADS, StateCfg<C>::SMEM, a.stream>>>(
-        tk, tv, a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N, n_chunks, acs, vfac, U, lam,
+        tk, tv, tu, a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N, n_chunks, acs, vfac, U, lam,
         status);
     // The state pass and the chunk scan are launched as programmatic dependents:
     // their CTAs may start while the previous kernel drains, and each waits
@@ -893,9 +945,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c3.stream = a.stream;
     c3.attrs = pdl;
     c3.numAttrs = 1;
-    if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, static_cast<const __nv_bfloat16 *>(a.v),
-                           static_cast<__nv_bfloat16 *>(a.out), (const float *)acs, (const float *)vfac, a.D,
-                           a.H, a.N, n_tiles, status) != cudaSuccess)
+    if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, to, (const float *)acs, (const float *)vfac,
+                           a.D, a.H, a.N, n_tiles, status) != cudaSuccess)
         return SSD_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
