@@ -124,7 +124,8 @@ __device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16 *__restrict__ out,
+                 const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ vglob,
+                 __nv_bfloat16 *__restrict__ out,
                  const float *__restrict__ dt_p, const float *__restrict__ A_log,
                  const float *__restrict__ dt_bias, const float *__restrict__ Dres,
                  const float *__restrict__ log_decay, int H, int N,
@@ -305,6 +306,70 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // per-token decay input: the dt projection, or the given log-decay (Algorithm 4)
         const float *dsrc = log_decay ? log_decay : dt_p;
         float dt_next = (ct < kC && nc > 0) ? dsrc[(size_t)row0 + ct] : 0.0f;
+        bool failed = false;
+        // Own rows of chunk cc: sum the R partials (distributed shared memory),
+        // release them, then y = (Y + T) / (r + Tn) [+ D v].
+        auto reduce_output = [&](int cc) -> bool {
+            const bool bad = !mbar_wait_cluster(&misc->ready[cc & 1], (cc >> 1) & 1, abort_flag);
+            if (named_bar_any(1, kTeam, bad)) {
+                if (elected) raise_timeout(misc, status, 34);
+                return false;
+            }
+            {
+                constexpr int NV = D / 4 + 1;  // float4 groups of a row, plus the normaliser
+                const uint32_t pb = smem_u32(part0 + (cc & 1) * kC * K::PR);
+                for (int it = ct; it < K::ROWS * NV; it += kTeam) {
+                    const int rr = it / NV, v = it % NV;
+                    const int row = rank * K::ROWS + rr;
+                    const uint32_t off = (uint32_t)(row * K::PR + (v < D / 4 ? v * 4 : D)) * 4u;
+                    if (v < D / 4) {
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                        for (int r2 = 0; r2 < K::R; ++r2) {
+                            const float4 x = ld_dsmem_f4(mapa_shared(pb + off, r2));
+                            acc.x += x.x;
+                            acc.y += x.y;
+                            acc.z += x.z;
+                            acc.w += x.w;
+                        }
+                        *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc;
+                    } else {
+                        float acc = 0.0f;
+                        for (int r2 = 0; r2 < K::R; ++r2) acc += ld_dsmem_f1(mapa_shared(pb + off, r2));
+                        res[rr * K::PR + D] = acc;
+                    }
+                }
+            }
+            named_bar_sync(1, kTeam);
+            if (ct < K::R) {
+                fence_acq_rel_cluster();
+                mbar_arrive_cluster(mapa_shared(smem_u32(&misc->consumed[cc & 1]), ct));
+            }
+            for (int it = ct; it < K::ROWS * (D / 8); it += kTeam) {
+                const int rr = it / (D / 8), ch = it % (D / 8);
+                const int row = rank * K::ROWS + rr;
+                const size_t grow = (size_t)row0 + (size_t)cc * kC + row;
+                const float *rrow = res + rr * K::PR;
+                const float inv = normalize ? 1.0f / rrow[D] : 1.0f;
+                uint4 vu = make_uint4(0u, 0u, 0u, 0u);
+                if (Dres) vu = __ldg(reinterpret_cast<const uint4 *>(vglob + grow * D + ch * 8));
+                const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c2 = ch * 8 + 2 * e;
+                    float y0 = rrow[c2] * inv, y1 = rrow[c2 + 1] * inv;
+                    if (Dres) {
+                        const float2 vf = bf2_to_f2(vw[e]);
+                        y0 = fmaf(misc->Dh[c2], vf.x, y0);
+                        y1 = fmaf(misc->Dh[c2 + 1], vf.y, y1);
+                    }
+                    w[e] = pack_bf16x2(y0, y1);
+                }
+                *reinterpret_cast<uint4 *>(out + grow * D + ch * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            named_bar_sync(1, kTeam);  // res is reused by the next reduction
+            return true;
+        };
         for (int c = 0; c < nc; ++c) {
             const int st = c % kStages;
             uint8_t *sQ = smem + K::OFF_STAGE + st * K::STAGE;
@@ -457,11 +522,19 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 ++slab_uses[b];
             }
 
+            // ---- the previous chunk's cluster reduction and output run here,
+            // while this chunk's last slab products are still on the tensor core
+            if (c >= 1 && !reduce_output(c - 1)) {
+                failed = true;
+                break;
+            }
+
             // ---- this CTA's partial (plus Y and r on its own rows) into part[c & 1]
             bad = !mbar_wait_abortable(&misc->chunk_done, c & 1, abort_flag);
             bad = bad || (c >= 2 && !mbar_wait_cluster(&misc->consumed[c & 1], ((c >> 1) - 1) & 1, abort_flag));
             if (named_bar_any(1, kTeam, bad)) {
                 if (elected) raise_timeout(misc, status, 33);
+                failed = true;
                 break;
             }
             tc_fence_after();
@@ -501,73 +574,17 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
             }
             named_bar_sync(1, kTeam);
-            if (elected) {
+            // thread r announces this CTA's partial to cluster CTA r; the R remote
+            // arrivals (each a cluster-scope release) run in parallel
+            if (ct < K::R) {
                 fence_acq_rel_cluster();
-                const uint32_t rdy = smem_u32(&misc->ready[c & 1]);
-                for (int r2 = 0; r2 < K::R; ++r2) mbar_arrive_cluster(mapa_shared(rdy, r2));
+                mbar_arrive_cluster(mapa_shared(smem_u32(&misc->ready[c & 1]), ct));
             }
-
-            // ---- own rows: sum the R partials (distributed shared memory), epilogue
-            bad = !mbar_wait_cluster(&misc->ready[c & 1], (c >> 1) & 1, abort_flag);
-            if (named_bar_any(1, kTeam, bad)) {
-                if (elected) raise_timeout(misc, status, 34);
-                break;
-            }
-            {
-                constexpr int NV = D / 4 + 1;  // float4 groups of a row, plus the normaliser
-                const uint32_t pb = smem_u32(part0 + (c & 1) * kC * K::PR);
-                for (int it = ct; it < K::ROWS * NV; it += kTeam) {
-                    const int rr = it / NV, v = it % NV;
-                    const int row = rank * K::ROWS + rr;
-                    const uint32_t off = (uint32_t)(row * K::PR + (v < D / 4 ? v * 4 : D)) * 4u;
-                    if (v < D / 4) {
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int r2 = 0; r2 < K::R; ++r2) {
-                            const float4 x = ld_dsmem_f4(mapa_shared(pb + off, r2));
-                            acc.x += x.x;
-                            acc.y += x.y;
-                            acc.z += x.z;
-                            acc.w += x.w;
-                        }
-                        *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc;
-                    } else {
-                        float acc = 0.0f;
-                        for (int r2 = 0; r2 < K::R; ++r2) acc += ld_dsmem_f1(mapa_shared(pb + off, r2));
-                        res[rr * K::PR + D] = acc;
-                    }
-                }
-            }
-            named_bar_sync(1, kTeam);
-            if (elected) {
-                fence_acq_rel_cluster();
-                const uint32_t cns = smem_u32(&misc->consumed[c & 1]);
-                for (int r2 = 0; r2 < K::R; ++r2) mbar_arrive_cluster(mapa_shared(cns, r2));
-            }
-            for (int it = ct; it < K::ROWS * (D / 8); it += kTeam) {
-                const int rr = it / (D / 8), ch = it % (D / 8);
-                const int row = rank * K::ROWS + rr;
-                const float *rrow = res + rr * K::PR;
-                const float inv = normalize ? 1.0f / rrow[D] : 1.0f;
-                const uint4 vu = *reinterpret_cast<const uint4 *>(sV + swz<K::RB>(row, ch));
-                const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int cc = ch * 8 + 2 * e;
-                    float y0 = rrow[cc] * inv, y1 = rrow[cc + 1] * inv;
-                    if (Dres) {
-                        const float2 vf = bf2_to_f2(vw[e]);
-                        y0 = fmaf(misc->Dh[cc], vf.x, y0);
-                        y1 = fmaf(misc->Dh[cc + 1], vf.y, y1);
-                    }
-                    w[e] = pack_bf16x2(y0, y1);
-                }
-                *reinterpret_cast<uint4 *>(out + (size_t)(row0 + c * kC + row) * D + ch * 8) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            named_bar_sync(1, kTeam);
+            // the stage is no longer read: features are built, the products are
+            // done and the output reads v from global memory
             if (elected) mbar_arrive(&misc->stage_empty[st]);
         }
+        if (!failed && nc >= 1) reduce_output(nc - 1);
     done:;
     }
 
@@ -638,6 +655,7 @@ int launch_d(const FwdArgs &a) {
     cfg.numAttrs = 1;
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
     cudaError_t e = cudaLaunchKernelEx(&cfg, tc_order2_kernel<D>, tq, tk, tv,
+                                       static_cast<const __nv_bfloat16 *>(a.v),
                                        static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log,
                                        a.dt_bias, a.D, a.log_decay, a.H, a.N, a.normalize, status);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
