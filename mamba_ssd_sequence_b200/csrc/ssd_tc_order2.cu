@@ -309,7 +309,14 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool failed = false;
         // Own rows of chunk cc: sum the R partials (distributed shared memory),
         // release them, then y = (Y + T) / (r + Tn) [+ D v].
+        static_assert(K::ROWS * (D / 8) <= kTeam, "one output item per thread");
         auto reduce_output = [&](int cc) -> bool {
+            // this thread's output item and its residual input, fetched before the waits
+            const int o_rr = ct / (D / 8), o_ch = ct % (D / 8);
+            const bool o_live = ct < K::ROWS * (D / 8);
+            const size_t o_grow = (size_t)row0 + (size_t)cc * kC + rank * K::ROWS + o_rr;
+            uint4 vu = make_uint4(0u, 0u, 0u, 0u);
+            if (Dres && o_live) vu = __ldg(reinterpret_cast<const uint4 *>(vglob + o_grow * D + o_ch * 8));
             const bool bad = !mbar_wait_cluster(&misc->ready[cc & 1], (cc >> 1) & 1, abort_flag);
             if (named_bar_any(1, kTeam, bad)) {
                 if (elected) raise_timeout(misc, status, 34);
@@ -322,19 +329,28 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     const int rr = it / NV, v = it % NV;
                     const int row = rank * K::ROWS + rr;
                     const uint32_t off = (uint32_t)(row * K::PR + (v < D / 4 ? v * 4 : D)) * 4u;
+                    // all R remote loads are issued before any is used, so their
+                    // latencies overlap
                     if (v < D / 4) {
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                        for (int r2 = 0; r2 < K::R; ++r2) {
-                            const float4 x = ld_dsmem_f4(mapa_shared(pb + off, r2));
-                            acc.x += x.x;
-                            acc.y += x.y;
-                            acc.z += x.z;
-                            acc.w += x.w;
+                        float4 x[K::R];
+#pragma unroll
+                        for (int r2 = 0; r2 < K::R; ++r2) x[r2] = ld_dsmem_f4(mapa_shared(pb + off, r2));
+                        float4 acc = x[0];
+#pragma unroll
+                        for (int r2 = 1; r2 < K::R; ++r2) {
+                            acc.x += x[r2].x;
+                            acc.y += x[r2].y;
+                            acc.z += x[r2].z;
+                            acc.w += x[r2].w;
                         }
                         *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc;
                     } else {
-                        float acc = 0.0f;
-                        for (int r2 = 0; r2 < K::R; ++r2) acc += ld_dsmem_f1(mapa_shared(pb + off, r2));
+                        float x[K::R];
+#pragma unroll
+                        for (int r2 = 0; r2 < K::R; ++r2) x[r2] = ld_dsmem_f1(mapa_shared(pb + off, r2));
+                        float acc = x[0];
+#pragma unroll
+                        for (int r2 = 1; r2 < K::R; ++r2) acc += x[r2];
                         res[rr * K::PR + D] = acc;
                     }
                 }
@@ -344,14 +360,11 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 fence_acq_rel_cluster();
                 mbar_arrive_cluster(mapa_shared(smem_u32(&misc->consumed[cc & 1]), ct));
             }
-            for (int it = ct; it < K::ROWS * (D / 8); it += kTeam) {
-                const int rr = it / (D / 8), ch = it % (D / 8);
-                const int row = rank * K::ROWS + rr;
-                const size_t grow = (size_t)row0 + (size_t)cc * kC + row;
+            if (o_live) {
+                const int rr = o_rr, ch = o_ch;
+                const size_t grow = o_grow;
                 const float *rrow = res + rr * K::PR;
                 const float inv = normalize ? 1.0f / rrow[D] : 1.0f;
-                uint4 vu = make_uint4(0u, 0u, 0u, 0u);
-                if (Dres) vu = __ldg(reinterpret_cast<const uint4 *>(vglob + grow * D + ch * 8));
                 const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
                 uint32_t w[4];
 #pragma unroll
