@@ -67,6 +67,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# DRAM bytes of one call, dram__bytes_read.sum + dram__bytes_write.sum summed
+# over the path's kernels, from the ncu captures summarised under profiles/
+# (taken on the kernels in this tree; a workload without a capture of the
+# current kernels reports null).
+DRAM_TRAFFIC = {
+    # chunk states 34.10 MB + state pass 0.04 MB + chunk outputs 24.29 MB,
+    # captured without cache flushes, as the kernels run in a call
+    "order1-bf16-B4H16N2048d64-c128": 58_443_008,
+    # one launch, captured after an L2 flush (as in the bench)
+    "order2-bf16-B4H16N4096d32-c64": 52_358_912,
+}
+
+
 def algorithmic_work(w: inputs.Workload):
     """Per-launch algorithmic bytes and FLOPs of one call.
 
@@ -374,7 +387,7 @@ def main():
         "tc_frac": tflops / float(peaks["bf16_tflops"]),
         "hbm_gbs": gbs,
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": DRAM_TRAFFIC.get(w.name),
                      "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "algorithmic_flops_per_launch": alg_flops},
