@@ -67,8 +67,12 @@ struct Cfg {
     static constexpr uint32_t OFF_FK = OFF_P + 8192;                      // 2 x 16 KiB
     static constexpr uint32_t OFF_FQ = OFF_FK + 2 * 16384;                // 2 x 16 KiB
     static constexpr uint32_t OFF_HB = OFF_FQ + 2 * 16384;                // 2 x 128 rows
-    static constexpr uint32_t OFF_ZB = OFF_HB + 2 * kSlab * RB;           // 2 x 128 x 32 B
-    static constexpr uint32_t OFF_ONES = OFF_ZB + 2 * 4096;               // 64 x 32 B
+    // z entering the chunk, one 128-row tile per buffer in hb's layout with z in
+    // column 0 and zeros elsewhere: hb and zb form one B operand of 2 D columns
+    // (two MN atoms LBO_HZ bytes apart), so T and Tn come from one product
+    static constexpr uint32_t OFF_ZB = OFF_HB + 2 * kSlab * RB;           // 2 x 128 rows
+    static constexpr uint32_t LBO_HZ = OFF_ZB - OFF_HB;
+    static constexpr uint32_t OFF_ONES = OFF_ZB + 2 * kSlab * RB;         // 64 x 32 B
     static constexpr uint32_t OFF_PART = OFF_ONES + 2048;                 // 2 x 64 x PR fp32
     static constexpr uint32_t OFF_RES = OFF_PART + 2 * kC * PR * 4;       // ROWS x PR fp32
     static constexpr uint32_t OFF_MISC = (OFF_RES + ROWS * PR * 4 + 1023) / 1024 * 1024;
@@ -77,9 +81,9 @@ struct Cfg {
     static constexpr uint32_t COL_H = 0;                   // kNs x D   h    (M = 128)
     static constexpr uint32_t COL_Z = COL_H + kNs * D;     // kNs x 16  z    (M = 128)
     static constexpr uint32_t COL_S = COL_Z + kNs * 16;    // 64: S, then Y = P V (M = 64)
-    static constexpr uint32_t COL_T = COL_S + 64;          // D: partial state readout (M = 64)
-    static constexpr uint32_t COL_TN = COL_T + D;          // 16: partial normaliser (M = 64)
-    static_assert(COL_TN + 16 <= 512, "TMEM budget");
+    static constexpr uint32_t COL_T = COL_S + 64;          // 2 D: partial readout [T | Tn 0...] (M = 64)
+    static constexpr uint32_t COL_TN = COL_T + D;          // Tn: first column of the second half
+    static_assert(COL_T + 2 * D <= 512, "TMEM budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -171,6 +175,9 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_alloc(&misc->tmem_base, 512);
         tmem_relinquish();
     }
+    // zb tiles: zero once; only column 0 of each row is written later
+    for (int i = tid; i < (int)(2 * kSlab * K::RB / 16); i += kThreads)
+        reinterpret_cast<uint4 *>(smem + K::OFF_ZB)[i] = make_uint4(0u, 0u, 0u, 0u);
     // constant B operand: [1, 0, ..., 0] per token (64 rows x 16 bf16, 32B swizzle)
     for (int i = tid; i < kC * 2; i += kThreads) {
         const int r = i >> 1, ch = i & 1;
@@ -218,7 +225,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             constexpr uint32_t idU = make_idesc_bf16(128, D, 1, 1);
             constexpr uint32_t idZ = make_idesc_bf16(128, 16, 1, 1);
             constexpr uint32_t idT = make_idesc_bf16(64, D, 0, 1);
-            constexpr uint32_t idTn = make_idesc_bf16(64, 16, 0, 1);
+            constexpr uint32_t idT2 = make_idesc_bf16(64, 2 * D, 0, 1);  // [T | Tn] in one product
             uint32_t slab_uses[2] = {0, 0};
             bool ok = true;
             for (int c = 0; ok && c < nc; ++c) {
@@ -259,18 +266,16 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                      (c > 0 || ks > 0));
                     }
                     if (c >= 1) {
-                        // T += Fq hb ;  Tn += Fq zb   (A: tokens x features, K-major)
+                        // [T | Tn] += Fq [hb | zb]   (A: tokens x features, K-major;
+                        // B: the hb and zb tiles as two MN atoms)
                         const uint32_t hbB = sbase + K::OFF_HB + b * kSlab * K::RB;
-                        const uint32_t zbB = sbase + K::OFF_ZB + b * 4096;
 #pragma unroll
                         for (int ks = 0; ks < kSlab / 16; ++ks) {
                             const uint64_t adesc =
                                 make_sdesc(fqA + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128);
-                            mma_bf16(tmem + K::COL_T, adesc, make_sdesc(hbB + ks * 16 * K::RB, 16, K::SBO, K::SW),
-                                     idT, (sl > 0 || ks > 0));
-                            if (normalize)
-                                mma_bf16(tmem + K::COL_TN, adesc, make_sdesc(zbB + ks * 512, 16, 256, kSw32), idTn,
-                                         (sl > 0 || ks > 0));
+                            mma_bf16(tmem + K::COL_T, adesc,
+                                     make_sdesc(hbB + ks * 16 * K::RB, K::LBO_HZ, K::SBO, K::SW),
+                                     normalize ? idT2 : idT, (sl > 0 || ks > 0));
                         }
                     }
                     mma_commit(&misc->slab_done[b]);
@@ -490,10 +495,10 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if constexpr (HC == 32) tmem_st32(ta, hv);
                     else tmem_st16(ta, hv);
                     if (normalize && hf == 0) {
-                        uint8_t *zb = smem + K::OFF_ZB + b * 4096;
-                        *reinterpret_cast<uint4 *>(zb + sw32_chunk(frow, 0)) =
+                        // column 0 of the zb row; the rest of the tile stays zero
+                        uint8_t *zb = smem + K::OFF_ZB + b * kSlab * K::RB;
+                        *reinterpret_cast<uint4 *>(zb + swz<K::RB>(frow, 0)) =
                             make_uint4(pack_bf16x2(zv, 0.0f), 0u, 0u, 0u);
-                        *reinterpret_cast<uint4 *>(zb + sw32_chunk(frow, 1)) = make_uint4(0u, 0u, 0u, 0u);
                         tmem_st1(tmem + lane_off + K::COL_Z + sl * 16, zv * dec);
                     }
                 }
