@@ -346,6 +346,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // =====================================================================
 // (2) state passing: one thread per 4 state entries of a head
 // =====================================================================
+template <int kBatch>
 __global__ void __launch_bounds__(256)
 state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __nv_bfloat16 *__restrict__ hin,
                   int nc, const float *__restrict__ h0, float *__restrict__ h_out) {
@@ -364,19 +365,21 @@ state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __
         const float *hp = h0 + (size_t)bh * 4096 + (size_t)k_ * 64 + n_;
         hs = make_float4(hp[0], hp[64], hp[128], hp[192]);
     }
-    // eight chunks' inputs are in flight before the dependent updates run
-    for (int c0 = 0; c0 < nc; c0 += 8) {
-        float4 ub[8];
-        float fb[8];
+    // kBatch chunks' inputs are in flight before the dependent updates run
+    // (16: a head of up to 16 chunks costs one L2 round trip; 8 for longer
+    // heads, which keeps more threads resident)
+    for (int c0 = 0; c0 < nc; c0 += kBatch) {
+        float4 ub[kBatch];
+        float fb[kBatch];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kBatch; ++j) {
             if (c0 + j < nc) {
                 ub[j] = __ldg(u + (size_t)(c0 + j) * 1024);
                 fb[j] = __ldg(lm + c0 + j);
             }
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < kBatch; ++j) {
             if (c0 + j < nc) {
                 const float f = ex2_approx(fb[j]);
                 out[(size_t)(c0 + j) * 1024] = make_uint2(pack_bf16x2(hs.x, hs.y), pack_bf16x2(hs.z, hs.w));
@@ -933,8 +936,12 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c2.stream = a.stream;
     c2.attrs = pdl;
     c2.numAttrs = 1;
-    if (cudaLaunchKernelEx(&c2, state_pass_kernel, (const float *)U, (const float *)lam, hin, nc, a.h0, a.h_out) !=
-        cudaSuccess)
+    const cudaError_t e2 =
+        nc <= 16 ? cudaLaunchKernelEx(&c2, state_pass_kernel<16>, (const float *)U, (const float *)lam, hin, nc, a.h0,
+                                      a.h_out)
+                 : cudaLaunchKernelEx(&c2, state_pass_kernel<8>, (const float *)U, (const float *)lam, hin, nc, a.h0,
+                                      a.h_out);
+    if (e2 != cudaSuccess)
         return SSD_ERR_CUDA;
     const int n_tiles = BH * nc * K::NRB;
     const int grid = n_tiles < sms ? n_tiles : sms;
