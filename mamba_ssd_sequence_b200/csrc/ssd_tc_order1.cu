@@ -428,7 +428,13 @@ struct ScanCfg {
     static constexpr uint32_t H_OFF = K_OFF + NKB * kBox;
     static constexpr uint32_t V_OFF = H_OFF + kHinBytes;
     static constexpr uint32_t STAGE = V_OFF + NKB * kBox;
-    static constexpr uint32_t MISC_OFF = STAGES * STAGE;
+    // C = 256 (two stages) stages each group's output tile in a slot of its
+    // own, so that a stage is free as soon as its P V product completes;
+    // C = 128 (three stages) stages it over the stage's Q box, which keeps
+    // the residual rows at hand in the stage's V box.
+    static constexpr bool OUT_SLOT = C == 256;
+    static constexpr uint32_t Y_OFF = STAGES * STAGE;
+    static constexpr uint32_t MISC_OFF = Y_OFF + (OUT_SLOT ? NG * kBox : 0);
     static constexpr uint32_t MISC_BYTES = 28 * NG * C + 1024;
     static constexpr uint32_t SMEM = MISC_OFF + MISC_BYTES + 1024;
     // TMEM: C = 128: S' buffers at 0 and 192 (keys at +0, Z at +128);
@@ -482,7 +488,7 @@ template <int C>
 __global__ void __launch_bounds__(ScanCfg<C>::THREADS, 1)
 chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
-                  const __grid_constant__ CUtensorMap tm_out,
+                  const __grid_constant__ CUtensorMap tm_out, const __nv_bfloat16 *__restrict__ vglob,
                   const float *__restrict__ acs_in, const float *__restrict__ vfac_in,
                   const float *__restrict__ Dres, int H, int N, int n_tiles, DeviceStatus *status) {
     using K = ScanCfg<C>;
@@ -501,9 +507,9 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (tid == 0) {
         for (int i = 0; i < K::STAGES; ++i) {
             mbar_init(&misc->stage_full[i], 1);
-            // released by the P V product (tcgen05.commit) and by the compute
-            // group once its output tile, staged over Q, has been stored
-            mbar_init(&misc->stage_empty[i], 2);
+            // released by the P V product (tcgen05.commit) and, with the output
+            // staged over Q, by the compute group once that tile has been stored
+            mbar_init(&misc->stage_empty[i], K::OUT_SLOT ? 1 : 2);
         }
         for (int i = 0; i < K::NSB; ++i) mbar_init(&misc->s_full[i], 1);
         for (int gi = 0; gi < NG; ++gi)
@@ -760,10 +766,22 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_arrive(&misc->p_full[gi][kb]);
             }
             // ---- epilogue: y = Y + 2^acs_i Z [+ D v], columns [32 hf, 32 hf + 32)
+            // With an output slot the stage may be refilled once P V completes,
+            // so the residual rows v_i (still in L2) are fetched from global
+            // memory while P V runs; otherwise they are read from the V box.
+            uint4 vres[4] = {};
+            if (K::OUT_SLOT && Dres) {
+                const uint4 *vp = reinterpret_cast<const uint4 *>(
+                                      vglob + ((size_t)x.bh * N + (size_t)x.c * C + 128 * x.rb + r) * kD) +
+                                  4 * hf;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vres[q] = __ldg(vp + q);
+            }
             bad = !mbar_wait_abortable(&misc->y_full[tb], (i >> 1) & 1, abort_flag);
             // the V box is read below: observe the stage's TMA completion here too
             // (long complete; the stage cannot be refilled before this group releases it)
-            bad = bad || !mbar_wait_abortable(&misc->stage_full[i % K::STAGES], (i / K::STAGES) & 1, abort_flag);
+            if (!K::OUT_SLOT)
+                bad = bad || !mbar_wait_abortable(&misc->stage_full[i % K::STAGES], (i / K::STAGES) & 1, abort_flag);
             if (named_bar_any(bar, 256, bad)) {
                 failed = true;
                 break;
@@ -771,10 +789,12 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_after();
             const float e = ex2_approx(ai);
             const float *dh = &misc->dres[gi][slot][hf * 32];
-            // residual v_i: row r of V box rb (this tile's own tokens); y is
-            // staged over Q (dead since S' completed) in the same swizzled layout
+            // residual v_i: row r of V box rb (this tile's own tokens).  y is
+            // staged in the swizzled layout of the TMA store, over Q (dead since
+            // S' completed) or in the group's slot, whose previous store was
+            // read before this group signalled P of this tile complete.
             const uint8_t *vrow = sp + K::V_OFF + x.rb * kBox;
-            uint8_t *ytile = sp + K::Q_OFF;
+            uint8_t *ytile = K::OUT_SLOT ? smem + K::Y_OFF + gi * kBox : sp + K::Q_OFF;
             const uint32_t zc = tmem + lane_off + z_col<C>(sb) + 32 * hf;
             const uint32_t yc = tmem + lane_off + K::COL_Y + 64 * tb + 32 * hf;
 #pragma unroll
@@ -791,8 +811,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int q2 = 0; q2 < 2; ++q2) {
                     const int q = 2 * half + q2;
                     uint32_t wv[4];
-                    uint4 vq = make_uint4(0u, 0u, 0u, 0u);
-                    if (Dres) vq = *reinterpret_cast<const uint4 *>(vrow + sw128_chunk(r, 4 * hf + q));
+                    uint4 vq = vres[q];
+                    if (!K::OUT_SLOT && Dres) vq = *reinterpret_cast<const uint4 *>(vrow + sw128_chunk(r, 4 * hf + q));
                     const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w};
 #pragma unroll
                     for (int pp = 0; pp < 4; ++pp) {
@@ -810,14 +830,15 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         make_uint4(wv[0], wv[1], wv[2], wv[3]);
                 }
             }
-            // one TMA store per tile; the stage is released once it has been read
+            // one TMA store per tile, read out before this thread goes on (and,
+            // staged over Q, before the stage is released)
             fence_proxy_async_smem();
             named_bar_sync(bar, 256);
             if (ct == 0) {
                 tma_store_2d(&tm_out, ytile, 0, x.bh * N + x.c * C + 128 * x.rb);
                 bulk_commit_group();
                 bulk_wait_group_read0();
-                mbar_arrive(&misc->stage_empty[i % K::STAGES]);
+                if (!K::OUT_SLOT) mbar_arrive(&misc->stage_empty[i % K::STAGES]);
             }
         }
         if (ct == 0) bulk_wait_group0();  // every output tile has reached global memory
@@ -952,8 +973,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c3.stream = a.stream;
     c3.attrs = pdl;
     c3.numAttrs = 1;
-    if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, to, (const float *)acs, (const float *)vfac,
-                           a.D, a.H, a.N, n_tiles, status) != cudaSuccess)
+    if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, to, (const __nv_bfloat16 *)a.v,
+                           (const float *)acs, (const float *)vfac, a.D, a.H, a.N, n_tiles, status) != cudaSuccess)
         return SSD_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }

@@ -20,6 +20,8 @@ if not torch.cuda.is_available():
 # (dtype, d_h, order, normalize, chunk, chunks)
 SHAPES = [
     ("bf16", 64, 1, False, 128, 5),   # order-1 tensor-core path
+    ("bf16", 64, 1, False, 128, 7),   # longer heads (more chunk states to carry)
+    ("bf16", 64, 1, False, 128, 15),
     ("bf16", 64, 1, False, 256, 3),   # order-1 tensor-core path, two 128-row tiles per chunk
     ("f32", 16, 1, False, 64, 5),     # SIMT path
     ("f32", 16, 1, True, 64, 4),      # SIMT path with the normaliser
@@ -39,7 +41,7 @@ def _run(x, ld, dtype, order, normalize, chunk, use_ld, vdt):
     return out.float().cpu().numpy().astype(np.float64)
 
 
-@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}-d{s[1]}-o{s[2]}-n{int(s[3])}-c{s[4]}")
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: f"{s[0]}-d{s[1]}-o{s[2]}-n{int(s[3])}-c{s[4]}x{s[5]}")
 @pytest.mark.parametrize("opt", OPTIONS, ids=lambda o: o[0])
 @pytest.mark.parametrize("residual", [True, False])
 def test_options_match_oracle(shape, opt, residual):

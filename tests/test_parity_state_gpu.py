@@ -30,20 +30,23 @@ def _state(B, H, d, order, seed, scale=0.5):
     return h0, z0
 
 
-# (dtype, d_h, order, normalize, chunk, use z)
+# (dtype, d_h, order, normalize, chunk, use z, chunks per head)
 PREFILL = [
-    ("bf16", 64, 1, False, 128, False),  # order-1 tensor-core path (h only)
-    ("bf16", 64, 1, False, 256, False),
-    ("f32", 16, 1, False, 64, True),     # SIMT path with the normaliser state
-    ("bf16", 32, 2, True, 64, True),     # order 2 with state: SIMT path
+    ("bf16", 64, 1, False, 128, False, 3),   # order-1 tensor-core path (h only)
+    ("bf16", 64, 1, False, 128, False, 7),   # longer heads: the state pass carries h0 over more chunks
+    ("bf16", 64, 1, False, 128, False, 15),
+    ("bf16", 64, 1, False, 256, False, 3),
+    ("f32", 16, 1, False, 64, True, 3),      # SIMT path with the normaliser state
+    ("bf16", 32, 2, True, 64, True, 3),      # order 2 with state: SIMT path
 ]
 
 
-@pytest.mark.parametrize("case", PREFILL, ids=lambda c: f"{c[0]}-d{c[1]}-o{c[2]}-c{c[4]}-z{int(c[5])}")
+@pytest.mark.parametrize("case", PREFILL,
+                         ids=lambda c: f"{c[0]}-d{c[1]}-o{c[2]}-c{c[4]}-z{int(c[5])}-n{c[6]}")
 @pytest.mark.parametrize("in_place", [False, True])
 def test_prefill_state_in_and_out(case, in_place):
-    dtype, d, order, norm, chunk, use_z = case
-    B, H, N = 1, 3, 3 * chunk
+    dtype, d, order, norm, chunk, use_z, n_chunks = case
+    B, H, N = 1, 3, n_chunks * chunk
     x = inputs.make_inputs(B, H, N, d, dtype, seed=41, residual=True)
     h0, z0 = _state(B, H, d, order, 41)
     dev = to_device(x, dtype)
