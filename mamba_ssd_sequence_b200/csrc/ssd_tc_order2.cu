@@ -89,6 +89,7 @@ struct Cfg {
 
 struct Misc {
     float acs2[kC];
+    float vfac[kC];  // value factor dt_j of the chunk's tokens (value discretisation)
     float rsum[2][kC];
     float Dh[64];
     float wtot[2];
@@ -132,7 +133,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  __nv_bfloat16 *__restrict__ out,
                  const float *__restrict__ dt_p, const float *__restrict__ A_log,
                  const float *__restrict__ dt_bias, const float *__restrict__ Dres,
-                 const float *__restrict__ log_decay, int H, int N,
+                 const float *__restrict__ log_decay, int value_dt, int H, int N,
                  int normalize, DeviceStatus *status) {
     using K = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -301,7 +302,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool mrow_ok = lane < 16;
         const bool own_row = mrow_ok && mrow / K::ROWS == (int)rank;
         const float A2 = log_decay ? 0.0f : -expf(A_log[h]) * kLog2e;
-        const float bias = log_decay ? 0.0f : dt_bias[h];
+        const float bias = dt_bias ? dt_bias[h] : 0.0f;  // given whenever dt is used
         const bool elected = ct == 0;
         const int tok = ct & 63, q4 = ct >> 6;      // feature generation: token, 32-feature part
         uint32_t slab_uses[2] = {0, 0};
@@ -311,6 +312,9 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // per-token decay input: the dt projection, or the given log-decay (Algorithm 4)
         const float *dsrc = log_decay ? log_decay : dt_p;
         float dt_next = (ct < kC && nc > 0) ? dsrc[(size_t)row0 + ct] : 0.0f;
+        // the dt projection for the value factor, when it is not already dsrc
+        const bool vdt_own = value_dt && log_decay;
+        float vdt_next = (vdt_own && ct < kC && nc > 0) ? dt_p[(size_t)row0 + ct] : 0.0f;
         bool failed = false;
         // Own rows of chunk cc: sum the R partials (distributed shared memory),
         // release them, then y = (Y + T) / (r + Tn) [+ D v].
@@ -395,6 +399,8 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             uint8_t *sV = sK + K::TILE;
             const float dtv = dt_next;
             if (ct < kC && c + 1 < nc) dt_next = dsrc[(size_t)row0 + (size_t)(c + 1) * kC + ct];
+            const float vdt = vdt_own ? vdt_next : dtv;
+            if (vdt_own && ct < kC && c + 1 < nc) vdt_next = dt_p[(size_t)row0 + (size_t)(c + 1) * kC + ct];
 
             bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
             // ---- decay (tokens 0..63 on threads 0..63)
@@ -407,10 +413,31 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     if (lane >= o) a += y;
                 }
                 if (lane == 31) misc->wtot[ct >> 5] = a;
+                if (value_dt) misc->vfac[ct] = softplus_f(vdt + bias);
             }
-            if (named_bar_any(1, kTeam, bad)) {
+            if (named_bar_any(1, kTeam, bad)) {  // also publishes wtot[] and vfac[]
                 if (elected) raise_timeout(misc, status, 30);
                 break;
+            }
+            if (value_dt) {
+                // value discretisation: V <- diag(dt) V in place, before P V and the
+                // state products read it (both wait for p_full below); the
+                // normaliser and the D residual use the raw scores and v
+                constexpr int CPR = D / 8;  // 16-byte chunks per row
+                for (int t = ct; t < kC * CPR; t += kTeam) {
+                    const int r = t / CPR, ch = t % CPR;
+                    uint4 *pv = reinterpret_cast<uint4 *>(sV + swz<K::RB>(r, ch));
+                    const float f = misc->vfac[r];
+                    const float2 f2 = make_float2(f, f);
+                    const uint4 x = *pv;
+                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 y = __fmul2_rn(bf2_to_f2(w[e]), f2);
+                        w[e] = pack_bf16x2(y.x, y.y);
+                    }
+                    *pv = make_uint4(w[0], w[1], w[2], w[3]);
+                }
             }
             if (ct >= 32 && ct < kC) a += misc->wtot[0];
             if (ct < kC) misc->acs2[ct] = a;
@@ -675,7 +702,7 @@ int launch_d(const FwdArgs &a) {
     cudaError_t e = cudaLaunchKernelEx(&cfg, tc_order2_kernel<D>, tq, tk, tv,
                                        static_cast<const __nv_bfloat16 *>(a.v),
                                        static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log,
-                                       a.dt_bias, a.D, a.log_decay, a.H, a.N, a.normalize, status);
+                                       a.dt_bias, a.D, a.log_decay, a.value_dt, a.H, a.N, a.normalize, status);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -25,8 +25,9 @@ SHAPES = [
     ("bf16", 64, 1, False, 256, 3),   # order-1 tensor-core path, two 128-row tiles per chunk
     ("f32", 16, 1, False, 64, 5),     # SIMT path
     ("f32", 16, 1, True, 64, 4),      # SIMT path with the normaliser
-    ("bf16", 32, 2, True, 64, 5),     # order-2 tensor-core path (SIMT with value dt)
-    ("bf16", 64, 2, True, 64, 3),     # order-2 cluster of 8 CTAs (SIMT with value dt)
+    ("bf16", 32, 2, True, 64, 5),     # order-2 tensor-core path (value dt scales V in place)
+    ("bf16", 32, 2, False, 64, 4),    # order 2 without the normaliser
+    ("bf16", 64, 2, True, 64, 3),     # order-2 cluster of 8 CTAs
 ]
 OPTIONS = [("log_decay", True, False), ("value_dt", False, True), ("both", True, True)]
 
