@@ -237,9 +237,10 @@ int ssd_fwd_noalloc(const void *q, const void *k, const void *v,
  *   z_out  device, [B, H, D_phi] fp32, the normaliser state after token N-1.
  *          May equal z0.
  * With value discretisation the state accumulates phi(k) (dt v)^T; the
- * normaliser state never sees dt.  Paths: order 1 with h0/h_out only runs on
- * the tensor-core path; z0/z_out for order 1, and any state for order 2, run
- * on the SIMT path.  Errors as ssd_fwd_ex().
+ * normaliser state never sees dt.  Paths: order 1 with h0/h_out only, and
+ * order 2 with any state, run on the tensor-core paths where the shape
+ * allows; z0/z_out for order 1 run on the SIMT path.  Errors as
+ * ssd_fwd_ex().
  */
 int ssd_fwd_state(const void *q, const void *k, const void *v,
                   const float *dt_p, const float *A_log, const float *dt_bias,

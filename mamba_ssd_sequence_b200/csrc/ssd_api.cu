@@ -40,7 +40,7 @@ bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, 
         p.path = PATH_TC_ORDER1;
         p.n_launches = 3;
         tc_order1_layout(B, H, N, chunk, &p);
-    } else if (order == 2 && !state && tc_order2_supports(B, H, N, d, dtype, chunk)) {
+    } else if (order == 2 && tc_order2_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER2;
         p.n_launches = 1;
         p.acs_off = p.lam_off = p.state_off = kStatusBytes;

@@ -25,6 +25,9 @@
 // writes y_i = (Y_i + sum T_i) / (r_i + sum Tn_i) [+ D v_i].  The
 // (q . k)^2 of the intra-chunk part is the same inner product as
 // (q (x) q) . (k (x) k) of the feature form (Algorithm 5 vs Algorithm 6).
+// Options: a per-token log-decay and value discretisation (Algorithm 4; V is
+// scaled by dt in shared memory); a carried state h0, z0 enters as the state
+// before chunk 0, and h_out, z_out receive the state after the last chunk.
 // All exponentials are of non-positive arguments.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -126,7 +129,9 @@ __device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
     *reinterpret_cast<volatile int *>(&misc->abort_flag) = 1;
 }
 
-template <int D>
+// kState: the call carries a state in or out (a separate instantiation, so
+// that calls without one run none of its code).
+template <int D, bool kState>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ vglob,
@@ -134,7 +139,8 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  const float *__restrict__ dt_p, const float *__restrict__ A_log,
                  const float *__restrict__ dt_bias, const float *__restrict__ Dres,
                  const float *__restrict__ log_decay, int value_dt, int H, int N,
-                 int normalize, DeviceStatus *status) {
+                 int normalize, const float *__restrict__ h0, const float *__restrict__ z0,
+                 float *__restrict__ h_out, float *__restrict__ z_out, DeviceStatus *status) {
     using K = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -148,6 +154,10 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int bh = blockIdx.x / K::R, h = bh % H;
     const int nc = N / kC;
     const int row0 = bh * N;
+    // a carried state enters before chunk 0 exactly as the state of a previous
+    // chunk does; the normaliser state is tracked when it is used or asked for
+    const bool carry = kState && (h0 != nullptr || z0 != nullptr);
+    const bool track_z = normalize || (kState && (z0 != nullptr || z_out != nullptr));
 
     if (tid == 0) {
         if (blockIdx.x == 0 && status) {
@@ -258,15 +268,16 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int ks = 0; ks < kC / 16; ++ks)
                         mma_bf16(tmem + K::COL_H + sl * D, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
-                                 make_sdesc(aV + ks * 16 * K::RB, 16, K::SBO, K::SW), idU, (c > 0 || ks > 0));
-                    if (normalize) {
+                                 make_sdesc(aV + ks * 16 * K::RB, 16, K::SBO, K::SW), idU,
+                                 (c > 0 || carry || ks > 0));
+                    if (track_z) {
 #pragma unroll
                         for (int ks = 0; ks < kC / 16; ++ks)
                             mma_bf16(tmem + K::COL_Z + sl * 16, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
                                      make_sdesc(sbase + K::OFF_ONES + ks * 512, 16, 256, kSw32), idZ,
-                                     (c > 0 || ks > 0));
+                                     (c > 0 || carry || ks > 0));
                     }
-                    if (c >= 1) {
+                    if (c >= 1 || carry) {
                         // [T | Tn] += Fq [hb | zb]   (A: tokens x features, K-major;
                         // B: the hb and zb tiles as two MN atoms)
                         const uint32_t hbB = sbase + K::OFF_HB + b * kSlab * K::RB;
@@ -495,15 +506,31 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tc_fence_after();
                 }
                 // h_{c-1} of this slab -> bf16, then h *= 2^lam (columns [hf D/2, hf D/2 + D/2));
-                // z likewise (column 0, half 0 only)
-                if (c >= 1) {
+                // z likewise (column 0, half 0 only).  Before chunk 0 the state
+                // is the carried one, read from global memory (zero if absent).
+                if (c >= 1 || carry) {
                     constexpr int HC = D / 2;
                     float hv[HC];
+                    float zv = 0.0f;
                     const uint32_t ta = tmem + lane_off + K::COL_H + sl * D + hf * HC;
-                    if constexpr (HC == 32) tmem_ld32(ta, hv);
-                    else tmem_ld16(ta, hv);
-                    const float zv = (normalize && hf == 0) ? tmem_ld1(tmem + lane_off + K::COL_Z + sl * 16) : 0.0f;
-                    tmem_wait_ld();
+                    const size_t m = (size_t)bh * D * D + rank * kFs + sl * kSlab + frow;  // feature row
+                    if (c >= 1) {
+                        if constexpr (HC == 32) tmem_ld32(ta, hv);
+                        else tmem_ld16(ta, hv);
+                        if (track_z && hf == 0) zv = tmem_ld1(tmem + lane_off + K::COL_Z + sl * 16);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < HC; j += 4) {
+                            const float4 x = h0 ? *reinterpret_cast<const float4 *>(h0 + m * D + hf * HC + j)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                            hv[j] = x.x;
+                            hv[j + 1] = x.y;
+                            hv[j + 2] = x.z;
+                            hv[j + 3] = x.w;
+                        }
+                        if (track_z && hf == 0 && z0) zv = z0[m];
+                    }
                     uint8_t *hb = smem + K::OFF_HB + b * kSlab * K::RB;
 #pragma unroll
                     for (int ch = 0; ch < HC / 8; ++ch)
@@ -521,7 +548,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     if constexpr (HC == 32) tmem_st32(ta, hv);
                     else tmem_st16(ta, hv);
-                    if (normalize && hf == 0) {
+                    if (track_z && hf == 0) {
                         // column 0 of the zb row; the rest of the tile stays zero
                         uint8_t *zb = smem + K::OFF_ZB + b * kSlab * K::RB;
                         *reinterpret_cast<uint4 *>(zb + swz<K::RB>(frow, 0)) =
@@ -603,7 +630,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     float *prow = part0 + (c & 1) * kC * K::PR + mrow * K::PR;
 #pragma unroll
                     for (int e = 0; e < HC; e += 4) {
-                        float4 v = c >= 1 ? make_float4(tv[e], tv[e + 1], tv[e + 2], tv[e + 3])
+                        float4 v = (c >= 1 || carry) ? make_float4(tv[e], tv[e + 1], tv[e + 2], tv[e + 3])
                                           : make_float4(0.f, 0.f, 0.f, 0.f);
                         if (own_row) {
                             v.x += yv[e];
@@ -614,7 +641,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                         *reinterpret_cast<float4 *>(prow + hf * HC + e) = v;
                     }
                     if (hf == 0)
-                        prow[D] = (c >= 1 ? tn : 0.0f) +
+                        prow[D] = ((c >= 1 || carry) ? tn : 0.0f) +
                                   (own_row ? misc->rsum[0][mrow] + misc->rsum[1][mrow] : 0.0f);
                 }
             }
@@ -630,6 +657,31 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (elected) mbar_arrive(&misc->stage_empty[st]);
         }
         if (!failed && nc >= 1) reduce_output(nc - 1);
+        // the state after the last token: TMEM holds it once the last chunk's
+        // products are done (waited for above)
+        if (kState && !failed && (h_out || z_out)) {
+            tc_fence_after();
+            constexpr int HC = D / 2;
+            for (int sl = 0; sl < kNs; ++sl) {
+                const size_t m = (size_t)bh * D * D + rank * kFs + sl * kSlab + frow;
+                if (h_out) {
+                    float hv[HC];
+                    const uint32_t ta = tmem + lane_off + K::COL_H + sl * D + hf * HC;
+                    if constexpr (HC == 32) tmem_ld32(ta, hv);
+                    else tmem_ld16(ta, hv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < HC; j += 4)
+                        *reinterpret_cast<float4 *>(h_out + m * D + hf * HC + j) =
+                            make_float4(hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
+                }
+                if (z_out) {
+                    const float zv = tmem_ld1(tmem + lane_off + K::COL_Z + sl * 16);
+                    tmem_wait_ld();
+                    if (hf == 0) z_out[m] = zv;
+                }
+            }
+        }
     done:;
     }
 
@@ -676,13 +728,14 @@ int launch_d(const FwdArgs &a) {
     CUtensorMap tq, tk, tv;
     if (!make_tmap(&tq, a.q, rows, D) || !make_tmap(&tk, a.k, rows, D) || !make_tmap(&tv, a.v, rows, D))
         return SSD_ERR_CUDA;
-    static std::atomic<uint64_t> attr_set{0};  // one bit per device
+    const bool state = a.h0 || a.z0 || a.h_out || a.z_out;
+    auto kern = state ? tc_order2_kernel<D, true> : tc_order2_kernel<D, false>;
+    static std::atomic<uint64_t> attr_set{0};  // one bit per device and instantiation
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SSD_ERR_CUDA;
-    const uint64_t bit = 1ull << (dev & 63);
+    const uint64_t bit = 1ull << (2 * (dev & 31) + (state ? 1 : 0));
     if (!(attr_set.load() & bit)) {
-        if (cudaFuncSetAttribute(tc_order2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)K::SMEM) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM) != cudaSuccess)
             return SSD_ERR_CUDA;
         attr_set.fetch_or(bit);
     }
@@ -699,10 +752,11 @@ int launch_d(const FwdArgs &a) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, tc_order2_kernel<D>, tq, tk, tv,
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv,
                                        static_cast<const __nv_bfloat16 *>(a.v),
                                        static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log,
-                                       a.dt_bias, a.D, a.log_decay, a.value_dt, a.H, a.N, a.normalize, status);
+                                       a.dt_bias, a.D, a.log_decay, a.value_dt, a.H, a.N, a.normalize,
+                                       a.h0, a.z0, a.h_out, a.z_out, status);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

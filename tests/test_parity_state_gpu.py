@@ -23,6 +23,15 @@ def _np(t):
 
 
 def _state(B, H, d, order, seed, scale=0.5):
+    """A carried state to start from.  Order 1: random entries (z0 > 0).
+    Order 2: the state a 64-token prefix leaves (the oracle's recurrence over
+    seeded inputs), since the normaliser phi(q) . z0 of an arbitrary z0 can
+    come out near zero or negative, which no real prefix gives."""
+    if order == 2:
+        p = inputs.make_inputs(B, H, 64, d, "f32", seed=seed)
+        _, _, h0, z0 = oracle.ssd_recurrent(p["q"], p["k"], p["v"], p["dt_p"], p["A_log"], p["dt_bias"],
+                                           None, 2, False, return_norm=True, return_state=True)
+        return h0.astype(np.float32), z0.astype(np.float32)
     rng = np.random.default_rng(seed)
     Dphi = d ** order
     h0 = (scale * rng.standard_normal((B, H, Dphi, d))).astype(np.float32)
@@ -37,7 +46,9 @@ PREFILL = [
     ("bf16", 64, 1, False, 128, False, 15),
     ("bf16", 64, 1, False, 256, False, 3),
     ("f32", 16, 1, False, 64, True, 3),      # SIMT path with the normaliser state
-    ("bf16", 32, 2, True, 64, True, 3),      # order 2 with state: SIMT path
+    ("bf16", 32, 2, True, 64, True, 3),      # order-2 tensor-core path with h and z
+    ("bf16", 32, 2, False, 64, True, 4),     # order 2 without the normaliser, z still carried
+    ("bf16", 64, 2, True, 64, True, 2),      # order 2, cluster of 8 CTAs per head
 ]
 
 
@@ -74,7 +85,7 @@ DECODE = [("f32", 16, 1, False), ("f32", 32, 1, True), ("bf16", 64, 1, False), (
 @pytest.mark.parametrize("case", DECODE, ids=lambda c: f"{c[0]}-d{c[1]}-o{c[2]}-n{int(c[3])}")
 @pytest.mark.parametrize("opt", ["plain", "log_decay", "value_dt"])
 def test_decode_steps_continue_the_recurrence(case, opt):
-    """Four decode steps from a random carried state agree with the oracle's
+    """Four decode steps from a carried state agree with the oracle's
     recurrence over the same tokens, output by output, and in the final state."""
     dtype, d, order, norm = case
     B, H, T = 2, 3, 4
