@@ -320,6 +320,30 @@ def main():
     total_ms = max_over_ranks(sum(step_ms), dev_name)
     status = ssd.ssd_status_from_workspace(ws)
 
+    # kernel (a) on its own: the chunk-local cumsum of A dt and the chunk
+    # totals, which the tensor-core paths fuse into their first kernel.  It
+    # reads dt_p and writes acs and the chunk totals: HBM-bound.
+    acs_a = torch.empty_like(dev["dt_p"])
+    csum_a = torch.empty((w.B, w.H, w.N // w.chunk), dtype=torch.float32, device=dev_name)
+
+    def step_a():
+        ssd.ssd_chunk_cumsum(dev["dt_p"], dev["A_log"], dev["dt_bias"], w.chunk, acs=acs_a,
+                             chunk_sum=csum_a, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush_l2(1.0)
+        step_a()
+    a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2(float(i))
+        a_ev[i][0].record(stream)
+        step_a()
+        a_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    a_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in a_ev), dev_name) / args.steps
+    a_bytes = 4 * (dev["dt_p"].numel() + acs_a.numel() + csum_a.numel())
+
     # end to end: pinned host inputs -> device -> ssd_fwd -> host, per step
     e2e = None
     if not args.no_e2e:
@@ -392,6 +416,10 @@ def main():
                      "algorithmic_bytes_per_launch": alg_bytes,
                      "algorithmic_flops_per_launch": alg_flops},
         "gpu_launches": n_launch * args.steps,
+        "kernel_a": {"what": "chunk cumsum of A dt and chunk totals, launched alone (L2 flushed before each)",
+                     "ms_per_launch": a_ms, "bytes_per_launch": a_bytes,
+                     "achieved_gbs": a_bytes / (a_ms / 1e3) / 1e9,
+                     "frac_of_hbm": a_bytes / (a_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
         "device_status": status,
         "clocks": clk.summary(),
     }

@@ -177,7 +177,8 @@ int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
  * A^CS_i - A^CS_j for i, j in one chunk equals acs[i] - acs[j]; across chunks
  * the global value is recovered by adding the chunk_sum of the chunks in
  * between.  dt_p, A_log, dt_bias, acs ([B,H,N]) and chunk_sum ([B,H,N/chunk])
- * are device pointers.  chunk in {64, 128, 256}; N % chunk == 0.
+ * are device pointers; dt_p and acs 16-byte aligned (SSD_ERR_ALIGN
+ * otherwise).  chunk in {64, 128, 256}; N % chunk == 0.
  */
 int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias,
                      int B, int H, int N, int chunk,

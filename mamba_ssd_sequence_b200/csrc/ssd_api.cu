@@ -217,6 +217,7 @@ int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias
     if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_CHUNK;
     if (B < 1 || H < 1 || N < 1 || N % chunk != 0 || (long long)B * H > 65535)
         return SSD_ERR_SHAPE;
+    if (!aligned16(dt_p) || !aligned16(acs)) return SSD_ERR_ALIGN;  // 16-byte vector accesses
     return launch_chunk_cumsum(dt_p, A_log, dt_bias, nullptr, B, H, N, chunk, acs, chunk_sum, nullptr,
                                static_cast<cudaStream_t>(stream));
 }

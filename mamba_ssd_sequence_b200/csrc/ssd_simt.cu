@@ -45,36 +45,89 @@ __device__ __forceinline__ float softplus_f(float x) {
 }
 
 // ---------------------------------------------------------------- kernel (a)
-// grid (n_chunks, B*H), block = chunk threads (64, 128 or 256).
-__global__ void chunk_cumsum_kernel(const float *__restrict__ dt_p,
-                                    const float *__restrict__ A_log,
-                                    const float *__restrict__ dt_bias,
-                                    const float *__restrict__ log_decay, int H, int N,
-                                    int chunk, float *__restrict__ acs,
-                                    float *__restrict__ chunk_sum,
-                                    DeviceStatus *status) {
-    __shared__ float warp_tot[8];
-    const int c = blockIdx.x, bh = blockIdx.y, h = bh % H;
+// Chunk-local inclusive cumsum of the per-token log-decay, and chunk totals.
+// 256 threads per CTA, kCumU blocks of 1024 tokens per CTA: in block u,
+// thread t takes the four consecutive tokens 4t..4t+3 (16-byte loads and
+// stores); every block's loads are issued before any is used.  One block per
+// CTA measured fastest: more keep more loads in flight per thread but leave
+// small problems with too few CTAs, and large ones are bound by the
+// per-token softplus (expf and log1pf) rather than by HBM.  A chunk of C
+// tokens is C/4 threads: a
+// segment of 16 or 32 lanes for C = 64 or 128, two warps for C = 256.
+// Chunks are contiguous in the flattened [B H N] order and never straddle a
+// head, since N % C == 0.  Index arithmetic is in I: 32-bit when B H N <
+// 2^31 (integer division by N being the costly step), else 64-bit.
+constexpr int kCumU = 1;
+
+template <typename I>
+__global__ void __launch_bounds__(256)
+chunk_cumsum_kernel(const float *__restrict__ dt_p, const float *__restrict__ A_log,
+                    const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int H,
+                    int N, int chunk_shift, I total, float *__restrict__ acs,
+                    float *__restrict__ chunk_sum, DeviceStatus *status) {
+    __shared__ float warp_tot[kCumU][8];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    if (status && c == 0 && bh == 0 && t == 0) {
+    if (status && blockIdx.x == 0 && t == 0) {
         status->code = 0;
         status->detail = 0;
     }
-    const size_t idx = (size_t)bh * N + (size_t)c * chunk + t;
-    float x = log_decay ? log_decay[idx] : -expf(A_log[h]) * softplus_f(dt_p[idx] + dt_bias[h]);
-    // inclusive warp scan, then add the totals of the warps before
+    const int chunk = 1 << chunk_shift;
+    I tok0[kCumU];
+    float4 x[kCumU];
+    int h[kCumU];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+    for (int u = 0; u < kCumU; ++u) {
+        tok0[u] = (((I)blockIdx.x * kCumU + (I)u) * 256 + (I)t) * 4;
+        h[u] = 0;
+        x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (tok0[u] < total) {  // total is a multiple of 64: whole chunks only
+            x[u] = __ldg(reinterpret_cast<const float4 *>((log_decay ? log_decay : dt_p) + tok0[u]));
+            h[u] = (int)((tok0[u] / (I)N) % (I)H);
+        }
     }
-    if (lane == 31) warp_tot[warp] = x;
-    __syncthreads();
-    float before = 0.0f;
-    for (int w = 0; w < warp; ++w) before += warp_tot[w];
-    x += before;
-    acs[idx] = x;
-    if (t == chunk - 1) chunk_sum[(size_t)bh * (N / chunk) + c] = x;
+    const int seg = chunk / 4;  // threads per chunk
+    const int width = seg < 32 ? seg : 32;
+    float a[kCumU][4], before[kCumU];
+#pragma unroll
+    for (int u = 0; u < kCumU; ++u) {
+        if (log_decay) {
+            a[u][0] = x[u].x, a[u][1] = x[u].y, a[u][2] = x[u].z, a[u][3] = x[u].w;
+        } else {
+            const bool live = tok0[u] < total;
+            const float A = live ? -expf(__ldg(A_log + h[u])) : 0.0f;
+            const float bias = live ? __ldg(dt_bias + h[u]) : 0.0f;
+            a[u][0] = A * softplus_f(x[u].x + bias);
+            a[u][1] = A * softplus_f(x[u].y + bias);
+            a[u][2] = A * softplus_f(x[u].z + bias);
+            a[u][3] = A * softplus_f(x[u].w + bias);
+        }
+        a[u][1] += a[u][0];
+        a[u][2] += a[u][1];
+        a[u][3] += a[u][2];
+        // inclusive scan of the thread totals within each chunk's lanes
+        float run = a[u][3];
+        for (int o = 1; o < width; o <<= 1) {
+            const float y = __shfl_up_sync(0xffffffffu, run, o, width);
+            if ((lane & (width - 1)) >= o) run += y;
+        }
+        before[u] = run - a[u][3];
+        if (lane == 31) warp_tot[u][warp] = run;
+    }
+    if (seg > 32) {  // C = 256: the second warp of a chunk adds the first's total
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kCumU; ++u)
+            if (warp & 1) before[u] += warp_tot[u][warp - 1];
+    }
+#pragma unroll
+    for (int u = 0; u < kCumU; ++u) {
+        if (tok0[u] < total) {
+            const float bf = before[u];
+            *reinterpret_cast<float4 *>(acs + tok0[u]) =
+                make_float4(a[u][0] + bf, a[u][1] + bf, a[u][2] + bf, a[u][3] + bf);
+            if ((((int)tok0[u] + 4) & (chunk - 1)) == 0) chunk_sum[tok0[u] >> chunk_shift] = a[u][3] + bf;
+        }
+    }
 }
 
 // ---------------------------------------------------------------- kernel (b)
@@ -336,9 +389,15 @@ int run_simt(const FwdArgs &a, const Plan &p) {
 int launch_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias,
                         const float *log_decay, int B, int H, int N, int chunk, float *acs,
                         float *chunk_sum, DeviceStatus *status, cudaStream_t stream) {
-    dim3 grid(N / chunk, B * H);
-    chunk_cumsum_kernel<<<grid, chunk, 0, stream>>>(dt_p, A_log, dt_bias, log_decay, H, N, chunk,
-                                                    acs, chunk_sum, status);
+    const size_t total = (size_t)B * H * N;
+    const int shift = chunk == 64 ? 6 : chunk == 128 ? 7 : 8;
+    const unsigned grid = (unsigned)((total + 1024 * kCumU - 1) / (1024 * kCumU));
+    if (total < (1ull << 31))
+        chunk_cumsum_kernel<uint32_t><<<grid, 256, 0, stream>>>(dt_p, A_log, dt_bias, log_decay, H, N, shift,
+                                                                (uint32_t)total, acs, chunk_sum, status);
+    else
+        chunk_cumsum_kernel<size_t><<<grid, 256, 0, stream>>>(dt_p, A_log, dt_bias, log_decay, H, N, shift,
+                                                              total, acs, chunk_sum, status);
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 

@@ -103,6 +103,9 @@ def test_cumsum_validation(lib):
     assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 100, 64, 64, 80, None) == 2
     assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 128, 48, 64, 80, None) == 5
     assert lib.ssd_chunk_cumsum(None, 32, 48, 1, 1, 128, 64, 64, 80, None) == 1
+    # 16-byte vector loads and stores: dt_p and acs must be aligned
+    assert lib.ssd_chunk_cumsum(20, 32, 48, 1, 1, 128, 64, 64, 80, None) == 6
+    assert lib.ssd_chunk_cumsum(16, 32, 48, 1, 1, 128, 64, 68, 80, None) == 6
 
 
 def _call_fwd_ex(lib, **over):
