@@ -174,15 +174,6 @@ __device__ __forceinline__ bool named_bar_any(int id, int nthreads, bool pred) {
     return r != 0;
 }
 
-// Per-warpgroup register budget (all 128 threads of the warpgroup execute it).
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
@@ -342,12 +333,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
-// 32 lanes x 8 consecutive 32-bit columns (store).
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
 // 32 lanes x 16 consecutive 32-bit columns (store).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
@@ -382,14 +367,10 @@ __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Byte offset of element (row, col) of a bf16 tile stored with rows of 128
-// bytes (64 elements) in the 128-byte swizzle pattern TMA produces with
-// CU_TENSOR_MAP_SWIZZLE_128B: the 16-byte chunk index is XORed with row % 8.
-// The tile base must be 1024-byte aligned.
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
-    return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
-}
-// Byte offset of the 16-byte chunk `ch` (elements 8ch..8ch+7) of `row`.
+// Byte offset of the 16-byte chunk `ch` (elements 8ch..8ch+7) of `row` of a
+// bf16 tile stored with rows of 128 bytes (64 elements) in the 128-byte
+// swizzle pattern TMA produces with CU_TENSOR_MAP_SWIZZLE_128B: the chunk
+// index is XORed with row % 8.  The tile base must be 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t ch) {
     return row * 128u + (((ch ^ (row & 7u)) & 7u) << 4);
 }
