@@ -182,18 +182,18 @@ def _oracle_sample(w, x, heads):
     return q, k, v, dt, x["A_log"][hidx], x["dt_bias"][hidx], D
 
 
-def _time_oracle(w, x, budget_s):
+def _time_oracle(w, x, target_s):
     """Times the oracle's quadratic form on a sample of (b, h) rows sized to
-    take about `budget_s` seconds; returns (tokens/s, threads, description)."""
+    take about `target_s` seconds; returns (tokens/s, threads, description)."""
     import oracle
     bh_all = w.B * w.H
     t0 = time.perf_counter()
     oracle.ssd_quadratic(*_oracle_sample(w, x, 1), w.order, w.normalize)
     t1 = max(time.perf_counter() - t0, 1e-6)
-    heads = max(1, min(bh_all, int(budget_s / t1)))
+    heads = max(1, min(bh_all, int(target_s / t1)))
     reps = 1
     if heads == bh_all:
-        reps = max(1, int(budget_s / (t1 * bh_all)))
+        reps = max(1, int(target_s / (t1 * bh_all)))
     args = _oracle_sample(w, x, heads)
     t0 = time.perf_counter()
     for _ in range(reps):
@@ -205,10 +205,10 @@ def _time_oracle(w, x, budget_s):
     return tokens / t, oracle.num_threads(), desc
 
 
-def cpu_baseline(w, x, budget_s=12.0):
+def cpu_baseline(w, x, target_s=12.0):
     """The CPU oracle as it stands, timed on the host cores on a bounded
     sample of the same workload (the JSON object of the bench line)."""
-    value, threads, desc = _time_oracle(w, x, budget_s)
+    value, threads, desc = _time_oracle(w, x, target_s)
     return {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
             "sample": desc}
 

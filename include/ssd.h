@@ -62,7 +62,7 @@ typedef enum {
     SSD_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than ssd_workspace_bytes() */
     SSD_ERR_CUDA = 8,        /* a CUDA runtime call or kernel launch failed */
     SSD_ERR_TIMEOUT = 9,     /* a device-side wait ran out (read back from the workspace) */
-    SSD_ERR_UNSUPPORTED = 10, /* a valid combination this build has no kernel for */
+    SSD_ERR_UNSUPPORTED = 10, /* a valid combination the library has no kernel for */
     SSD_ERR_FLAGS = 11       /* unknown bits in the flags of ssd_fwd_ex() */
 } ssd_status;
 
