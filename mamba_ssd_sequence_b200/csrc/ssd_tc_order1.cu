@@ -684,6 +684,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         };
 
         bool failed = false;
+        int pend_st = -1;  // thread ct = 0: stage of an output store not yet waited for
         pdl_wait();  // acs (chunk-state kernel) is visible
         Raw raw_next = fetch(gi);
         for (int i = gi; i < my_tiles; i += NG) {
@@ -701,6 +702,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 misc->acs[gi][slot][ct] = raw.acs;
                 misc->colf[gi][slot][ct] = ex2_approx(aref - raw.acs) * raw.vf;
                 misc->vf[gi][slot][ct] = raw.vf;
+            }
+            // ---- the group's previous output store: its read of shared memory is
+            // waited for here, where the group waits for S anyway, rather than
+            // right after the store, which held the whole group at its next barrier
+            if (ct == 0 && pend_st >= 0) {
+                bulk_wait_group_read0();
+                if (!K::OUT_SLOT) mbar_arrive(&misc->stage_empty[pend_st]);
+                pend_st = -1;
             }
             // ---- S of this tile
             bool bad = !mbar_wait_abortable(&misc->s_full[sb], (i / K::NSB) & 1, abort_flag);
@@ -830,15 +839,14 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         make_uint4(wv[0], wv[1], wv[2], wv[3]);
                 }
             }
-            // one TMA store per tile, read out before this thread goes on (and,
-            // staged over Q, before the stage is released)
+            // one TMA store per tile; its read of the tile (and, staged over Q,
+            // the stage's release) is settled before the group's next S
             fence_proxy_async_smem();
             named_bar_sync(bar, 256);
             if (ct == 0) {
                 tma_store_2d(&tm_out, ytile, 0, x.bh * N + x.c * C + 128 * x.rb);
                 bulk_commit_group();
-                bulk_wait_group_read0();
-                if (!K::OUT_SLOT) mbar_arrive(&misc->stage_empty[i % K::STAGES]);
+                pend_st = i % K::STAGES;
             }
         }
         if (ct == 0) bulk_wait_group0();  // every output tile has reached global memory
