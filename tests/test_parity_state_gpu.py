@@ -133,3 +133,43 @@ def test_prefill_then_decode_equals_one_pass():
     y = np.concatenate(ys, axis=2)
     ref = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"], 1, False)
     assert rel_err(y, ref) <= TOL["bf16"]
+
+
+# (dtype, d_h, order, normalize, chunk, chunks per head): every path that takes a state
+MAMBA2S_PREFILL = [
+    ("bf16", 64, 1, False, 128, 5),   # order-1 tensor-core path
+    ("bf16", 64, 1, False, 256, 2),
+    ("bf16", 32, 2, True, 64, 4),     # order-2 tensor-core path
+    ("bf16", 64, 2, True, 64, 2),
+    ("f32", 16, 1, False, 64, 3),     # SIMT path
+]
+
+
+@pytest.mark.parametrize("case", MAMBA2S_PREFILL, ids=lambda c: f"{c[0]}-d{c[1]}-o{c[2]}-c{c[4]}-n{c[5]}")
+def test_prefill_state_with_mamba2s_options(case):
+    """A given per-token log-decay and value discretisation (Algorithm 4)
+    together with a carried state in and out, against the oracle's
+    recurrence with the same options."""
+    dtype, d, order, norm, chunk, n_chunks = case
+    B, H, N = 1, 3, n_chunks * chunk
+    x = inputs.make_inputs(B, H, N, d, dtype, seed=44, residual=True)
+    ld = inputs.make_log_decay(B, H, N, seed=44)
+    h0, z0 = _state(B, H, d, order, 44)
+    use_z = norm
+    dev = to_device(x, dtype)
+    h0d = torch.from_numpy(h0).cuda()
+    z0d = torch.from_numpy(z0).cuda() if use_z else None
+    ho = torch.empty_like(h0d)
+    zo = torch.empty_like(z0d) if use_z else None
+    y = ssd.ssd_fwd_state(dev["q"], dev["k"], dev["v"], dev["dt_p"], None, dev["dt_bias"], dev["D"],
+                          order, norm, chunk, h0=h0d, z0=z0d, h_out=ho, z_out=zo,
+                          log_decay=torch.from_numpy(ld).cuda(), value_dt=True)
+    torch.cuda.synchronize()
+    y_ref, _, h_ref, z_ref = oracle.ssd_recurrent(
+        x["q"], x["k"], x["v"], x["dt_p"], None, x["dt_bias"], x["D"], order, norm,
+        return_norm=True, return_state=True, log_decay=ld, value_dt=True, h0=h0,
+        z0=z0 if use_z else None)
+    assert rel_err(_np(y), y_ref) <= TOL[dtype]
+    assert rel_err(_np(ho), h_ref) <= TOL[dtype]
+    if use_z:
+        assert rel_err(_np(zo), z_ref) <= TOL[dtype]
