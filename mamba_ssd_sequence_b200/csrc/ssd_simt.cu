@@ -40,6 +40,27 @@ __device__ __forceinline__ void store_elem(__nv_bfloat16 *p, size_t i, float x) 
 }
 
 // softplus(x) = log(1 + e^x) in the overflow-free form.
+// softplus for kernel (a), whose time the accurate expf and log1pf bounded:
+// softplus(x) = max(x, 0) + log1p(u), u = exp(-|x|) in (0, 1], with u from
+// the hardware base-2 exponential (ex2.approx, relative error about 2^-22;
+// u below 2^-126 flushes to zero, where softplus(x) = x or 0 to float
+// precision anyway) and log1p(u) = u p(u), p the degree-8 Chebyshev
+// interpolant of log1p(u)/u on [0, 1] (coefficients from
+// mamba_ssd_sequence_b200/gen_log1p_poly.py; relative error 2.6e-7 in float32).
+__device__ __forceinline__ float softplus_fast(float x) {
+    float u;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(u) : "f"(-fabsf(x) * 1.4426950408889634f));
+    float p = 5.126102362e-03f;
+    p = fmaf(p, u, -2.907406539e-02f);
+    p = fmaf(p, u, 7.751608640e-02f);
+    p = fmaf(p, u, -1.360224783e-01f);
+    p = fmaf(p, u, 1.907688081e-01f);
+    p = fmaf(p, u, -2.483539879e-01f);
+    p = fmaf(p, u, 3.331812024e-01f);
+    p = fmaf(p, u, -4.999944568e-01f);
+    p = fmaf(p, u, 9.999999404e-01f);
+    return fmaxf(x, 0.0f) + u * p;
+}
 __device__ __forceinline__ float softplus_f(float x) {
     return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
 }
@@ -50,8 +71,7 @@ __device__ __forceinline__ float softplus_f(float x) {
 // thread t takes the four consecutive tokens 4t..4t+3 (16-byte loads and
 // stores); every block's loads are issued before any is used.  One block per
 // CTA measured fastest: more keep more loads in flight per thread but leave
-// small problems with too few CTAs, and large ones are bound by the
-// per-token softplus (expf and log1pf) rather than by HBM.  A chunk of C
+// small problems with too few CTAs.  A chunk of C
 // tokens is C/4 threads: a
 // segment of 16 or 32 lanes for C = 64 or 128, two warps for C = 256.
 // Chunks are contiguous in the flattened [B H N] order and never straddle a
@@ -96,10 +116,10 @@ chunk_cumsum_kernel(const float *__restrict__ dt_p, const float *__restrict__ A_
             const bool live = tok0[u] < total;
             const float A = live ? -expf(__ldg(A_log + h[u])) : 0.0f;
             const float bias = live ? __ldg(dt_bias + h[u]) : 0.0f;
-            a[u][0] = A * softplus_f(x[u].x + bias);
-            a[u][1] = A * softplus_f(x[u].y + bias);
-            a[u][2] = A * softplus_f(x[u].z + bias);
-            a[u][3] = A * softplus_f(x[u].w + bias);
+            a[u][0] = A * softplus_fast(x[u].x + bias);
+            a[u][1] = A * softplus_fast(x[u].y + bias);
+            a[u][2] = A * softplus_fast(x[u].z + bias);
+            a[u][3] = A * softplus_fast(x[u].w + bias);
         }
         a[u][1] += a[u][0];
         a[u][2] += a[u][1];
