@@ -136,8 +136,8 @@ int ssd_fwd(const void *q, const void *k, const void *v,
  *              be NULL.
  * ssd_fwd(...) is ssd_fwd_ex(..., log_decay = NULL, flags = 0).
  * workspace_bytes must be at least ssd_workspace_bytes_ex(..., flags, 0).
- * Paths: order 1 and order-2 decay options run on the tensor-core paths; order
- * 2 with SSD_VALUE_DT runs on the SIMT path.
+ * Paths: both options run on the tensor-core paths where the shape allows
+ * (value discretisation scales V by dt on chip); otherwise on the SIMT path.
  * Errors as ssd_fwd(), plus SSD_ERR_FLAGS for unknown flag bits.
  */
 int ssd_fwd_ex(const void *q, const void *k, const void *v,
