@@ -4,11 +4,12 @@
 // The chunked form of 2Mamba2Furious (thelatestinai.com summary page,
 // Algorithms 3-5) splits the masked product into work that is independent per
 // chunk and one short recurrence over chunk states.  Three launches:
-//   (1) chunk_state_kernel, one CTA per chunk c of a head:
+//   (1) chunk_state_kernel, persistent, one compute group per chunk c of a head:
 //         acs_t = chunk-local inclusive cumsum of A dt (log2 units), lam = acs_{C-1}
 //         U_c   = sum_j 2^(lam - acs_j) k_j v_j^T          (tcgen05, M = N = 64, K = C)
-//   (2) state_pass_kernel: h_{-1} = 0, hin_c = bf16(h_{c-1}),
+//   (2) state_pass_kernel: h_{-1} = h0 (or 0), hin_c = bf16(h_{c-1}),
 //         h_c = 2^lam_c h_{c-1} + U_c                      (fp32, elementwise over the 64 x 64 state)
+//         and h_out = h of the last chunk when asked for
 //   (3) chunk_scan_kernel, persistent, one 128-row output tile per step:
 //         S = Q K^T over the keys of the chunk up to the tile's last row   (tcgen05)
 //         P_ij = S_ij 2^(acs_i - acs_j) [j <= i]           (CUDA cores)
