@@ -336,6 +336,44 @@ def main():
     a_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in a_ev), dev_name) / args.steps
     a_bytes = 4 * (dev["dt_p"].numel() + acs_a.numel() + csum_a.numel())
 
+    # the memory-bound entry points beside the operator, each timed alone with
+    # the L2 flushed before every call: one order-2 decode step at d_h = 64
+    # (it reads and writes the whole state, 1 MiB per head) and the conv1d +
+    # SiLU prologue over this workload's q
+    def time_calls(fn):
+        for _ in range(max(3, args.warmup)):
+            flush_l2(1.0)
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_l2(float(i))
+            ev[i][0].record(stream)
+            fn()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(sum(s_.elapsed_time(e_) for s_, e_ in ev), dev_name) / args.steps
+
+    dB, dH, dd = 2, 8, 64
+    xd = inputs.make_inputs(dB, dH, 1, dd, "bf16", seed=rank)
+    dq, dk, dv = (torch.from_numpy(xd[n + "_bits"].view(np.int16)).view(torch.bfloat16)
+                  .reshape(dB, dH, dd).to(dev_name) for n in ("q", "k", "v"))
+    ddt = torch.from_numpy(xd["dt_p"]).reshape(dB, dH).to(dev_name)
+    dpar = {n: torch.from_numpy(xd[n]).to(dev_name) for n in ("A_log", "dt_bias", "D")}
+    hst = torch.zeros((dB, dH, dd * dd, dd), dtype=torch.float32, device=dev_name)
+    zst = torch.zeros((dB, dH, dd * dd), dtype=torch.float32, device=dev_name)
+    dout = torch.empty_like(dq)
+    dws = torch.empty(ssd.ssd_decode_workspace_bytes(dB, dH, dd, 2), dtype=torch.uint8, device=dev_name)
+    dec_ms = time_calls(lambda: ssd.ssd_decode_step(dq, dk, dv, ddt, dpar["A_log"], dpar["dt_bias"], dpar["D"],
+                                                    2, True, hst, zst, out=dout, workspace=dws, stream=stream))
+    dec_bytes = 2 * 4 * (hst.numel() + zst.numel()) + 2 * (4 * dq.numel()) + 4 * ddt.numel()
+
+    cw = torch.from_numpy(np.random.default_rng(rank).standard_normal((w.H * w.d, 4)).astype(np.float32) / 2.0)
+    cw = cw.to(dev_name)
+    cout = torch.empty_like(dev["q"])
+    conv_ms = time_calls(lambda: ssd.ssd_conv1d(dev["q"], cw, None, True, out=cout, stream=stream))
+    conv_bytes = 2 * dev["q"].numel() * dev["q"].element_size() + 4 * cw.numel()
+
     # end to end: pinned host inputs -> device -> ssd_fwd -> host, per step
     e2e = None
     if not args.no_e2e:
@@ -412,6 +450,16 @@ def main():
                      "ms_per_launch": a_ms, "bytes_per_launch": a_bytes,
                      "achieved_gbs": a_bytes / (a_ms / 1e3) / 1e9,
                      "frac_of_hbm": a_bytes / (a_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
+        "decode_step": {"what": "one order-2 recurrent step with the normaliser, B=2 H=8 d_h=64 "
+                                "(reads and writes h and z), L2 flushed before each",
+                        "ms_per_call": dec_ms, "bytes_per_call": dec_bytes,
+                        "achieved_gbs": dec_bytes / (dec_ms / 1e3) / 1e9,
+                        "frac_of_hbm": dec_bytes / (dec_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
+        "conv1d": {"what": "causal depthwise conv1d (width 4) + SiLU over this workload's q, "
+                           "L2 flushed before each",
+                   "ms_per_call": conv_ms, "bytes_per_call": conv_bytes,
+                   "achieved_gbs": conv_bytes / (conv_ms / 1e3) / 1e9,
+                   "frac_of_hbm": conv_bytes / (conv_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
         "device_status": status,
         "clocks": clk.summary(),
     }
