@@ -115,21 +115,32 @@ decode_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     if (tid <= d) part[((size_t)bh * S + s) * (d + 1) + tid] = ys[tid];
 }
 
+// Block (65, 4): thread (c, g) sums column c (c = d: the normaliser) over the
+// slices s = g, g + 4, ..., so that four independent chains of loads are in
+// flight per column rather than one chain over all S slices.
 template <typename T>
-__global__ void decode_output_kernel(const T *__restrict__ v, const float *__restrict__ D,
-                                     const float *__restrict__ part, int H, int d, int S,
-                                     int normalize, T *__restrict__ out) {
-    const int bh = blockIdx.x, c = threadIdx.x;
-    if (c >= d) return;
+__global__ void __launch_bounds__(65 * 4)
+decode_output_kernel(const T *__restrict__ v, const float *__restrict__ D,
+                     const float *__restrict__ part, int H, int d, int S,
+                     int normalize, T *__restrict__ out) {
+    __shared__ float red[4][65];
+    const int bh = blockIdx.x, c = threadIdx.x, g = threadIdx.y;
     const float *p = part + (size_t)bh * S * (d + 1);
-    float y = 0.0f, n = 0.0f;
-    for (int s = 0; s < S; ++s) {
-        y += p[(size_t)s * (d + 1) + c];
-        n += p[(size_t)s * (d + 1) + d];
+    float acc = 0.0f;
+    if (c <= d) {
+#pragma unroll 4
+        for (int s = g; s < S; s += 4) acc += p[(size_t)s * (d + 1) + c];
     }
-    if (normalize) y /= n;
-    if (D) y = fmaf(D[(bh % H) * d + c], load_elem(v, (size_t)bh * d + c), y);
-    store_elem(out, (size_t)bh * d + c, y);
+    red[g][c] = acc;
+    __syncthreads();
+    if (g == 0 && c <= d) red[0][c] = (red[0][c] + red[1][c]) + (red[2][c] + red[3][c]);
+    __syncthreads();
+    if (g == 0 && c < d) {
+        float y = red[0][c];
+        if (normalize) y /= red[0][d];
+        if (D) y = fmaf(D[(bh % H) * d + c], load_elem(v, (size_t)bh * d + c), y);
+        store_elem(out, (size_t)bh * d + c, y);
+    }
 }
 
 template <typename T>
@@ -140,8 +151,8 @@ int run_decode(const FwdArgs &a, float *h, float *z) {
     decode_state_kernel<T><<<dim3(BH, S), kDecThreads, 0, a.stream>>>(
         static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.dt_p,
         a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.d, a.order, h, z, part);
-    decode_output_kernel<T><<<BH, 64, 0, a.stream>>>(static_cast<const T *>(a.v), a.D, part, a.H,
-                                                     a.d, S, a.normalize, static_cast<T *>(a.out));
+    decode_output_kernel<T><<<BH, dim3(65, 4), 0, a.stream>>>(static_cast<const T *>(a.v), a.D, part, a.H,
+                                                              a.d, S, a.normalize, static_cast<T *>(a.out));
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
