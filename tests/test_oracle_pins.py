@@ -484,3 +484,23 @@ def test_conv1d_identity_and_shift_and_causality():
     x3 = x.copy()
     x3[:, 1] = 0.0                                        # another head only
     np.testing.assert_array_equal(oracle.conv1d(x3, w, silu=True)[:, 0], y[:, 0])
+
+
+def test_conv1d_hand_worked_per_head_weights():
+    """Two heads of two channels, window 2, with a different weight row for
+    every channel h*d + c (the weight row of channel c of head h), and a second
+    batch holding the negated tokens.  Worked by hand:
+      head 0, w = (1, 10), (2, 20), tokens (1, 2), (3, 4):
+        u_0 = (1*1, 2*2) = (1, 4);  u_1 = (1*3 + 10*1, 2*4 + 20*2) = (13, 48)
+      head 1, w = (3, 30), (4, 40), tokens (5, 6), (7, 8):
+        u_0 = (3*5, 4*6) = (15, 24); u_1 = (3*7 + 30*5, 4*8 + 40*6) = (171, 272)
+    The second batch gives the negated values (the weights depend on the head
+    only).  Indexing the weights by the channel alone, by b*H + h, or with the
+    weight array transposed changes at least one of these values."""
+    x = np.asarray([[[[1, 2], [3, 4]], [[5, 6], [7, 8]]]], np.float32)
+    x = np.concatenate([x, -x], axis=0)                   # [B=2, H=2, N=2, d=2]
+    w = np.asarray([[1, 10], [2, 20], [3, 30], [4, 40]], np.float32)
+    u = oracle.conv1d(x, w, None, silu=False)
+    want = np.asarray([[[1, 4], [13, 48]], [[15, 24], [171, 272]]], np.float64)
+    np.testing.assert_array_equal(u[0], want)
+    np.testing.assert_array_equal(u[1], -want)
