@@ -207,9 +207,14 @@ int ssd_status_from_workspace(const void *workspace, void *stream);
  *  - Problems whose scratch (the same as ssd_fwd's SIMT path: about
  *    4*B*H*N + 4*B*H*(N/chunk)*d_h^order*(d_h+1) bytes) exceeds 16 MiB are
  *    rejected with SSD_ERR_WORKSPACE before anything is enqueued.
- *  - The first call on a device looks up the buffer's device address on
- *    that device (cudaGetSymbolAddress); make that first call before any
- *    stream capture.
+ *  - It runs in the CUDA context current on the calling thread (the
+ *    runtime's primary context, or a context the host application made
+ *    itself with the driver API).  The first call in each context looks up
+ *    the buffer's device address there (cudaGetSymbolAddress, which also
+ *    loads the library's module into that context if needed); make that
+ *    first call before any stream capture.  Later calls in the same context
+ *    reuse the address; a new context -- one created later, or the primary
+ *    context re-created after cudaDeviceReset -- gets its own lookup.
  *  - All calls on one device share the one buffer and it keeps the last
  *    call's contents (the kernels write everything they later read).  Calls
  *    that can overlap on the GPU -- on different streams without ordering

@@ -21,19 +21,21 @@ static int check_shape(int B, int H, int N, int d, int dtype, int order, int chu
     return SSD_OK;
 }
 
-static size_t simt_total(int B, int H, int N, int d, int order, int chunk, Plan *p) {
+void simt_layout(int B, int H, int N, int d, int order, int chunk, Plan *p) {
     const size_t BH = (size_t)B * H, nc = (size_t)N / chunk;
     const size_t Dphi = order == 1 ? (size_t)d : (size_t)d * d;
+    p->path = PATH_SIMT;
+    p->n_launches = 4;
     p->acs_off = kStatusBytes;
     p->lam_off = align_up(p->acs_off + BH * N * sizeof(float), 256);
     p->state_off = align_up(p->lam_off + BH * nc * sizeof(float), 256);
     p->total = align_up(p->state_off + BH * nc * Dphi * (d + 1) * sizeof(float), 256);
-    return p->total;
 }
 
-bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
-               int value_dt, int state, Plan *plan) {
-    if (check_shape(B, H, N, d, dtype, order, chunk) != SSD_OK) return false;
+int make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
+              int value_dt, int state, Plan *plan) {
+    const int rc = check_shape(B, H, N, d, dtype, order, chunk);
+    if (rc != SSD_OK) return rc;
     Plan p{};
     if (order == 1 && !normalize && !(state & SSD_STATE_Z) &&
         tc_order1_supports(B, H, N, d, dtype, chunk)) {
@@ -46,12 +48,11 @@ bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, 
         p.acs_off = p.lam_off = p.state_off = kStatusBytes;
         p.total = kStatusBytes + tc_order2_workspace(B, H, N, d, chunk);
     } else {
-        p.path = PATH_SIMT;
-        p.n_launches = 4;
-        simt_total(B, H, N, d, order, chunk, &p);
+        if (N / chunk > kMaxSimtChunks) return SSD_ERR_SHAPE;
+        simt_layout(B, H, N, d, order, chunk, &p);
     }
     *plan = p;
-    return true;
+    return SSD_OK;
 }
 
 }  // namespace ssd
@@ -67,7 +68,7 @@ size_t ssd_workspace_bytes_ex(int B, int H, int N, int d_h, int dtype, int order
     size_t need = 0;
     for (int norm = 0; norm < 2; ++norm) {
         Plan p;
-        if (!make_plan(B, H, N, d_h, dtype, order, norm, chunk, flags & SSD_VALUE_DT, state, &p))
+        if (make_plan(B, H, N, d_h, dtype, order, norm, chunk, flags & SSD_VALUE_DT, state, &p) != SSD_OK)
             return 0;
         if (p.total > need) need = p.total;
     }
@@ -81,7 +82,7 @@ size_t ssd_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, i
 int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
                  int *n_launches) {
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, 0, chunk, 0, 0, &p)) return -1;
+    if (make_plan(B, H, N, d_h, dtype, order, 0, chunk, 0, 0, &p) != SSD_OK) return -1;
     if (n_launches) *n_launches = p.n_launches;
     return p.path;
 }
@@ -106,8 +107,8 @@ int ssd_fwd_state(const void *q, const void *k, const void *v, const float *dt_p
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
     const int state = ((h0 || h_out) ? SSD_STATE_H : 0) | ((z0 || z_out) ? SSD_STATE_Z : 0);
     Plan p;
-    if (!make_plan(B, H, N, d_h, dtype, order, normalize, chunk, value_dt, state, &p))
-        return SSD_ERR_UNSUPPORTED;
+    rc = make_plan(B, H, N, d_h, dtype, order, normalize, chunk, value_dt, state, &p);
+    if (rc != SSD_OK) return rc;
     if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
     FwdArgs a{q, k, v, need_dt ? dt_p : nullptr, log_decay ? nullptr : A_log,
               need_dt ? dt_bias : nullptr, D, log_decay, value_dt, h0, z0, h_out, z_out,

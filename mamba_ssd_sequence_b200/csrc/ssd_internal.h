@@ -46,10 +46,20 @@ struct Plan {
     size_t acs_off, lam_off, state_off, aux_off, vfac_off, total;
 };
 
-// Fills `plan` for validated arguments; returns false if no kernel exists.
-// state: SSD_STATE_H / SSD_STATE_Z bits of the state arguments in use.
-bool make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
-               int value_dt, int state, Plan *plan);
+// Fills `plan` for the arguments and returns SSD_OK, or the status that
+// rejects them (SSD_ERR_SHAPE etc. for invalid shapes, SSD_ERR_UNSUPPORTED
+// when no kernel exists).  state: SSD_STATE_H / SSD_STATE_Z bits of the
+// state arguments in use.
+int make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, int chunk,
+              int value_dt, int state, Plan *plan);
+
+// Scratch layout of the SIMT path: status block, chunk-local decay, chunk
+// totals, per-chunk carried states with the normaliser column.  Fills the
+// offsets and the total of `p` (path and launch count included).
+void simt_layout(int B, int H, int N, int d, int order, int chunk, Plan *p);
+
+// The SIMT path puts the chunk index in gridDim.y.
+constexpr int kMaxSimtChunks = 65535;
 
 // Path launchers (each returns an ssd_status).
 int launch_simt(const FwdArgs &a, const Plan &p);

@@ -4,8 +4,13 @@
 //
 // The scratch is a file-scope __device__ array.  In host code its name is
 // only a host-side stand-in, never a device address, so the address handed
-// to the kernels comes from cudaGetSymbolAddress, looked up once per device
-// (with that device current) on the first call made on it.
+// to the kernels comes from cudaGetSymbolAddress, looked up with the context
+// current.  A __device__ symbol's address belongs to the context the module
+// was loaded into, so the address is remembered per context -- keyed by the
+// context's ID, which the driver never reuses within a process -- and looked
+// up again for a context not seen before: a plugin whose host application
+// creates its own contexts, or any context made after cudaDeviceReset.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -15,25 +20,57 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB per GPU
-constexpr int kMaxDevices = 64;
+constexpr int kCacheSlots = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-void *g_scratch_dev_ptr[kMaxDevices] = {};
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
+
+struct CacheSlot {
+    unsigned long long ctx_id;
+    void *ptr;
+};
+CacheSlot g_cache[kCacheSlots] = {};
+int g_cache_next = 0;
 std::mutex g_scratch_mutex;
 
-// Device address of g_noalloc_scratch on the current device (nullptr on error).
-void *scratch_for_current_device() {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_dev_ptr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-            return nullptr;
-        g_scratch_dev_ptr[dev] = p;
+template <typename F>
+F driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<F>(p);
+}
+
+// Device address of g_noalloc_scratch in the calling thread's current context
+// (nullptr on error).  The first call in a context loads the library's module
+// there if it is not loaded yet.
+void *scratch_for_current_context() {
+    static PfnCtxGetCurrent get_ctx = driver_fn<PfnCtxGetCurrent>("cuCtxGetCurrent");
+    static PfnCtxGetId get_id = driver_fn<PfnCtxGetId>("cuCtxGetId");
+    if (!get_ctx || !get_id) return nullptr;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
+    if (ctx == nullptr) {
+        // no context current on this thread yet: make the runtime's primary
+        // context of the current device current (this allocates nothing)
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return nullptr;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
     }
-    return g_scratch_dev_ptr[dev];
+    unsigned long long id = 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    for (const CacheSlot &s : g_cache)
+        if (s.ptr != nullptr && s.ctx_id == id) return s.ptr;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_cache[g_cache_next] = CacheSlot{id, p};
+    g_cache_next = (g_cache_next + 1) % kCacheSlots;
+    return p;
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -46,32 +83,23 @@ extern "C" int ssd_fwd_noalloc(const void *q, const void *k, const void *v, cons
                                int chunk, void *out, void *stream) {
     using namespace ssd;
     if (!q || !k || !v || !dt_p || !A_log || !dt_bias || !out) return SSD_ERR_NULL;
-    // ssd_workspace_bytes validates shape, dtype, order and chunk (0 = invalid)
-    if (ssd_workspace_bytes(B, H, N, d_h, dtype, order, chunk) == 0) {
-        if (dtype != SSD_F32 && dtype != SSD_BF16) return SSD_ERR_DTYPE;
-        if (order != 1 && order != 2) return SSD_ERR_ORDER;
-        if (chunk != 64 && chunk != 128 && chunk != 256) return SSD_ERR_CHUNK;
-        return SSD_ERR_SHAPE;
-    }
+    // make_plan validates shape, dtype, order and chunk
+    Plan chosen{};
+    const int rc = make_plan(B, H, N, d_h, dtype, order, normalize, chunk, 0, 0, &chosen);
+    if (rc != SSD_OK) return rc;
+    if ((size_t)N / chunk > (size_t)kMaxSimtChunks) return SSD_ERR_SHAPE;
     const void *ptrs[] = {q, k, v, dt_p, A_log, dt_bias, out};
     for (const void *p : ptrs)
         if (!aligned16(p)) return SSD_ERR_ALIGN;
     if (D && !aligned16(D)) return SSD_ERR_ALIGN;
 
-    // Layout of the SIMT path's scratch: status block, chunk-local decay,
-    // chunk totals, per-chunk carried states (with the normaliser column).
-    const size_t BH = (size_t)B * H, nc = (size_t)N / chunk;
-    const size_t Dphi = order == 1 ? (size_t)d_h : (size_t)d_h * d_h;
+    // this entry point always runs the SIMT path, with the same scratch layout
+    // as ssd_fwd's SIMT path
     Plan p{};
-    p.path = PATH_SIMT;
-    p.n_launches = 4;
-    p.acs_off = kStatusBytes;
-    p.lam_off = align_up(p.acs_off + BH * N * sizeof(float), 256);
-    p.state_off = align_up(p.lam_off + BH * nc * sizeof(float), 256);
-    p.total = align_up(p.state_off + BH * nc * Dphi * (d_h + 1) * sizeof(float), 256);
+    simt_layout(B, H, N, d_h, order, chunk, &p);
     if (p.total > kNoAllocScratchBytes) return SSD_ERR_WORKSPACE;
 
-    void *scratch = scratch_for_current_device();
+    void *scratch = scratch_for_current_context();
     if (!scratch) return SSD_ERR_CUDA;
     FwdArgs a{q, k, v, dt_p, A_log, dt_bias, D, nullptr, 0, nullptr, nullptr, nullptr, nullptr,
               B, H, N, d_h, dtype, order, normalize ? 1 : 0,

@@ -73,6 +73,16 @@ def test_fwd_validation_codes(lib):
     assert _call_fwd(lib, ws_bytes=100) == 7
 
 
+def test_simt_path_chunk_count_bound(lib):
+    """The SIMT path puts the chunk index in gridDim.y (at most 65535): a
+    problem that would need more chunks there is rejected as a shape error
+    before anything is enqueued, and has no workspace size."""
+    N = 65536 * 64  # 65536 chunks of 64 tokens on the fp32 (SIMT) path
+    assert ssd.ssd_workspace_bytes(1, 1, N, 16, ssd.SSD_F32, 1, 64) == 0
+    assert _call_fwd(lib, B=1, H=1, N=N) == 2   # SSD_ERR_SHAPE
+    assert ssd.ssd_workspace_bytes(1, 1, 65535 * 64, 16, ssd.SSD_F32, 1, 64) > 0
+
+
 def test_status_strings(lib):
     for code in range(11):
         s = ssd.status_str(code)
