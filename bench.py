@@ -97,6 +97,26 @@ def algorithmic_work(w: inputs.Workload):
     return T * per_tok_bytes, T * per_tok_flops, per_tok_bytes, per_tok_flops
 
 
+def roofline_of(w: inputs.Workload, mean_ms: float, peaks, peak_src: str):
+    """The roofline object of one call of workload `w` that took `mean_ms`:
+    order 1 is bound by HBM (algorithmic bytes / time against hbm_gbs), order
+    2 by the tensor cores (algorithmic FLOPs / time against bf16_tflops)."""
+    alg_bytes, alg_flops, _, _ = algorithmic_work(w)
+    tflops = alg_flops / (mean_ms / 1e3) / 1e12
+    gbs = alg_bytes / (mean_ms / 1e3) / 1e9
+    if w.order == 1:
+        bound, achieved, peak, unit = "hbm", gbs, float(peaks["hbm_gbs"]), "GB/s"
+    else:
+        bound, achieved, peak, unit = "tensor", tflops, float(peaks["bf16_tflops"]), "TFLOP/s"
+    traffic = DRAM_TRAFFIC.get(w.name)
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic,
+            "traffic_over_algorithmic": None if traffic is None else traffic / alg_bytes,
+            "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
+            "algorithmic_bytes_per_launch": alg_bytes,
+            "algorithmic_flops_per_launch": alg_flops}, tflops, gbs
+
+
 class ClockSampler:
     """nvidia-smi clocks/throttle reasons sampled every 200 ms while running."""
 
@@ -247,6 +267,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="time only the selected workload (skip the other bf16 workloads)")
     args = ap.parse_args()
     w = inputs.WORKLOADS[args.workload]
     if args.impl == "reference":
@@ -311,6 +333,45 @@ def main():
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), dev_name)
     status = ssd.ssd_status_from_workspace(ws)
+
+    # the other bf16 workloads (order 2 at 4K tokens, order 1 at 64K tokens,
+    # order 2 at 16K tokens with d_h = 64), each timed the same way: inputs
+    # resident, L2 flushed before every step, one CUDA-event pair per step
+    others = {}
+    if not args.no_workloads:
+        for name in inputs.WORKLOAD_ORDER[1:]:
+            if name == w.name:
+                continue
+            ow = inputs.WORKLOADS[name]
+            _, oh = make_device_inputs(ow, seed=rank, torch=torch)
+            od = {k: (v.to(dev_name) if v is not None else None) for k, v in oh.items()}
+            del oh
+            oout = torch.empty_like(od["q"])
+            ows = ssd.alloc_workspace(ow.B, ow.H, ow.N, ow.d, ssd.SSD_BF16, ow.order, ow.chunk, dev_name)
+            opath, olaunch = ssd.ssd_fwd_path(ow.B, ow.H, ow.N, ow.d, ssd.SSD_BF16, ow.order, ow.chunk)
+
+            def ostep(od=od, oout=oout, ows=ows, ow=ow):
+                ssd.ssd_fwd(od["q"], od["k"], od["v"], od["dt_p"], od["A_log"], od["dt_bias"], od["D"],
+                            ow.order, ow.normalize, ow.chunk, out=oout, workspace=ows, stream=stream)
+
+            osteps = max(5, min(args.steps, 20))
+            for _ in range(max(3, args.warmup)):
+                flush_l2(1.0)
+                ostep()
+            oev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(osteps)]
+            for i in range(osteps):
+                flush_l2(float(i))
+                oev[i][0].record(stream)
+                ostep()
+                oev[i][1].record(stream)
+            torch.cuda.synchronize()
+            oms = max_over_ranks(sum(a_.elapsed_time(b_) for a_, b_ in oev), dev_name) / osteps
+            others[name] = {"ms": oms, "steps": osteps, "path": opath, "launches_per_step": olaunch,
+                            "status": ssd.ssd_status_from_workspace(ows),
+                            "value": weak_scaling_rate(ow.tokens, osteps, world, oms * osteps)}
+            del od, oout, ows
+            torch.cuda.empty_cache()
 
     # kernel (a) on its own: the chunk-local cumsum of A dt and the chunk
     # totals, which the tensor-core paths fuse into their first kernel.  It
@@ -411,15 +472,9 @@ def main():
     if rank != 0:
         return 0
 
-    alg_bytes, alg_flops, bpt, fpt = algorithmic_work(w)
     mean_ms = total_ms / args.steps
     peaks, peak_src = load_peaks()
-    tflops = alg_flops / (mean_ms / 1e3) / 1e12
-    gbs = alg_bytes / (mean_ms / 1e3) / 1e9
-    if w.order == 1:
-        bound, achieved, peak, unit = "hbm", gbs, float(peaks["hbm_gbs"]), "GB/s"
-    else:
-        bound, achieved, peak, unit = "tensor", tflops, float(peaks["bf16_tflops"]), "TFLOP/s"
+    roofline, tflops, gbs = roofline_of(w, mean_ms, peaks, peak_src)
     line = {
         "metric": METRIC,
         "value": weak_scaling_rate(w.tokens, args.steps, world, total_ms),
@@ -440,11 +495,7 @@ def main():
         "tflops": tflops,
         "tc_frac": tflops / float(peaks["bf16_tflops"]),
         "hbm_gbs": gbs,
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak, "traffic": DRAM_TRAFFIC.get(w.name),
-                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops'})",
-                     "algorithmic_bytes_per_launch": alg_bytes,
-                     "algorithmic_flops_per_launch": alg_flops},
+        "roofline": roofline,
         "gpu_launches": n_launch * args.steps,
         "kernel_a": {"what": "chunk cumsum of A dt and chunk totals, launched alone (L2 flushed before each)",
                      "ms_per_launch": a_ms, "bytes_per_launch": a_bytes,
@@ -463,6 +514,19 @@ def main():
         "device_status": status,
         "clocks": clk.summary(),
     }
+    if others:
+        wl = {}
+        for name, o in others.items():
+            ow = inputs.WORKLOADS[name]
+            rl, otf, ogbs = roofline_of(ow, o["ms"], peaks, peak_src)
+            wl[name] = {"ms_per_step": o["ms"], "steps": o["steps"], "tokens_per_s": o["value"],
+                        "tflops": otf, "hbm_gbs": ogbs, "roofline": rl,
+                        "path": {0: "simt", 1: "tc_order1", 2: "tc_order2"}.get(o["path"], o["path"]),
+                        "launches_per_step": o["launches_per_step"], "device_status": o["status"],
+                        "config": {"B": ow.B, "H": ow.H, "N": ow.N, "d_h": ow.d, "chunk": ow.chunk,
+                                   "order": ow.order, "normalize": ow.normalize,
+                                   "residual": ow.residual}}
+        line["workloads"] = wl
     if e2e is not None:
         line["e2e"] = e2e
     if not args.no_cpu_baseline:

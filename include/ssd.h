@@ -309,6 +309,31 @@ int ssd_decode_step(const void *q, const void *k, const void *v,
 int ssd_conv1d(const void *x, const float *w, const float *bias, int B, int H, int N, int d_h,
                int width, int silu, int dtype, void *out, void *stream);
 
+/*
+ * Test hook for the device-side failure detection; the pages have no
+ * counterpart.  ssd_fwd() with two arguments that only failure tests use:
+ *   skip_publish  >= 0: on the tensor-core paths, one producer inside the
+ *                 kernels skips its publication at that pipeline step, so
+ *                 the consumer's bounded wait runs out; -1: none (the call
+ *                 is then ssd_fwd())
+ *   wait_ns       limit of every bounded device-side wait in nanoseconds
+ *                 (0: the default of one second)
+ * A wait that runs out never traps: it records SSD_ERR_TIMEOUT in the
+ * workspace status, every role of the kernel stops, the copies and matrix
+ * products already in flight complete, the tensor memory is freed and the
+ * kernel returns.  ssd_status_from_workspace() then reports
+ * SSD_ERR_TIMEOUT; the output is incomplete.  The same workspace can be
+ * used by the next call (every call resets the status).  Other errors as
+ * ssd_fwd(), plus SSD_ERR_SHAPE for a negative wait_ns.
+ */
+int ssd_debug_fwd(const void *q, const void *k, const void *v,
+                  const float *dt_p, const float *A_log, const float *dt_bias,
+                  const float *D,
+                  int B, int H, int N, int d_h, int dtype,
+                  int order, int normalize, int chunk,
+                  void *out, void *workspace, size_t workspace_bytes,
+                  void *stream, int skip_publish, long long wait_ns);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *ssd_status_str(int status);
 

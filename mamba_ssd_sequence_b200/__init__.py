@@ -72,6 +72,8 @@ def load_library():
     lib.ssd_status_str.restype = ctypes.c_char_p
     lib.ssd_fwd_path.argtypes = [ci] * 7 + [ctypes.POINTER(ci)]
     lib.ssd_fwd_path.restype = ci
+    lib.ssd_debug_fwd.argtypes = [vp] * 7 + [ci] * 8 + [vp, vp, sz, vp, ci, ctypes.c_longlong]
+    lib.ssd_debug_fwd.restype = ci
     _lib = lib
     return lib
 
@@ -173,6 +175,29 @@ def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk
             SSD_VALUE_DT if value_dt else 0, _ptr(out), _ptr(workspace), workspace.numel(),
             _stream_handle(stream))
         _check(rc, "ssd_fwd_ex")
+    return out
+
+
+def ssd_debug_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk: int,
+                  skip_publish: int, wait_ns: int, out=None, workspace=None, stream=None):
+    """Failure-detection test hook (include/ssd.h: ssd_debug_fwd): ssd_fwd in
+    which one producer skips its publication at pipeline step `skip_publish`
+    (-1: none) and every bounded device-side wait gives up after `wait_ns`
+    nanoseconds.  Returns `out`; read the device status with
+    ssd_status_from_workspace(workspace)."""
+    import torch
+    B, H, N, d = q.shape
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device)
+    rc = load_library().ssd_debug_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
+        B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk),
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream),
+        int(skip_publish), int(wait_ns))
+    _check(rc, "ssd_debug_fwd")
     return out
 
 

@@ -140,6 +140,10 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
         }
     }
 }
+// Store to the shared memory of CTA `rank` of the cluster (address from mapa_shared).
+__device__ __forceinline__ void st_dsmem_u32(uint32_t cluster_addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
 // Orders this thread's (and, through an earlier CTA barrier, its CTA's)
 // memory accesses before its later ones at cluster scope.
 __device__ __forceinline__ void fence_acq_rel_cluster() {
@@ -349,6 +353,23 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
     for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
     tmem_st16(taddr, u);
 }
+// 16 lanes x 64 consecutive 32-bit columns (eight repetitions of the
+// 16x256b pattern).  Thread t of the warp holds lanes (base + t/4) and
+// (base + t/4 + 8); in repetition g, columns 8g + 2(t%4) and 8g + 2(t%4) + 1:
+// v[4g + 0] = (lane t/4, col 8g + 2(t%4)), v[4g + 1] = (lane t/4, col + 1),
+// v[4g + 2] = (lane t/4 + 8, col 8g + 2(t%4)), v[4g + 3] = (lane t/4 + 8, col + 1).
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
 // 32 lanes x 1 32-bit column.
 __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     uint32_t r;
@@ -381,6 +402,13 @@ __device__ __forceinline__ uint32_t sw64_chunk(uint32_t row, uint32_t ch) {
 }
 __device__ __forceinline__ uint32_t sw32_chunk(uint32_t row, uint32_t ch) {
     return row * 32u + (((ch ^ (row >> 2)) & 1u) << 4);
+}
+
+// Element-wise bf16x2 product, rounded to nearest even.
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -87,11 +87,15 @@ int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,
     return p.path;
 }
 
-int ssd_fwd_state(const void *q, const void *k, const void *v, const float *dt_p,
-                  const float *A_log, const float *dt_bias, const float *D, const float *log_decay,
-                  int B, int H, int N, int d_h, int dtype, int order, int normalize, int chunk,
-                  int flags, const float *h0, const float *z0, float *h_out, float *z_out,
-                  void *out, void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, const float *A_log,
+               const float *dt_bias, const float *D, const float *log_decay, int B, int H, int N,
+               int d_h, int dtype, int order, int normalize, int chunk, int flags, const float *h0,
+               const float *z0, float *h_out, float *z_out, void *out, void *workspace,
+               size_t workspace_bytes, void *stream, int dbg_skip, unsigned long long wait_ns) {
     if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
     const int value_dt = (flags & SSD_VALUE_DT) ? 1 : 0;
     if (!q || !k || !v || !out) return SSD_ERR_NULL;
@@ -114,11 +118,38 @@ int ssd_fwd_state(const void *q, const void *k, const void *v, const float *dt_p
               need_dt ? dt_bias : nullptr, D, log_decay, value_dt, h0, z0, h_out, z_out,
               B, H, N, d_h, dtype, order, normalize ? 1 : 0, chunk, out, workspace,
               workspace_bytes, static_cast<cudaStream_t>(stream)};
+    a.dbg_skip = dbg_skip;
+    a.wait_ns = wait_ns;
     switch (p.path) {
     case PATH_TC_ORDER1: return launch_tc_order1(a, p);
     case PATH_TC_ORDER2: return launch_tc_order2(a, p);
     default: return launch_simt(a, p);
     }
+}
+
+}  // namespace
+
+extern "C" {
+
+int ssd_fwd_state(const void *q, const void *k, const void *v, const float *dt_p,
+                  const float *A_log, const float *dt_bias, const float *D, const float *log_decay,
+                  int B, int H, int N, int d_h, int dtype, int order, int normalize, int chunk,
+                  int flags, const float *h0, const float *z0, float *h_out, float *z_out,
+                  void *out, void *workspace, size_t workspace_bytes, void *stream) {
+    return fwd_common(q, k, v, dt_p, A_log, dt_bias, D, log_decay, B, H, N, d_h, dtype, order, normalize,
+                      chunk, flags, h0, z0, h_out, z_out, out, workspace, workspace_bytes, stream, -1, 0);
+}
+
+int ssd_debug_fwd(const void *q, const void *k, const void *v, const float *dt_p,
+                  const float *A_log, const float *dt_bias, const float *D, int B, int H, int N,
+                  int d_h, int dtype, int order, int normalize, int chunk, void *out,
+                  void *workspace, size_t workspace_bytes, void *stream, int skip_publish,
+                  long long wait_ns) {
+    if (wait_ns < 0) return SSD_ERR_SHAPE;
+    if (!dt_p || !A_log || !dt_bias) return SSD_ERR_NULL;
+    return fwd_common(q, k, v, dt_p, A_log, dt_bias, D, nullptr, B, H, N, d_h, dtype, order, normalize,
+                      chunk, 0, nullptr, nullptr, nullptr, nullptr, out, workspace, workspace_bytes, stream,
+                      skip_publish, (unsigned long long)wait_ns);
 }
 
 int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,

@@ -23,6 +23,11 @@ struct FwdArgs {
     void *workspace;
     size_t workspace_bytes;
     cudaStream_t stream;
+    // failure-detection test hook (ssd_debug_fwd): the iteration whose
+    // publication a producer skips (-1: none), and the bounded waits' limit in
+    // nanoseconds (0: the default of one second)
+    int dbg_skip = -1;
+    unsigned long long wait_ns = 0;
 };
 
 // Device status block at the start of every workspace: status code (an

@@ -1,34 +1,47 @@
 // Order-2 (2Mamba, squared scores) tensor-core path (tcgen05 + TMEM, TMA) of
-// the SSD forward operator for bf16 inputs, d_h in {32, 64}, chunk = 64.
+// the SSD forward operator for bf16 inputs, d_h = D in {32, 64}, chunk = 64.
 //
 // Order 2 squares the score: w_ij = (q_i . k_j)^2 2^(acs_i - acs_j), whose
 // recurrent form (2Mamba2Furious, Algorithm 6) carries the state
-// h = sum_j 2^(A_t - A_j) (k_j (x) k_j) v_j^T of d_h^2 x d_h values, plus the
-// normaliser state z = sum_j 2^(A_t - A_j) (k_j (x) k_j).  The state of one
-// head does not fit one SM at d_h = 64 (1 MiB), so a thread-block cluster of
-// R = d_h^2 / 512 CTAs shares a head: CTA r keeps feature rows
-// [512 r, 512 r + 512) of h and z in tensor memory (fp32) -- feature (a, b)
-// is row a d_h + b -- and the cluster walks the chunks together.  Per chunk
-// of C = 64 tokens, every CTA:
-//   acs_t = chunk-local inclusive cumsum of A dt (log2 units)   (kernel (a), fused)
-//   S     = Q K^T                                      tcgen05 (M = 64)
-//   P_ij  = S_ij^2 2^(acs_i - acs_j) [i >= j],  r_i = sum_j P_ij   CUDA cores
-//   Y     = P V                                        tcgen05
-//   over its 4 slabs of 128 feature rows:
-//     hb    = bf16(h_slab)  (the state entering the chunk); h_slab *= 2^lam
-//     Fk    = [w_j k_ja k_jb]_{j, (a,b)},  w_j = 2^(lam - acs_j)
-//     Fq    = [2^acs_i q_ia q_ib]_{i, (a,b)}
-//     h_slab += Fk^T V,   z_slab += Fk^T 1             tcgen05 (M = 128)
-//     T     += Fq hb,     Tn += Fq zb                  tcgen05 (M = 64)
-// The cluster then sums the partial T, Tn of its CTAs through distributed
-// shared memory: CTA r owns rows [64 r / R, 64 (r + 1) / R) of the chunk and
-// writes y_i = (Y_i + sum T_i) / (r_i + sum Tn_i) [+ D v_i].  The
-// (q . k)^2 of the intra-chunk part is the same inner product as
-// (q (x) q) . (k (x) k) of the feature form (Algorithm 5 vs Algorithm 6).
+// h = sum_j 2^(A_t - A_j) (k_j (x) k_j) v_j^T of D^2 x D values and the
+// normaliser state z = sum_j 2^(A_t - A_j) (k_j (x) k_j).  One head's state
+// does not fit one SM at D = 64 (1 MiB), so R = D^2 / 512 CTAs share a head:
+// each keeps 512 of the D^2 feature rows of h in tensor memory (fp32), as
+// four slabs of 128 rows, and z of those features in registers.  The feature
+// of TMEM lane L of slab s of CTA r is (a, b) with
+//     a = r (512 / D) + 4 (L / D) + s,   b = L % D,
+// so the four slabs of a lane share b, and a warp shares a.
+//
+// Per chunk c of 64 tokens (acs_t = chunk-local inclusive cumsum of A dt in
+// log2 units, lam = acs_63; kernel (a), fused), every CTA, slab by slab:
+//   state build   h <- 2^lam h + Fk^T V                    tcgen05, M = 128
+//                 Fk[j][(a,b)] = 2^(lam - acs_j) k_ja k_jb (A operand in TMEM)
+//                 z <- 2^lam z + sum_j Fk[j]               CUDA cores (fp32)
+//   readout       [T | Tn] += Fq [hb | zb]                 tcgen05, M = 64
+//                 Fq[i][(a,b)] = 2^acs_i q_ia q_ib         (A operand in smem)
+//                 hb, zb = bf16 of the state entering the chunk (B in smem)
+// and one CTA of the head (c mod R) adds the chunk's own quadratic part:
+//   S = Q K^T,  P_ij = S_ij^2 2^(acs_i - acs_j) [i >= j],  T += P V,
+// with the row sums of P added to Tn.  The R partial [T | Tn] of a chunk are
+// summed across the head's CTAs -- through distributed shared memory within
+// a thread-block cluster at D = 32, through L2 with counters at D = 64 (where
+// a cluster of 8 per head would not fit all heads at once) -- and CTA r
+// writes rows [64r/R, 64(r+1)/R):   y_i = T_i / Tn_i (normaliser on) [+ D v_i].
+// The (q . k)^2 of the quadratic part and (q (x) q) . (k (x) k) of the state
+// part are the same inner product (Algorithm 5 against Algorithm 6).
+//
+// Roles (608 threads): warp 0 TMA; warp 1 MMA issue; warps 2-9 the state
+// team (slabs 0, 2 and slabs 1, 3: state conversion and scaling, Fk, z);
+// warps 10-13 the query team (Fq, P); warps 14-17 the output team (partials,
+// reduction across the head's CTAs, output); warp 18 the decay warp (kernel
+// (a): the chunk's decay, key weights and value discretisation, one chunk
+// ahead).  Every slab has a buffer of its own in each ring, so a slab's
+// preparation for chunk c waits only for that slab's products of chunk c - 1.
 // Options: a per-token log-decay and value discretisation (Algorithm 4; V is
-// scaled by dt in shared memory); a carried state h0, z0 enters as the state
-// before chunk 0, and h_out, z_out receive the state after the last chunk.
-// All exponentials are of non-positive arguments.  Every wait is bounded.
+// scaled by dt in shared memory, the normaliser and the residual use the raw
+// scores and v); a carried state h0, z0 enters as the state before chunk 0,
+// and h_out, z_out receive the state after the last chunk.  All exponentials
+// are of non-positive arguments.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -48,57 +61,73 @@ constexpr int kC = 64;          // chunk length
 constexpr int kFs = 512;        // feature rows per CTA
 constexpr int kSlab = 128;      // feature rows per slab (one M = 128 tile)
 constexpr int kNs = kFs / kSlab;
-constexpr int kStages = 2;
-constexpr int kTeam = 256;      // compute threads: warps 2-9
-constexpr int kThreads = 64 + kTeam;
-constexpr uint32_t kSw128 = 2, kSw64 = 4, kSw32 = 6;  // descriptor swizzle modes
+constexpr int kStages = 3;      // Q, K, V tiles
+constexpr int kNQ = 3;          // Fq ring
+constexpr int kNP = 4;          // partial ring of the reduction through L2
+constexpr int kSTT = 256;       // state team: warps 2-9
+constexpr int kQ1T = 128;       // query team: warps 10-13
+constexpr int kQ2T = 128;       // output team: warps 14-17
+constexpr int kQ1W0 = (64 + kSTT) / 32;
+constexpr int kQ2W0 = kQ1W0 + kQ1T / 32;
+constexpr int kDW = kQ2W0 + kQ2T / 32;           // decay warp
+constexpr int kThreads = (kDW + 1) * 32;
+constexpr uint32_t kSw128 = 2, kSw64 = 4;        // descriptor swizzle modes
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kHalf1 = 16u << 16;           // lane offset of the second M = 64 tile
+constexpr uint32_t kBarQ2 = 1;                   // named barrier of the output team
+constexpr size_t kCounterStride = 64;            // bytes of reduction counters per head
+static_assert((2 * kNP + 1) * 4 <= kCounterStride, "counters of a head");
 
 template <int D>
 struct Cfg {
-    static constexpr int R = D * D / kFs;              // CTAs per head
-    static constexpr int ROWS = kC / R;                // output rows owned per CTA
-    static constexpr uint32_t RB = D * 2;              // bytes per bf16 row of q/k/v/hb
+    static constexpr int R = D * D / kFs;          // CTAs per head
+    static constexpr int ROWS = kC / R;            // output rows owned per CTA
+    static constexpr int NA = kFs / D;             // values of a per CTA
+    static constexpr uint32_t RB = D * 2;          // bytes per bf16 row of q/k/v/hb
     static constexpr uint32_t SW = RB == 128 ? kSw128 : kSw64;
-    static constexpr uint32_t SBO = 8 * RB;            // 8-row swizzle atom
-    static constexpr uint32_t TILE = kC * RB;          // q/k/v tile
-    static constexpr uint32_t STAGE = 3 * TILE;
-    static constexpr int PR = D + 4;                   // padded row (floats) of a partial
-    // shared memory map
+    static constexpr uint32_t SBO = 8 * RB;        // 8-row swizzle atom
+    static constexpr uint32_t TILE = kC * RB;      // q/k/v tile
+    static constexpr uint32_t STAGE = 3 * TILE;    // Q | K | V
+    static constexpr uint32_t HBT = kSlab * RB;    // hb tile of one slab
+    static constexpr int NT = D + 8;               // readout columns: T, Tn, zeros
+    static constexpr int PR = D + 4;               // padded partial row (floats)
+    static constexpr bool GLOBAL = D == 64;        // reduction through L2 (no cluster)
+    // shared memory map (bytes from a 1024-aligned base)
     static constexpr uint32_t OFF_STAGE = 0;
-    static constexpr uint32_t OFF_P = OFF_STAGE + kStages * STAGE;       // 64 x 64 bf16
-    static constexpr uint32_t OFF_FK = OFF_P + 8192;                      // 2 x 16 KiB
-    static constexpr uint32_t OFF_FQ = OFF_FK + 2 * 16384;                // 2 x 16 KiB
-    static constexpr uint32_t OFF_HB = OFF_FQ + 2 * 16384;                // 2 x 128 rows
-    // z entering the chunk, one 128-row tile per buffer in hb's layout with z in
-    // column 0 and zeros elsewhere: hb and zb form one B operand of 2 D columns
-    // (two MN atoms LBO_HZ bytes apart), so T and Tn come from one product
-    static constexpr uint32_t OFF_ZB = OFF_HB + 2 * kSlab * RB;           // 2 x 128 rows
-    static constexpr uint32_t LBO_HZ = OFF_ZB - OFF_HB;
-    static constexpr uint32_t OFF_ONES = OFF_ZB + 2 * kSlab * RB;         // 64 x 32 B
-    static constexpr uint32_t OFF_PART = OFF_ONES + 2048;                 // 2 x 64 x PR fp32
-    static constexpr uint32_t OFF_RES = OFF_PART + 2 * kC * PR * 4;       // ROWS x PR fp32
-    static constexpr uint32_t OFF_MISC = (OFF_RES + ROWS * PR * 4 + 1023) / 1024 * 1024;
+    static constexpr uint32_t OFF_HB = kStages * STAGE;                 // kNs x 128 rows
+    // z of slab s in logical 16-byte chunk s of each row: the readout's
+    // descriptor for slab s starts its second N atom 16 s bytes in
+    static constexpr uint32_t OFF_ZB = OFF_HB + kNs * HBT;              // 128 rows
+    static constexpr uint32_t OFF_FQ = OFF_ZB + HBT;                    // kNQ x 16 KiB
+    static constexpr uint32_t OFF_P = OFF_FQ + kNQ * 16384;             // 64 x 64 bf16
+    static constexpr uint32_t OFF_PART = OFF_P + 8192;                  // 2 x 64 x PR (cluster only)
+    static constexpr uint32_t OFF_RES = OFF_PART + (GLOBAL ? 0 : 2 * kC * PR * 4);  // ROWS x PR
+    static constexpr uint32_t OFF_WK = (OFF_RES + ROWS * PR * 4 + 15) / 16 * 16;      // 2 x NA x 32
+    static constexpr uint32_t OFF_MISC = (OFF_WK + 2 * NA * 32 * 4 + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM = OFF_MISC + 2048 + 1024;
-    // tensor memory columns
-    static constexpr uint32_t COL_H = 0;                   // kNs x D   h    (M = 128)
-    static constexpr uint32_t COL_Z = COL_H + kNs * D;     // kNs x 16  z    (M = 128)
-    static constexpr uint32_t COL_S = COL_Z + kNs * 16;    // 64: S, then Y = P V (M = 64)
-    static constexpr uint32_t COL_T = COL_S + 64;          // 2 D: partial readout [T | Tn 0...] (M = 64)
-    static constexpr uint32_t COL_TN = COL_T + D;          // Tn: first column of the second half
-    static_assert(COL_T + 2 * D <= 512, "TMEM budget");
+    // tensor memory columns.  The readout and S are M = 64 accumulators
+    // sharing columns: the readout in lanes 0-15 of each quarter, S in lanes
+    // 16-31 (the second M = 64 tile).
+    static constexpr uint32_t COL_H = 0;                  // kNs x D    h            (M = 128)
+    static constexpr uint32_t COL_FK = kNs * D;           // kNs x 32   Fk^T ring    (M = 128)
+    static constexpr uint32_t COL_T = COL_FK + kNs * 32;  // NT         [T | Tn]     (M = 64, lanes 0-15)
+    static constexpr uint32_t COL_S = COL_T;              // 64         S            (M = 64, lanes 16-31)
+    static_assert(COL_T + NT <= 512 && COL_S + 64 <= 512, "TMEM budget");
     static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(OFF_HB % 1024 == 0 && OFF_ZB % 1024 == 0 && OFF_FQ % 1024 == 0 && OFF_P % 1024 == 0,
+                  "swizzle atoms");
 };
 
 struct Misc {
-    float acs2[kC];
-    float vfac[kC];  // value factor dt_j of the chunk's tokens (value discretisation)
-    float rsum[2][kC];
-    float Dh[64];
-    float wtot[2];
+    float acs2[2][kC];   // chunk-local cumsum per chunk parity (decay warp -> query team)
+    float vfac[kC];      // value factors dt_j of the decay warp's current chunk
+    float rsum[kC];      // row sums of P (chunks whose quadratic part this CTA adds)
+    float Dh[64];        // D of the head
+    float lam2[2];       // chunk total per chunk parity (state team reads it)
     uint64_t stage_full[kStages], stage_empty[kStages];
-    uint64_t s_full, p_full, y_free, chunk_done;
-    uint64_t slab_full[2], slab_done[2];
+    uint64_t decay_ready[2], decay_free[2];
+    uint64_t st_ready[kNs], slab_done[kNs], q_ready[kNQ];
+    uint64_t t_full, t_free, s_full, p_full;
     uint64_t ready[2], consumed[2];
     uint64_t drain;
     uint32_t tmem_base;
@@ -112,21 +141,62 @@ __device__ __forceinline__ float softplus_f(float x) {
 __device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
-__device__ __forceinline__ float bf16_at(const uint8_t *p) {
-    return __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(p) << 16);
+__device__ __forceinline__ uint32_t bf16_bits_at(const uint8_t *p) {
+    return (uint32_t)*reinterpret_cast<const uint16_t *>(p);
 }
+__device__ __forceinline__ float bf16_at(const uint8_t *p) { return __uint_as_float(bf16_bits_at(p) << 16); }
 template <uint32_t RB>
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t ch) {
     if constexpr (RB == 128) return sw128_chunk(row, ch);
     else return sw64_chunk(row, ch);
 }
+// byte offset of element `col` of `row` in a swizzled bf16 tile
+template <uint32_t RB>
+__device__ __forceinline__ uint32_t swz_elem(uint32_t row, uint32_t col) {
+    return swz<RB>(row, col >> 3) + (col & 7u) * 2u;
+}
 
-__device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where) {
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Waits until the counter reaches `target`; gives up (false) on a raised
+// abort flag (this CTA's or the head's) or after limit_ns of wall time.
+__device__ bool counter_wait(const uint32_t *cnt, uint32_t target, const volatile int *abort,
+                             const uint32_t *head_abort, unsigned long long limit_ns) {
+    if (ld_acquire_gpu(cnt) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (ld_acquire_gpu(cnt) >= target) return true;
+        if ((it & 63u) == 63u) {
+            if (*abort || ld_acquire_gpu(head_abort)) return false;
+            if (globaltimer_ns() - t0 > limit_ns) return false;
+        }
+        __nanosleep(32);
+    }
+}
+
+// Records a timeout (the first one wins) and raises the abort flags: this
+// CTA's, and every other CTA's of the head (the cluster's through
+// distributed shared memory, or the head's flag in global memory).
+template <bool kGlobal, int R>
+__device__ void raise_timeout(Misc *misc, DeviceStatus *status, int where, uint32_t *head_abort) {
     if (status) {
         atomicCAS(&status->code, 0, (int)SSD_ERR_TIMEOUT);
         atomicCAS(&status->detail, 0, where);
     }
-    *reinterpret_cast<volatile int *>(&misc->abort_flag) = 1;
+    if constexpr (kGlobal) {
+        *reinterpret_cast<volatile int *>(&misc->abort_flag) = 1;
+        atomicExch(head_abort, 1u);
+    } else {
+        const uint32_t a = smem_u32(&misc->abort_flag);
+        for (int r = 0; r < R; ++r) st_dsmem_u32(mapa_shared(a, (uint32_t)r), 1u);
+        fence_acq_rel_cluster();
+    }
 }
 
 // kState: the call carries a state in or out (a separate instantiation, so
@@ -135,13 +205,17 @@ template <int D, bool kState>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __nv_bfloat16 *__restrict__ vglob,
-                 __nv_bfloat16 *__restrict__ out,
-                 const float *__restrict__ dt_p, const float *__restrict__ A_log,
-                 const float *__restrict__ dt_bias, const float *__restrict__ Dres,
-                 const float *__restrict__ log_decay, int value_dt, int H, int N,
-                 int normalize, const float *__restrict__ h0, const float *__restrict__ z0,
-                 float *__restrict__ h_out, float *__restrict__ z_out, DeviceStatus *status) {
+                 __nv_bfloat16 *__restrict__ out, const float *__restrict__ dt_p,
+                 const float *__restrict__ A_log, const float *__restrict__ dt_bias,
+                 const float *__restrict__ Dres, const float *__restrict__ log_decay, int value_dt,
+                 int H, int N, int normalize, const float *__restrict__ h0, const float *__restrict__ z0,
+                 float *__restrict__ h_out, float *__restrict__ z_out, DeviceStatus *status,
+                 uint32_t *__restrict__ counters, float *__restrict__ gpart, int dbg_skip,
+                 unsigned long long wait_ns) {
     using K = Cfg<D>;
+    constexpr int R = K::R;
+    constexpr uint32_t RB = K::RB;
+    constexpr bool GL = K::GLOBAL;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -150,14 +224,16 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t sbase = smem_u32(smem);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const uint32_t rank = cluster_ctarank();
-    const int bh = blockIdx.x / K::R, h = bh % H;
+    const uint32_t rank = GL ? (uint32_t)(blockIdx.x % R) : cluster_ctarank();
+    const int bh = blockIdx.x / R, h = bh % H;
     const int nc = N / kC;
     const int row0 = bh * N;
-    // a carried state enters before chunk 0 exactly as the state of a previous
-    // chunk does; the normaliser state is tracked when it is used or asked for
+    // a carried state enters before chunk 0 exactly as the state of a previous chunk does
     const bool carry = kState && (h0 != nullptr || z0 != nullptr);
-    const bool track_z = normalize || (kState && (z0 != nullptr || z_out != nullptr));
+    // per head: ready[kNP], consumed[kNP] (per slot of the partial ring), abort
+    uint32_t *hcnt = GL ? counters + bh * (kCounterStride / 4) : nullptr;
+    uint32_t *head_abort = GL ? hcnt + 2 * kNP : nullptr;
+    auto timeout = [&](int where) { raise_timeout<GL, R>(misc, status, where, head_abort); };
 
     if (tid == 0) {
         if (blockIdx.x == 0 && status) {
@@ -166,19 +242,24 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&misc->stage_full[i], 1);
-            mbar_init(&misc->stage_empty[i], 1);
+            mbar_init(&misc->stage_empty[i], 1 + kSTT + kQ1T + 32);
         }
-        mbar_init(&misc->s_full, 1);
-        mbar_init(&misc->p_full, kTeam);
-        mbar_init(&misc->y_free, kTeam);
-        mbar_init(&misc->chunk_done, 1);
-        mbar_init(&misc->drain, 1);
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&misc->slab_full[b], kTeam);
-            mbar_init(&misc->slab_done[b], 1);
-            mbar_init(&misc->ready[b], K::R);
-            mbar_init(&misc->consumed[b], K::R);
+            mbar_init(&misc->decay_ready[b], 32);
+            mbar_init(&misc->decay_free[b], kSTT + kQ1T);
+            mbar_init(&misc->ready[b], R);
+            mbar_init(&misc->consumed[b], R);
         }
+        for (int s = 0; s < kNs; ++s) {
+            mbar_init(&misc->st_ready[s], kSTT / 2);
+            mbar_init(&misc->slab_done[s], 1);
+        }
+        for (int e = 0; e < kNQ; ++e) mbar_init(&misc->q_ready[e], kQ1T);
+        mbar_init(&misc->t_full, 1);
+        mbar_init(&misc->t_free, kQ2T);
+        mbar_init(&misc->s_full, 1);
+        mbar_init(&misc->p_full, kQ1T);
+        mbar_init(&misc->drain, 1);
         misc->abort_flag = 0;
         fence_mbar_init();
     }
@@ -186,24 +267,15 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_alloc(&misc->tmem_base, 512);
         tmem_relinquish();
     }
-    // zb tiles: zero once; only column 0 of each row is written later
-    for (int i = tid; i < (int)(2 * kSlab * K::RB / 16); i += kThreads)
-        reinterpret_cast<uint4 *>(smem + K::OFF_ZB)[i] = make_uint4(0u, 0u, 0u, 0u);
-    // constant B operand: [1, 0, ..., 0] per token (64 rows x 16 bf16, 32B swizzle)
-    for (int i = tid; i < kC * 2; i += kThreads) {
-        const int r = i >> 1, ch = i & 1;
-        *reinterpret_cast<uint4 *>(smem + K::OFF_ONES + sw32_chunk(r, ch)) =
-            make_uint4(ch == 0 ? 0x3F80u : 0u, 0u, 0u, 0u);
-    }
     if (tid < D) misc->Dh[tid] = Dres ? Dres[h * D + tid] : 0.0f;
-    fence_proxy_async_smem();
     tc_fence_before();
-    cluster_sync_all();  // every CTA's barriers exist before any remote arrive
+    if constexpr (GL) __syncthreads();
+    else cluster_sync_all();  // every CTA's barriers exist before any remote access
     tc_fence_after();
     const uint32_t tmem = misc->tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
@@ -212,8 +284,8 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             for (int c = 0; c < nc; ++c) {
                 const int st = c % kStages;
                 if (c >= kStages &&
-                    !mbar_wait_abortable(&misc->stage_empty[st], ((c / kStages) - 1) & 1, abort_flag)) {
-                    raise_timeout(misc, status, 10);
+                    !mbar_wait_abortable(&misc->stage_empty[st], ((c / kStages) - 1) & 1, abort_flag, wait_ns)) {
+                    timeout(10);
                     break;
                 }
                 uint8_t *dst = smem + K::OFF_STAGE + st * K::STAGE;
@@ -229,167 +301,345 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_wait_bounded(&misc->stage_full[c % kStages], (c / kStages) & 1);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
+            constexpr uint32_t idBuild = make_idesc_bf16(128, D, 0, 1);
+            constexpr uint32_t idRead = make_idesc_bf16(64, K::NT, 0, 1);
             constexpr uint32_t idS = make_idesc_bf16(64, 64, 0, 0);
             constexpr uint32_t idPV = make_idesc_bf16(64, D, 0, 1);
-            constexpr uint32_t idU = make_idesc_bf16(128, D, 1, 1);
-            constexpr uint32_t idZ = make_idesc_bf16(128, 16, 1, 1);
-            constexpr uint32_t idT = make_idesc_bf16(64, D, 0, 1);
-            constexpr uint32_t idT2 = make_idesc_bf16(64, 2 * D, 0, 1);  // [T | Tn] in one product
-            uint32_t slab_uses[2] = {0, 0};
+            constexpr uint64_t kStepRows = (16 * RB) >> 4;  // descriptor units per 16 rows
+            const uint64_t dP = make_sdesc(sbase + K::OFF_P, 16, 1024, kSw128);
+            const uint64_t dFq = make_sdesc(sbase + K::OFF_FQ, 16, 1024, kSw128);
+            const uint32_t tT = tmem + K::COL_T, tS = tmem + kHalf1 + K::COL_S;
             bool ok = true;
+            int kown = 0;
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                ok = ok && mbar_wait_abortable(bar, parity, abort_flag, wait_ns);
+                return ok;
+            };
             for (int c = 0; ok && c < nc; ++c) {
-                const int st = c % kStages;
-                const uint32_t aQ = sbase + K::OFF_STAGE + st * K::STAGE;
-                const uint32_t aK = aQ + K::TILE, aV = aK + K::TILE;
-                if (!(ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag))) break;
-                if (c >= 1 && !(ok = mbar_wait_abortable(&misc->y_free, (c - 1) & 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    mma_bf16(tmem + K::COL_S, make_sdesc(aQ + ks * 32, 16, K::SBO, K::SW),
-                             make_sdesc(aK + ks * 32, 16, K::SBO, K::SW), idS, ks > 0);
-                mma_commit(&misc->s_full);
-                if (!(ok = mbar_wait_abortable(&misc->p_full, c & 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < kC / 16; ++ks)
-                    mma_bf16(tmem + K::COL_S, make_sdesc(sbase + K::OFF_P + ks * 32, 16, 1024, kSw128),
-                             make_sdesc(aV + ks * 16 * K::RB, 16, K::SBO, K::SW), idPV, ks > 0);
-                for (int sl = 0; sl < kNs; ++sl) {
-                    const int b = sl & 1;
-                    if (!(ok = mbar_wait_abortable(&misc->slab_full[b], slab_uses[b] & 1, abort_flag))) break;
-                    ++slab_uses[b];
+                const int st = c % kStages, c3 = c % kNQ;
+                const bool has_read = c >= 1 || carry;
+                const bool owner = (c % R) == (int)rank;
+                const uint32_t acc = (c >= 1 || carry) ? 1u : 0u;
+                if (!wait(&misc->stage_full[st], (c / kStages) & 1)) break;
+                const uint32_t soff = K::OFF_STAGE + st * K::STAGE;
+                const uint64_t dQ = make_sdesc(sbase + soff, 16, K::SBO, K::SW);
+                const uint64_t dK = make_sdesc(sbase + soff + K::TILE, 16, K::SBO, K::SW);
+                const uint64_t dV = make_sdesc(sbase + soff + 2 * K::TILE, 16, K::SBO, K::SW);
+                if (owner) {  // S = Q K^T into the second M = 64 tile of the readout's columns
                     tc_fence_after();
-                    const uint32_t fkA = sbase + K::OFF_FK + b * 16384;
-                    const uint32_t fqA = sbase + K::OFF_FQ + b * 16384;
-                    // h_slab += Fk^T V  (A: features x tokens, MN-major, two 64-feature groups)
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        mma_bf16(tS, dQ + ks * 2, dK + ks * 2, idS, ks > 0 ? 1u : 0u);
+                    mma_commit(&misc->s_full);
+                }
+                // state builds of the four slabs (they do not touch the readout's columns)
+#pragma unroll
+                for (int s = 0; s < kNs; ++s) {
+                    if (!wait(&misc->st_ready[s], c & 1)) break;
+                    tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < kC / 16; ++ks)
-                        mma_bf16(tmem + K::COL_H + sl * D, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
-                                 make_sdesc(aV + ks * 16 * K::RB, 16, K::SBO, K::SW), idU,
-                                 (c > 0 || carry || ks > 0));
-                    if (track_z) {
-#pragma unroll
-                        for (int ks = 0; ks < kC / 16; ++ks)
-                            mma_bf16(tmem + K::COL_Z + sl * 16, make_sdesc(fkA + ks * 2048, 8192, 1024, kSw128),
-                                     make_sdesc(sbase + K::OFF_ONES + ks * 512, 16, 256, kSw32), idZ,
-                                     (c > 0 || carry || ks > 0));
-                    }
-                    if (c >= 1 || carry) {
-                        // [T | Tn] += Fq [hb | zb]   (A: tokens x features, K-major;
-                        // B: the hb and zb tiles as two MN atoms)
-                        const uint32_t hbB = sbase + K::OFF_HB + b * kSlab * K::RB;
-#pragma unroll
-                        for (int ks = 0; ks < kSlab / 16; ++ks) {
-                            const uint64_t adesc =
-                                make_sdesc(fqA + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kSw128);
-                            mma_bf16(tmem + K::COL_T, adesc,
-                                     make_sdesc(hbB + ks * 16 * K::RB, K::LBO_HZ, K::SBO, K::SW),
-                                     normalize ? idT2 : idT, (sl > 0 || ks > 0));
-                        }
-                    }
-                    mma_commit(&misc->slab_done[b]);
+                        mma_bf16_ts(tmem + K::COL_H + s * D, tmem + K::COL_FK + s * 32 + ks * 8, dV + ks * kStepRows,
+                                    idBuild, (acc | (ks > 0 ? 1u : 0u)));
                 }
                 if (!ok) break;
-                mma_commit(&misc->chunk_done);
+                if (c >= 1 && !wait(&misc->t_free, (c - 1) & 1)) break;  // previous partial read
+                // readouts, slab by slab; each slab's buffers are released by slab_done
+#pragma unroll
+                for (int s = 0; s < kNs; ++s) {
+                    const int it = 4 * c + s, e = (c3 + s) % kNQ;
+                    if (!wait(&misc->q_ready[e], (it / kNQ) & 1)) break;
+                    tc_fence_after();
+                    if (has_read) {
+                        const uint64_t dA = dFq + (((uint32_t)e * 16384u) >> 4);
+                        const uint64_t dB = make_sdesc(sbase + K::OFF_HB + s * K::HBT,
+                                                       (K::OFF_ZB + 16u * s) - (K::OFF_HB + s * K::HBT), K::SBO, K::SW);
+#pragma unroll
+                        for (int ks = 0; ks < kSlab / 16; ++ks)
+                            mma_bf16(tT, dA + (((ks >> 2) * 8192u + (ks & 3) * 32u) >> 4), dB + ks * kStepRows, idRead,
+                                     (s > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&misc->slab_done[s]);
+                    if (s == 1 && owner) {
+                        if (!wait(&misc->p_full, kown & 1)) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < kC / 16; ++ks)
+                            mma_bf16(tT, dP + ks * 2, dV + ks * kStepRows, idPV, (has_read || ks > 0) ? 1u : 0u);
+                        ++kown;
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&misc->t_full);
+                mma_commit(&misc->stage_empty[st]);
             }
             if (!ok) {
-                raise_timeout(misc, status, 20);
-                // matrix products still in flight finish before TMEM is released (bounded)
+                timeout(20);
+                // products still in flight finish before TMEM is released (bounded)
                 mma_commit(&misc->drain);
                 mbar_wait_bounded(&misc->drain, 0);
             }
         }
-    } else {
-        // ------------------------------------------------------ compute team
-        const int ct = tid - 64;                    // 0..255
-        const int g = warp & 3;                     // TMEM lane quarter
-        const int hf = (warp - 2) >> 2;             // which half of the columns
-        const uint32_t lane_off = (uint32_t)(g * 32) << 16;
-        const int frow = g * 32 + lane;             // feature row of a slab (M = 128 layout)
-        const int mrow = g * 16 + lane;             // chunk row (M = 64 layout, lane < 16)
-        const bool mrow_ok = lane < 16;
-        const bool own_row = mrow_ok && mrow / K::ROWS == (int)rank;
-        const float A2 = log_decay ? 0.0f : -expf(A_log[h]) * kLog2e;
-        const float bias = dt_bias ? dt_bias[h] : 0.0f;  // given whenever dt is used
-        const bool elected = ct == 0;
-        const int tok = ct & 63, q4 = ct >> 6;      // feature generation: token, 32-feature part
-        uint32_t slab_uses[2] = {0, 0};
-        float *part0 = reinterpret_cast<float *>(smem + K::OFF_PART);
-        float *res = reinterpret_cast<float *>(smem + K::OFF_RES);
-
-        // per-token decay input: the dt projection, or the given log-decay (Algorithm 4)
-        const float *dsrc = log_decay ? log_decay : dt_p;
-        float dt_next = (ct < kC && nc > 0) ? dsrc[(size_t)row0 + ct] : 0.0f;
-        // the dt projection for the value factor, when it is not already dsrc
-        const bool vdt_own = value_dt && log_decay;
-        float vdt_next = (vdt_own && ct < kC && nc > 0) ? dt_p[(size_t)row0 + ct] : 0.0f;
-        bool failed = false;
-        // Own rows of chunk cc: sum the R partials (distributed shared memory),
-        // release them, then y = (Y + T) / (r + Tn) [+ D v].
-        static_assert(K::ROWS * (D / 8) <= kTeam, "one output item per thread");
-        auto reduce_output = [&](int cc) -> bool {
-            // this thread's output item and its residual input, fetched before the waits
-            const int o_rr = ct / (D / 8), o_ch = ct % (D / 8);
-            const bool o_live = ct < K::ROWS * (D / 8);
-            const size_t o_grow = (size_t)row0 + (size_t)cc * kC + rank * K::ROWS + o_rr;
-            uint4 vu = make_uint4(0u, 0u, 0u, 0u);
-            if (Dres && o_live) vu = __ldg(reinterpret_cast<const uint4 *>(vglob + o_grow * D + o_ch * 8));
-            const bool bad = !mbar_wait_cluster(&misc->ready[cc & 1], (cc >> 1) & 1, abort_flag);
-            if (named_bar_any(1, kTeam, bad)) {
-                if (elected) raise_timeout(misc, status, 34);
-                return false;
-            }
-            {
-                constexpr int NV = D / 4 + 1;  // float4 groups of a row, plus the normaliser
-                const uint32_t pb = smem_u32(part0 + (cc & 1) * kC * K::PR);
-                for (int it = ct; it < K::ROWS * NV; it += kTeam) {
-                    const int rr = it / NV, v = it % NV;
-                    const int row = rank * K::ROWS + rr;
-                    const uint32_t off = (uint32_t)(row * K::PR + (v < D / 4 ? v * 4 : D)) * 4u;
-                    // all R remote loads are issued before any is used, so their
-                    // latencies overlap
-                    if (v < D / 4) {
-                        float4 x[K::R];
+    } else if (warp < kQ1W0) {
+        // ------------------------------------------------------------ state team
+        const int q = warp & 3;                      // TMEM lane quarter
+        const int hh = (warp - 2) >> 2;              // slabs hh and hh + 2
+        const int L = q * 32 + lane;                 // lane of every slab
+        const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+        const int bcol = L % D;                      // b of this lane's features
+        const int lg = L / D;                        // a = rank NA + 4 lg + s
+        bool ok = true;
+        auto wait = [&](uint64_t *bar, uint32_t parity) {
+            ok = ok && mbar_wait_abortable(bar, parity, abort_flag, wait_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            return ok;
+        };
+        auto feature = [&](int s) -> size_t {  // global feature row of slab s
+            return (size_t)bh * D * D + (size_t)(rank * K::NA + 4 * lg + s) * D + bcol;
+        };
+        // z of this lane's features (slabs hh, hh + 2): the state entering the next chunk
+        float zr[2];
 #pragma unroll
-                        for (int r2 = 0; r2 < K::R; ++r2) x[r2] = ld_dsmem_f4(mapa_shared(pb + off, r2));
-                        float4 acc = x[0];
+        for (int si = 0; si < 2; ++si) zr[si] = (kState && z0) ? z0[feature(hh + 2 * si)] : 0.0f;
+        for (int c = 0; c < nc; ++c) {
+            const int st = c % kStages;
+            if (!wait(&misc->stage_full[st], (c / kStages) & 1)) break;
+            // k_jb of the chunk's 64 tokens, as bf16 pairs (j, j + 1)
+            const uint8_t *sK = smem + K::OFF_STAGE + st * K::STAGE + K::TILE;
+            uint32_t kp[32];
 #pragma unroll
-                        for (int r2 = 1; r2 < K::R; ++r2) {
-                            acc.x += x[r2].x;
-                            acc.y += x[r2].y;
-                            acc.z += x[r2].z;
-                            acc.w += x[r2].w;
+            for (int p = 0; p < 32; ++p)
+                kp[p] = bf16_bits_at(sK + swz_elem<RB>(2 * p, bcol)) | (bf16_bits_at(sK + swz_elem<RB>(2 * p + 1, bcol)) << 16);
+            mbar_arrive(&misc->stage_empty[st]);
+            if (!wait(&misc->decay_ready[c & 1], (c >> 1) & 1)) break;
+            const float dec = ex2_approx(misc->lam2[c & 1]);
+            const uint32_t *wk = reinterpret_cast<const uint32_t *>(smem + K::OFF_WK) + (c & 1) * K::NA * 32;
+#pragma unroll
+            for (int si = 0; si < 2; ++si) {
+                const int s = hh + 2 * si;
+                if (c >= 1 && !wait(&misc->slab_done[s], (c - 1) & 1)) break;
+                tc_fence_after();
+                // ---- the state entering the chunk -> hb, zb (bf16); the state *= 2^lam
+                if (c >= 1 || carry) {
+                    uint8_t *hb = smem + K::OFF_HB + s * K::HBT;
+#pragma unroll
+                    for (int half = 0; half < D / 32; ++half) {
+                        float hv[32];
+                        const uint32_t ta = tmem + lane_off + K::COL_H + s * D + 32 * half;
+                        if (c >= 1) {
+                            tmem_ld32(ta, hv);
+                            tmem_wait_ld();
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4) {
+                                const float4 x = h0 ? *reinterpret_cast<const float4 *>(h0 + feature(s) * D + 32 * half + j)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                                hv[j] = x.x;
+                                hv[j + 1] = x.y;
+                                hv[j + 2] = x.z;
+                                hv[j + 3] = x.w;
+                            }
                         }
-                        *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc;
-                    } else {
-                        float x[K::R];
 #pragma unroll
-                        for (int r2 = 0; r2 < K::R; ++r2) x[r2] = ld_dsmem_f1(mapa_shared(pb + off, r2));
-                        float acc = x[0];
+                        for (int ch = 0; ch < 4; ++ch)
+                            *reinterpret_cast<uint4 *>(hb + swz<RB>(L, 4 * half + ch)) =
+                                make_uint4(pack_bf16x2(hv[ch * 8], hv[ch * 8 + 1]), pack_bf16x2(hv[ch * 8 + 2], hv[ch * 8 + 3]),
+                                           pack_bf16x2(hv[ch * 8 + 4], hv[ch * 8 + 5]),
+                                           pack_bf16x2(hv[ch * 8 + 6], hv[ch * 8 + 7]));
+                        const float2 d2 = make_float2(dec, dec);
 #pragma unroll
-                        for (int r2 = 1; r2 < K::R; ++r2) acc += x[r2];
-                        res[rr * K::PR + D] = acc;
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 r2 = __fmul2_rn(make_float2(hv[e], hv[e + 1]), d2);
+                            hv[e] = r2.x;
+                            hv[e + 1] = r2.y;
+                        }
+                        tmem_st32(ta, hv);
+                    }
+                    *reinterpret_cast<uint4 *>(smem + K::OFF_ZB + swz<RB>(L, s)) =
+                        make_uint4(pack_bf16x2(zr[si], 0.0f), 0u, 0u, 0u);
+                }
+                // ---- Fk^T row of feature (a, b) over the 64 tokens, and z
+                {
+                    const uint4 *wr = reinterpret_cast<const uint4 *>(wk + (4 * lg + s) * 32);
+                    float2 zs = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int th = 0; th < 2; ++th) {
+                        uint32_t fk[16];
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4) {
+                            const uint4 w = wr[4 * th + v4];
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                fk[4 * v4 + e] = mul_bf16x2(ww[e], kp[16 * th + 4 * v4 + e]);
+                                zs = __fadd2_rn(zs, bf2_to_f2(fk[4 * v4 + e]));
+                            }
+                        }
+                        tmem_st16(tmem + lane_off + K::COL_FK + s * 32 + th * 16, fk);
+                    }
+                    zr[si] = fmaf(zr[si], dec, zs.x + zs.y);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                fence_proxy_async_smem();
+                if (4 * c + s != dbg_skip) mbar_arrive(&misc->st_ready[s]);
+            }
+            if (!ok) break;
+            mbar_arrive(&misc->decay_free[c & 1]);
+        }
+        // the state after the last token: TMEM holds h once the last products are done
+        if (kState && ok && (h_out || z_out)) {
+#pragma unroll
+            for (int si = 0; si < 2; ++si) {
+                const int s = hh + 2 * si;
+                if (!wait(&misc->slab_done[s], (nc - 1) & 1)) break;
+                tc_fence_after();
+                if (h_out) {
+#pragma unroll
+                    for (int half = 0; half < D / 32; ++half) {
+                        float hv[32];
+                        tmem_ld32(tmem + lane_off + K::COL_H + s * D + 32 * half, hv);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4 *>(h_out + feature(s) * D + 32 * half + j) =
+                                make_float4(hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
                     }
                 }
+                if (z_out) z_out[feature(s)] = zr[si];
             }
-            named_bar_sync(1, kTeam);
-            if (ct < K::R) {
-                fence_acq_rel_cluster();
-                mbar_arrive_cluster(mapa_shared(smem_u32(&misc->consumed[cc & 1]), ct));
+        }
+    } else if (warp < kQ2W0) {
+        // ------------------------------------------------------------ query team
+        const int q1 = tid - kQ1W0 * 32;             // 0..127
+        const int qq = warp & 3;                     // TMEM lane quarter
+        const uint32_t lane_off = (uint32_t)(qq * 32) << 16;
+        // Fq: thread q1 writes row tk of the 64-feature atom `at` of every slab
+        const int tk = q1 & 63, at = q1 >> 6;
+        bool ok = true;
+        int kown = 0;
+        auto wait = [&](uint64_t *bar, uint32_t parity) {
+            ok = ok && mbar_wait_abortable(bar, parity, abort_flag, wait_ns);
+            ok = __all_sync(0xffffffffu, ok);
+            return ok;
+        };
+        for (int c = 0; c < nc; ++c) {
+            const int st = c % kStages, c3 = c % kNQ;
+            const bool owner = (c % R) == (int)rank;
+            if (!wait(&misc->stage_full[st], (c / kStages) & 1)) break;
+            if (!wait(&misc->decay_ready[c & 1], (c >> 1) & 1)) break;
+            const uint8_t *sQ = smem + K::OFF_STAGE + st * K::STAGE;
+            const float *acs = misc->acs2[c & 1];
+            // this thread's query row (bf16 pairs) and 2^acs of its token
+            uint32_t qr[D / 2];
+#pragma unroll
+            for (int ch = 0; ch < D / 8; ++ch) {
+                const uint4 x = *reinterpret_cast<const uint4 *>(sQ + swz<RB>(tk, ch));
+                qr[4 * ch] = x.x;
+                qr[4 * ch + 1] = x.y;
+                qr[4 * ch + 2] = x.z;
+                qr[4 * ch + 3] = x.w;
             }
-            if (o_live) {
-                const int rr = o_rr, ch = o_ch;
-                const size_t grow = o_grow;
-                const float *rrow = res + rr * K::PR;
+            const float ut = ex2_approx(acs[tk]);
+            for (int s = 0; s < kNs; ++s) {
+                if (s == 2 && owner) {
+                    // ---- quadratic part of the chunk: P = S^2 2^(acs_i - acs_j) [i >= j]
+                    if (!wait(&misc->s_full, kown & 1)) break;
+                    tc_fence_after();
+                    float sv0[32], sv1[32];
+                    tmem_ld32(tmem + lane_off + K::COL_S, sv0);
+                    tmem_ld32(tmem + lane_off + K::COL_S + 32, sv1);
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    if (lane >= 16) {  // rows of the second M = 64 tile
+                        const int i = 16 * qq + lane - 16;
+                        const float ai = acs[i];
+                        float rs = 0.0f;
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                const int j = ch * 8 + e;
+                                const float x0 = j < 32 ? sv0[j & 31] : sv1[j & 31];
+                                const float x1 = j + 1 < 32 ? sv0[(j + 1) & 31] : sv1[(j + 1) & 31];
+                                float p0 = x0 * x0 * ex2_approx(ai - acs[j]);
+                                float p1 = x1 * x1 * ex2_approx(ai - acs[j + 1]);
+                                if (j > i) p0 = 0.0f;
+                                if (j + 1 > i) p1 = 0.0f;
+                                rs += p0 + p1;
+                                pk[e >> 1] = pack_bf16x2(p0, p1);
+                            }
+                            *reinterpret_cast<uint4 *>(smem + K::OFF_P + sw128_chunk(i, ch)) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                        misc->rsum[i] = rs;
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&misc->p_full);
+                    ++kown;
+                }
+                const int it = 4 * c + s, e = (c3 + s) % kNQ;
+                // the Fq buffer's previous user (iteration it - kNQ) has been read
+                if (it >= kNQ && !wait(&misc->slab_done[(it - kNQ) & 3], ((it - kNQ) >> 2) & 1)) break;
+                // ---- Fq slab s (K-major, 64 x 128): feature k of the slab is
+                // (a = rank NA + 4 (k / D) + s, b = k % D); this thread writes row tk
+                // of atom at, i.e. k = 64 at + kk for kk in [0, 64)
+                constexpr int NAA = 64 / D;  // values of a in one 64-feature atom
+                uint32_t ca[NAA];
+#pragma unroll
+                for (int ag = 0; ag < NAA; ++ag) {
+                    const int av = rank * K::NA + 4 * (NAA * at + ag) + s;
+                    const float cv = ut * bf16_at(sQ + swz_elem<RB>(tk, av));
+                    ca[ag] = pack_bf16x2(cv, cv);
+                }
+                uint8_t *fq = smem + K::OFF_FQ + e * 16384 + at * 8192;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const int kk = 8 * ch;
+                    const uint32_t cp = ca[kk / D];
+                    const int qp = (kk % D) / 2;  // first bf16 pair of q_ib
+                    *reinterpret_cast<uint4 *>(fq + sw128_chunk(tk, ch)) =
+                        make_uint4(mul_bf16x2(cp, qr[qp]), mul_bf16x2(cp, qr[qp + 1]), mul_bf16x2(cp, qr[qp + 2]),
+                                   mul_bf16x2(cp, qr[qp + 3]));
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&misc->q_ready[e]);
+            }
+            if (!ok) break;
+            mbar_arrive(&misc->decay_free[c & 1]);
+            mbar_arrive(&misc->stage_empty[st]);
+        }
+        if (!ok) timeout(30);
+    } else if (warp < kDW) {
+        // ------------------------------------------------------------ output team
+        const int q2 = tid - kQ2W0 * 32;             // 0..127
+        const int qq = warp & 3;
+        const uint32_t lane_off = (uint32_t)(qq * 32) << 16;
+        const bool row_t = lane < 16;                // holds a row of the M = 64 readout
+        const int row = 16 * qq + lane;
+        float *res = reinterpret_cast<float *>(smem + K::OFF_RES);
+        bool failed = false;
+        int kown = 0;
+        auto team_ok = [&](bool good) { return !named_bar_any(kBarQ2, kQ2T, !good); };
+        static_assert(K::ROWS * (D / 8) <= kQ2T, "one output item per thread");
+        constexpr int NV = D / 4 + 1;  // float4 groups of a row, plus the normaliser
+        // y of chunk cc from the summed rows in res: y = T / Tn [+ D v]
+        auto write_output = [&](int cc) {
+            const int o_rr = q2 / (D / 8), o_ch = q2 % (D / 8);
+            if (q2 < K::ROWS * (D / 8)) {
+                const size_t o_grow = (size_t)row0 + (size_t)cc * kC + rank * K::ROWS + o_rr;
+                uint4 vu = make_uint4(0u, 0u, 0u, 0u);
+                if (Dres) vu = __ldg(reinterpret_cast<const uint4 *>(vglob + o_grow * D + o_ch * 8));
+                const float *rrow = res + o_rr * K::PR;
                 const float inv = normalize ? 1.0f / rrow[D] : 1.0f;
                 const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const int c2 = ch * 8 + 2 * e;
+                    const int c2 = o_ch * 8 + 2 * e;
                     float y0 = rrow[c2] * inv, y1 = rrow[c2 + 1] * inv;
                     if (Dres) {
                         const float2 vf = bf2_to_f2(vw[e]);
@@ -398,46 +648,234 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     w[e] = pack_bf16x2(y0, y1);
                 }
-                *reinterpret_cast<uint4 *>(out + grow * D + ch * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(out + o_grow * D + o_ch * 8) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            named_bar_sync(1, kTeam);  // res is reused by the next reduction
-            return true;
         };
+        // ---- this CTA's partial [T | Tn] of chunk c, read from TMEM into
+        // `dst_row` (this thread's row); releases the readout's columns
+        auto drain = [&](int c, float *dst_row, bool owner) {
+            const bool has_read = c >= 1 || carry;
+            const float rs = (owner && row_t) ? misc->rsum[row] : 0.0f;
+#pragma unroll
+            for (int half = 0; half < D / 32; ++half) {
+                float tv[32];
+                tmem_ld32(tmem + lane_off + K::COL_T + 32 * half, tv);
+                tmem_wait_ld();
+                if (row_t)
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4 *>(dst_row + 32 * half + e) =
+                            (has_read || owner) ? make_float4(tv[e], tv[e + 1], tv[e + 2], tv[e + 3])
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            const float tn = tmem_ld1(tmem + lane_off + K::COL_T + D);
+            tmem_wait_ld();
+            if (row_t) dst_row[D] = (has_read ? tn : 0.0f) + rs;
+            tc_fence_before();
+            mbar_arrive(&misc->t_free);
+        };
+        if constexpr (GL) {
+            // reduction through L2: partials[bh][c % kNP][rank][row][PR].  Per
+            // slot of the ring, ready counts the CTAs' published partials and
+            // consumed their finished reductions; each use of a slot adds
+            // exactly R to both, because a slot is rewritten only after all R
+            // CTAs have reduced its previous chunk (CTAs may run ahead of one
+            // another by up to kNP chunks)
+            uint32_t *ready_cnt = hcnt, *consumed_cnt = hcnt + kNP;
+            float *hpart = gpart + (size_t)bh * kNP * R * kC * K::PR;
+            for (int c = 0; c <= nc; ++c) {
+                if (c < nc) {
+                    const bool owner = (c % R) == (int)rank;
+                    bool good = mbar_wait_abortable(&misc->t_full, c & 1, abort_flag, wait_ns);
+                    if (owner) good = good && mbar_wait_abortable(&misc->p_full, kown & 1, abort_flag, wait_ns);
+                    // every CTA has reduced the slot's previous chunk, c - kNP
+                    if (c >= kNP && q2 == 0)
+                        good = good && counter_wait(consumed_cnt + c % kNP, (uint32_t)(R * (c / kNP)), abort_flag,
+                                                    head_abort, wait_ns);
+                    if (!team_ok(good)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    drain(c, hpart + (((size_t)(c % kNP) * R + rank) * kC + row) * K::PR, owner);
+                    if (owner) ++kown;
+                    __threadfence();
+                    named_bar_sync(kBarQ2, kQ2T);
+                    if (q2 == 0) red_release_gpu_add(ready_cnt + c % kNP, 1u);
+                }
+                if (c >= 1) {
+                    // ---- own rows of chunk cr: sum the R partials
+                    const int cr = c - 1;
+                    bool good = true;
+                    if (q2 == 0)
+                        good = counter_wait(ready_cnt + cr % kNP, (uint32_t)(R * (cr / kNP + 1)), abort_flag, head_abort,
+                                            wait_ns);
+                    if (!team_ok(good)) {
+                        failed = true;
+                        break;
+                    }
+                    const float *cpart = hpart + (size_t)(cr % kNP) * R * kC * K::PR;
+                    for (int itm = q2; itm < K::ROWS * NV; itm += kQ2T) {
+                        const int rr = itm / NV, v = itm % NV;
+                        const size_t off = (size_t)(rank * K::ROWS + rr) * K::PR + (v < D / 4 ? v * 4 : D);
+                        if (v < D / 4) {
+                            float4 x[R];
+#pragma unroll
+                            for (int r2 = 0; r2 < R; ++r2)
+                                x[r2] = __ldcg(reinterpret_cast<const float4 *>(cpart + (size_t)r2 * kC * K::PR + off));
+                            float4 acc4 = x[0];
+#pragma unroll
+                            for (int r2 = 1; r2 < R; ++r2) {
+                                acc4.x += x[r2].x;
+                                acc4.y += x[r2].y;
+                                acc4.z += x[r2].z;
+                                acc4.w += x[r2].w;
+                            }
+                            *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc4;
+                        } else {
+                            float accs = 0.0f;
+#pragma unroll
+                            for (int r2 = 0; r2 < R; ++r2) accs += __ldcg(cpart + (size_t)r2 * kC * K::PR + off);
+                            res[rr * K::PR + D] = accs;
+                        }
+                    }
+                    named_bar_sync(kBarQ2, kQ2T);
+                    if (q2 == 0) red_release_gpu_add(consumed_cnt + cr % kNP, 1u);
+                    write_output(cr);
+                    named_bar_sync(kBarQ2, kQ2T);  // res is reused by the next chunk
+                }
+            }
+        } else {
+            // reduction through distributed shared memory within the cluster
+            float *part0 = reinterpret_cast<float *>(smem + K::OFF_PART);
+            for (int c = 0; c < nc; ++c) {
+                const bool owner = (c % R) == (int)rank;
+                bool good = mbar_wait_abortable(&misc->t_full, c & 1, abort_flag, wait_ns);
+                if (owner) good = good && mbar_wait_abortable(&misc->p_full, kown & 1, abort_flag, wait_ns);
+                if (c >= 2)
+                    good = good && mbar_wait_cluster(&misc->consumed[c & 1], ((c >> 1) - 1) & 1, abort_flag, wait_ns);
+                if (!team_ok(good)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                drain(c, part0 + (c & 1) * kC * K::PR + row * K::PR, owner);
+                if (owner) ++kown;
+                named_bar_sync(kBarQ2, kQ2T);
+                // thread r announces this CTA's partial to cluster CTA r
+                if (q2 < R) {
+                    fence_acq_rel_cluster();
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&misc->ready[c & 1]), (uint32_t)q2));
+                }
+                good = mbar_wait_cluster(&misc->ready[c & 1], (c >> 1) & 1, abort_flag, wait_ns);
+                if (!team_ok(good)) {
+                    failed = true;
+                    break;
+                }
+                const uint32_t pb = smem_u32(part0 + (c & 1) * kC * K::PR);
+                for (int itm = q2; itm < K::ROWS * NV; itm += kQ2T) {
+                    const int rr = itm / NV, v = itm % NV;
+                    const uint32_t off = (uint32_t)((rank * K::ROWS + rr) * K::PR + (v < D / 4 ? v * 4 : D)) * 4u;
+                    if (v < D / 4) {
+                        float4 x[R];
+#pragma unroll
+                        for (int r2 = 0; r2 < R; ++r2) x[r2] = ld_dsmem_f4(mapa_shared(pb + off, (uint32_t)r2));
+                        float4 acc4 = x[0];
+#pragma unroll
+                        for (int r2 = 1; r2 < R; ++r2) {
+                            acc4.x += x[r2].x;
+                            acc4.y += x[r2].y;
+                            acc4.z += x[r2].z;
+                            acc4.w += x[r2].w;
+                        }
+                        *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc4;
+                    } else {
+                        float x[R];
+#pragma unroll
+                        for (int r2 = 0; r2 < R; ++r2) x[r2] = ld_dsmem_f1(mapa_shared(pb + off, (uint32_t)r2));
+                        float accs = x[0];
+#pragma unroll
+                        for (int r2 = 1; r2 < R; ++r2) accs += x[r2];
+                        res[rr * K::PR + D] = accs;
+                    }
+                }
+                named_bar_sync(kBarQ2, kQ2T);
+                if (q2 < R) {
+                    fence_acq_rel_cluster();
+                    mbar_arrive_cluster(mapa_shared(smem_u32(&misc->consumed[c & 1]), (uint32_t)q2));
+                }
+                write_output(c);
+                named_bar_sync(kBarQ2, kQ2T);  // res is reused by the next chunk
+            }
+        }
+        if (failed && q2 == 0) timeout(40);
+    } else {
+        // ------------------------------------------------------------ decay warp
+        // kernel (a): chunk-local inclusive cumsum of the log-decay (log2 units),
+        // the chunk total, the key weights wk[a][j / 2] = bf16 pair of
+        // 2^(lam - acs_j) k_ja, and V <- diag(dt) V under value discretisation
+        const float A2 = log_decay ? 0.0f : -expf(A_log[h]) * kLog2e;
+        const float bias = dt_bias ? dt_bias[h] : 0.0f;  // given whenever dt is used
+        const float *dsrc = log_decay ? log_decay : dt_p;
+        const bool vdt_own = value_dt && log_decay;  // the dt projection, when it is not dsrc
+        float2 dnext = make_float2(0.f, 0.f), vnext = make_float2(0.f, 0.f);
+        if (nc > 0) {
+            dnext = *reinterpret_cast<const float2 *>(dsrc + (size_t)row0 + 2 * lane);
+            if (vdt_own) vnext = *reinterpret_cast<const float2 *>(dt_p + (size_t)row0 + 2 * lane);
+        }
+        bool ok = true;
         for (int c = 0; c < nc; ++c) {
             const int st = c % kStages;
-            uint8_t *sQ = smem + K::OFF_STAGE + st * K::STAGE;
-            uint8_t *sK = sQ + K::TILE;
-            uint8_t *sV = sK + K::TILE;
-            const float dtv = dt_next;
-            if (ct < kC && c + 1 < nc) dt_next = dsrc[(size_t)row0 + (size_t)(c + 1) * kC + ct];
-            const float vdt = vdt_own ? vdt_next : dtv;
-            if (vdt_own && ct < kC && c + 1 < nc) vdt_next = dt_p[(size_t)row0 + (size_t)(c + 1) * kC + ct];
-
-            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag);
-            // ---- decay (tokens 0..63 on threads 0..63)
-            float a = 0.0f;
-            if (ct < kC) {
-                a = log_decay ? dtv * kLog2e : A2 * softplus_f(dtv + bias);
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, a, o);
-                    if (lane >= o) a += y;
-                }
-                if (lane == 31) misc->wtot[ct >> 5] = a;
-                if (value_dt) misc->vfac[ct] = softplus_f(vdt + bias);
+            const float2 dv = dnext, vv = vdt_own ? vnext : dnext;
+            if (c + 1 < nc) {
+                dnext = *reinterpret_cast<const float2 *>(dsrc + (size_t)row0 + (size_t)(c + 1) * kC + 2 * lane);
+                if (vdt_own) vnext = *reinterpret_cast<const float2 *>(dt_p + (size_t)row0 + (size_t)(c + 1) * kC + 2 * lane);
             }
-            if (named_bar_any(1, kTeam, bad)) {  // also publishes wtot[] and vfac[]
-                if (elected) raise_timeout(misc, status, 30);
-                break;
+            // tokens 2 lane and 2 lane + 1
+            const float a0 = log_decay ? dv.x * kLog2e : A2 * softplus_f(dv.x + bias);
+            const float a1 = log_decay ? dv.y * kLog2e : A2 * softplus_f(dv.y + bias);
+            float incl = a0 + a1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const float lam = __shfl_sync(0xffffffffu, incl, 31);
+            if (c >= 2) {
+                ok = mbar_wait_abortable(&misc->decay_free[c & 1], ((c >> 1) - 1) & 1, abort_flag, wait_ns);
+                if (!__all_sync(0xffffffffu, ok)) break;
+            }
+            misc->acs2[c & 1][2 * lane] = incl - a1;
+            misc->acs2[c & 1][2 * lane + 1] = incl;
+            if (value_dt) {
+                misc->vfac[2 * lane] = softplus_f(vv.x + bias);
+                misc->vfac[2 * lane + 1] = softplus_f(vv.y + bias);
+            }
+            if (lane == 0) misc->lam2[c & 1] = lam;
+            ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag, wait_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            __syncwarp();
+            uint8_t *sK = smem + K::OFF_STAGE + st * K::STAGE + K::TILE;
+            uint8_t *sV = sK + K::TILE;
+            const float *acs = misc->acs2[c & 1];
+            uint32_t *wk = reinterpret_cast<uint32_t *>(smem + K::OFF_WK) + (c & 1) * K::NA * 32;
+            // key weights: lane handles token pair jp = lane for every a of the CTA
+            {
+                const int j = 2 * lane;
+                const float w0 = ex2_approx(lam - acs[j]), w1 = ex2_approx(lam - acs[j + 1]);
+#pragma unroll 4
+                for (int al = 0; al < K::NA; ++al) {
+                    const int av = rank * K::NA + al;
+                    wk[al * 32 + lane] = pack_bf16x2(w0 * bf16_at(sK + swz_elem<RB>(j, av)),
+                                                     w1 * bf16_at(sK + swz_elem<RB>(j + 1, av)));
+                }
             }
             if (value_dt) {
-                // value discretisation: V <- diag(dt) V in place, before P V and the
-                // state products read it (both wait for p_full below); the
-                // normaliser and the D residual use the raw scores and v
+                // value discretisation: V <- diag(dt) V in place, before any product reads it
                 constexpr int CPR = D / 8;  // 16-byte chunks per row
-                for (int t = ct; t < kC * CPR; t += kTeam) {
+                for (int t = lane; t < kC * CPR; t += 32) {
                     const int r = t / CPR, ch = t % CPR;
-                    uint4 *pv = reinterpret_cast<uint4 *>(sV + swz<K::RB>(r, ch));
+                    uint4 *pv = reinterpret_cast<uint4 *>(sV + swz<RB>(r, ch));
                     const float f = misc->vfac[r];
                     const float2 f2 = make_float2(f, f);
                     const uint4 x = *pv;
@@ -449,245 +887,18 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                     *pv = make_uint4(w[0], w[1], w[2], w[3]);
                 }
-            }
-            if (ct >= 32 && ct < kC) a += misc->wtot[0];
-            if (ct < kC) misc->acs2[ct] = a;
-            const float lam2 = misc->wtot[0] + misc->wtot[1];
-
-            // ---- P = S^2 2^(acs_i - acs_j) [i >= j]: row mrow, columns [32 hf, 32 hf + 32)
-            bad = !mbar_wait_abortable(&misc->s_full, c & 1, abort_flag);
-            if (named_bar_any(1, kTeam, bad)) {  // also publishes acs2[]
-                if (elected) raise_timeout(misc, status, 31);
-                break;
-            }
-            tc_fence_after();
-            {
-                float sv[32];
-                tmem_ld32(tmem + lane_off + K::COL_S + hf * 32, sv);
-                tmem_wait_ld();
-                if (own_row) {  // rows of other CTAs are never read back from Y
-                    const float ai = misc->acs2[mrow];
-                    float rs = 0.0f;
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int j = hf * 32 + e;
-                        float p0 = sv[e] * sv[e] * ex2_approx(ai - misc->acs2[j]);
-                        float p1 = sv[e + 1] * sv[e + 1] * ex2_approx(ai - misc->acs2[j + 1]);
-                        if (j > mrow) p0 = 0.0f;
-                        if (j + 1 > mrow) p1 = 0.0f;
-                        rs += p0 + p1;
-                        pk[e >> 1] = pack_bf16x2(p0, p1);
-                    }
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4)
-                        *reinterpret_cast<uint4 *>(smem + K::OFF_P + sw128_chunk(mrow, hf * 4 + k4)) =
-                            make_uint4(pk[k4 * 4], pk[k4 * 4 + 1], pk[k4 * 4 + 2], pk[k4 * 4 + 3]);
-                    misc->rsum[hf][mrow] = rs;
-                }
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            mbar_arrive(&misc->p_full);
-
-            // ---- state slabs
-            const float acs_tok = misc->acs2[tok];
-            const float wk = ex2_approx(lam2 - acs_tok);   // w_j for F_k
-            const float sqs = ex2_approx(acs_tok);         // 2^acs_i for F_q
-            const float dec = ex2_approx(lam2);            // decay over the whole chunk
-            for (int sl = 0; sl < kNs; ++sl) {
-                const int b = sl & 1;
-                if (slab_uses[b] > 0) {
-                    bad = !mbar_wait_abortable(&misc->slab_done[b], (slab_uses[b] - 1) & 1, abort_flag);
-                    if (named_bar_any(1, kTeam, bad)) {
-                        if (elected) raise_timeout(misc, status, 32);
-                        goto done;
-                    }
-                    tc_fence_after();
-                }
-                // h_{c-1} of this slab -> bf16, then h *= 2^lam (columns [hf D/2, hf D/2 + D/2));
-                // z likewise (column 0, half 0 only).  Before chunk 0 the state
-                // is the carried one, read from global memory (zero if absent).
-                if (c >= 1 || carry) {
-                    constexpr int HC = D / 2;
-                    float hv[HC];
-                    float zv = 0.0f;
-                    const uint32_t ta = tmem + lane_off + K::COL_H + sl * D + hf * HC;
-                    const size_t m = (size_t)bh * D * D + rank * kFs + sl * kSlab + frow;  // feature row
-                    if (c >= 1) {
-                        if constexpr (HC == 32) tmem_ld32(ta, hv);
-                        else tmem_ld16(ta, hv);
-                        if (track_z && hf == 0) zv = tmem_ld1(tmem + lane_off + K::COL_Z + sl * 16);
-                        tmem_wait_ld();
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < HC; j += 4) {
-                            const float4 x = h0 ? *reinterpret_cast<const float4 *>(h0 + m * D + hf * HC + j)
-                                                : make_float4(0.f, 0.f, 0.f, 0.f);
-                            hv[j] = x.x;
-                            hv[j + 1] = x.y;
-                            hv[j + 2] = x.z;
-                            hv[j + 3] = x.w;
-                        }
-                        if (track_z && hf == 0 && z0) zv = z0[m];
-                    }
-                    uint8_t *hb = smem + K::OFF_HB + b * kSlab * K::RB;
-#pragma unroll
-                    for (int ch = 0; ch < HC / 8; ++ch)
-                        *reinterpret_cast<uint4 *>(hb + swz<K::RB>(frow, hf * (HC / 8) + ch)) =
-                            make_uint4(pack_bf16x2(hv[ch * 8], hv[ch * 8 + 1]),
-                                       pack_bf16x2(hv[ch * 8 + 2], hv[ch * 8 + 3]),
-                                       pack_bf16x2(hv[ch * 8 + 4], hv[ch * 8 + 5]),
-                                       pack_bf16x2(hv[ch * 8 + 6], hv[ch * 8 + 7]));
-                    const float2 d2 = make_float2(dec, dec);
-#pragma unroll
-                    for (int e = 0; e < HC; e += 2) {
-                        const float2 r2 = __fmul2_rn(make_float2(hv[e], hv[e + 1]), d2);
-                        hv[e] = r2.x;
-                        hv[e + 1] = r2.y;
-                    }
-                    if constexpr (HC == 32) tmem_st32(ta, hv);
-                    else tmem_st16(ta, hv);
-                    if (track_z && hf == 0) {
-                        // column 0 of the zb row; the rest of the tile stays zero
-                        uint8_t *zb = smem + K::OFF_ZB + b * kSlab * K::RB;
-                        *reinterpret_cast<uint4 *>(zb + swz<K::RB>(frow, 0)) =
-                            make_uint4(pack_bf16x2(zv, 0.0f), 0u, 0u, 0u);
-                        tmem_st1(tmem + lane_off + K::COL_Z + sl * 16, zv * dec);
-                    }
-                }
-                // features: token `tok`, slab-local features [32 q4, 32 q4 + 32)
-                {
-                    const int fl0 = q4 * 32;
-                    const int a = (int)(rank * kFs + sl * kSlab + fl0) / D;  // first index of the pair
-                    const int b0 = (rank * kFs + sl * kSlab + fl0) % D;
-                    const float ka = bf16_at(sK + swz<K::RB>(tok, a >> 3) + (a & 7) * 2);
-                    const float qa = bf16_at(sQ + swz<K::RB>(tok, a >> 3) + (a & 7) * 2);
-                    const float2 sk2 = make_float2(wk * ka, wk * ka), sq2 = make_float2(sqs * qa, sqs * qa);
-                    uint8_t *fk = smem + K::OFF_FK + b * 16384 + (fl0 >> 6) * 8192;
-                    uint8_t *fq = smem + K::OFF_FQ + b * 16384 + (fl0 >> 6) * 8192;
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) {
-                        const int bb = b0 + ch * 8;
-                        const uint4 ku = *reinterpret_cast<const uint4 *>(sK + swz<K::RB>(tok, bb >> 3));
-                        const uint4 qu = *reinterpret_cast<const uint4 *>(sQ + swz<K::RB>(tok, bb >> 3));
-                        const uint32_t kw[4] = {ku.x, ku.y, ku.z, ku.w}, qw[4] = {qu.x, qu.y, qu.z, qu.w};
-                        uint32_t ok4[4], oq4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 kv = __fmul2_rn(bf2_to_f2(kw[e]), sk2);
-                            const float2 qv = __fmul2_rn(bf2_to_f2(qw[e]), sq2);
-                            ok4[e] = pack_bf16x2(kv.x, kv.y);
-                            oq4[e] = pack_bf16x2(qv.x, qv.y);
-                        }
-                        const int cidx = ((fl0 & 63) >> 3) + ch;  // 16B chunk in the 128B feature row
-                        *reinterpret_cast<uint4 *>(fk + sw128_chunk(tok, cidx)) =
-                            make_uint4(ok4[0], ok4[1], ok4[2], ok4[3]);
-                        *reinterpret_cast<uint4 *>(fq + sw128_chunk(tok, cidx)) =
-                            make_uint4(oq4[0], oq4[1], oq4[2], oq4[3]);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
                 fence_proxy_async_smem();
-                mbar_arrive(&misc->slab_full[b]);
-                ++slab_uses[b];
             }
-
-            // ---- the previous chunk's cluster reduction and output run here,
-            // while this chunk's last slab products are still on the tensor core
-            if (c >= 1 && !reduce_output(c - 1)) {
-                failed = true;
-                break;
-            }
-
-            // ---- this CTA's partial (plus Y and r on its own rows) into part[c & 1]
-            bad = !mbar_wait_abortable(&misc->chunk_done, c & 1, abort_flag);
-            bad = bad || (c >= 2 && !mbar_wait_cluster(&misc->consumed[c & 1], ((c >> 1) - 1) & 1, abort_flag));
-            if (named_bar_any(1, kTeam, bad)) {
-                if (elected) raise_timeout(misc, status, 33);
-                failed = true;
-                break;
-            }
-            tc_fence_after();
-            {
-                constexpr int HC = D / 2;
-                float tv[HC], yv[HC];
-                const uint32_t tt = tmem + lane_off + K::COL_T + hf * HC;
-                const uint32_t ty = tmem + lane_off + K::COL_S + hf * HC;
-                if constexpr (HC == 32) {
-                    tmem_ld32(tt, tv);
-                    tmem_ld32(ty, yv);
-                } else {
-                    tmem_ld16(tt, tv);
-                    tmem_ld16(ty, yv);
-                }
-                const float tn = (normalize && hf == 0) ? tmem_ld1(tmem + lane_off + K::COL_TN) : 0.0f;
-                tmem_wait_ld();
-                tc_fence_before();
-                mbar_arrive(&misc->y_free);
-                if (mrow_ok) {
-                    float *prow = part0 + (c & 1) * kC * K::PR + mrow * K::PR;
-#pragma unroll
-                    for (int e = 0; e < HC; e += 4) {
-                        float4 v = (c >= 1 || carry) ? make_float4(tv[e], tv[e + 1], tv[e + 2], tv[e + 3])
-                                          : make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (own_row) {
-                            v.x += yv[e];
-                            v.y += yv[e + 1];
-                            v.z += yv[e + 2];
-                            v.w += yv[e + 3];
-                        }
-                        *reinterpret_cast<float4 *>(prow + hf * HC + e) = v;
-                    }
-                    if (hf == 0)
-                        prow[D] = ((c >= 1 || carry) ? tn : 0.0f) +
-                                  (own_row ? misc->rsum[0][mrow] + misc->rsum[1][mrow] : 0.0f);
-                }
-            }
-            named_bar_sync(1, kTeam);
-            // thread r announces this CTA's partial to cluster CTA r; the R remote
-            // arrivals (each a cluster-scope release) run in parallel
-            if (ct < K::R) {
-                fence_acq_rel_cluster();
-                mbar_arrive_cluster(mapa_shared(smem_u32(&misc->ready[c & 1]), ct));
-            }
-            // the stage is no longer read: features are built, the products are
-            // done and the output reads v from global memory
-            if (elected) mbar_arrive(&misc->stage_empty[st]);
+            mbar_arrive(&misc->decay_ready[c & 1]);
+            mbar_arrive(&misc->stage_empty[st]);
         }
-        if (!failed && nc >= 1) reduce_output(nc - 1);
-        // the state after the last token: TMEM holds it once the last chunk's
-        // products are done (waited for above)
-        if (kState && !failed && (h_out || z_out)) {
-            tc_fence_after();
-            constexpr int HC = D / 2;
-            for (int sl = 0; sl < kNs; ++sl) {
-                const size_t m = (size_t)bh * D * D + rank * kFs + sl * kSlab + frow;
-                if (h_out) {
-                    float hv[HC];
-                    const uint32_t ta = tmem + lane_off + K::COL_H + sl * D + hf * HC;
-                    if constexpr (HC == 32) tmem_ld32(ta, hv);
-                    else tmem_ld16(ta, hv);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < HC; j += 4)
-                        *reinterpret_cast<float4 *>(h_out + m * D + hf * HC + j) =
-                            make_float4(hv[j], hv[j + 1], hv[j + 2], hv[j + 3]);
-                }
-                if (z_out) {
-                    const float zv = tmem_ld1(tmem + lane_off + K::COL_Z + sl * 16);
-                    tmem_wait_ld();
-                    if (hf == 0) z_out[m] = zv;
-                }
-            }
-        }
-    done:;
+        if (!ok) timeout(50);
     }
 
     __syncwarp();
     tc_fence_before();
-    cluster_sync_all();  // no CTA leaves while another may still read its shared memory
+    if constexpr (GL) __syncthreads();
+    else cluster_sync_all();  // no CTA leaves while another may still read its shared memory
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
@@ -721,6 +932,12 @@ bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, int d) {
     return r == CUDA_SUCCESS;
 }
 
+// Workspace of the reduction through L2 (D = 64): per head, 64 bytes of
+// counters [ready[kNP], consumed[kNP], abort], then the partial ring
+// [B H][kNP][R][64][PR] fp32.
+size_t counters_bytes(int BH) { return align_up((size_t)BH * kCounterStride, 256); }
+size_t partials_bytes(int BH) { return (size_t)BH * kNP * Cfg<64>::R * kC * Cfg<64>::PR * sizeof(float); }
+
 template <int D>
 int launch_d(const FwdArgs &a) {
     using K = Cfg<D>;
@@ -739,24 +956,38 @@ int launch_d(const FwdArgs &a) {
             return SSD_ERR_CUDA;
         attr_set.fetch_or(bit);
     }
+    const int BH = a.B * a.H;
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    uint32_t *counters = nullptr;
+    float *gpart = nullptr;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.B * a.H * K::R);
+    cfg.gridDim = dim3(BH * K::R);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = K::SMEM;
     cfg.stream = a.stream;
     cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = K::R;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    if constexpr (K::GLOBAL) {
+        // the head's CTAs wait on one another through L2: a cooperative launch
+        // guarantees that all of them are resident (or the launch fails)
+        counters = reinterpret_cast<uint32_t *>(ws + kStatusBytes);
+        gpart = reinterpret_cast<float *>(ws + kStatusBytes + counters_bytes(BH));
+        if (cudaMemsetAsync(counters, 0, counters_bytes(BH), a.stream) != cudaSuccess) return SSD_ERR_CUDA;
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+    } else {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = K::R;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+    }
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     DeviceStatus *status = reinterpret_cast<DeviceStatus *>(a.workspace);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv,
-                                       static_cast<const __nv_bfloat16 *>(a.v),
-                                       static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log,
-                                       a.dt_bias, a.D, a.log_decay, a.value_dt, a.H, a.N, a.normalize,
-                                       a.h0, a.z0, a.h_out, a.z_out, status);
+    const unsigned long long wait_ns = a.wait_ns ? a.wait_ns : 1000000000ull;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, static_cast<const __nv_bfloat16 *>(a.v),
+                                       static_cast<__nv_bfloat16 *>(a.out), a.dt_p, a.A_log, a.dt_bias, a.D,
+                                       a.log_decay, a.value_dt, a.H, a.N, a.normalize, a.h0, a.z0, a.h_out,
+                                       a.z_out, status, counters, gpart, a.dbg_skip, wait_ns);
     return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
@@ -767,7 +998,11 @@ bool tc_order2_supports(int B, int H, int N, int d, int dtype, int chunk) {
            (long long)B * H * N < (1ll << 31);
 }
 
-size_t tc_order2_workspace(int, int, int, int, int) { return 0; }
+size_t tc_order2_workspace(int B, int H, int, int d, int) {
+    if (d != 64) return 0;
+    const int BH = B * H;
+    return counters_bytes(BH) + partials_bytes(BH);
+}
 
 int launch_tc_order2(const FwdArgs &a, const Plan &) {
     return a.d == 64 ? launch_d<64>(a) : launch_d<32>(a);

@@ -28,6 +28,8 @@ def _kind_of_param(p):
         return "ptr"
     if "size_t" in p:
         return "size"
+    if "long long" in p:
+        return "int64"
     return "int"
 
 
@@ -38,6 +40,8 @@ def _kind_of_argtype(t):
         return "size"
     if t is ctypes.c_int:
         return "int"
+    if t is ctypes.c_longlong:
+        return "int64"
     return repr(t)
 
 

@@ -173,3 +173,25 @@ def test_prefill_state_with_mamba2s_options(case):
     assert rel_err(_np(ho), h_ref) <= TOL[dtype]
     if use_z:
         assert rel_err(_np(zo), z_ref) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("n_chunks", [17, 20, 64])
+def test_prefill_state_heads_longer_than_sixteen_chunks(n_chunks):
+    """The order-1 state pass keeps sixteen chunks' inputs in flight for heads
+    of up to 16 chunks and eight for longer ones; a carried state in and out on
+    heads of 17, 20 and 64 chunks runs the second variant."""
+    d, chunk = 64, 128
+    B, H, N = 1, 2, n_chunks * chunk
+    x = inputs.make_inputs(B, H, N, d, "bf16", seed=45 + n_chunks, residual=True)
+    h0, _ = _state(B, H, d, 1, 45)
+    dev = to_device(x, "bf16")
+    h0d = torch.from_numpy(h0).cuda()
+    ho = torch.empty_like(h0d)
+    y = ssd.ssd_fwd_state(dev["q"], dev["k"], dev["v"], dev["dt_p"], dev["A_log"], dev["dt_bias"], dev["D"],
+                          1, False, chunk, h0=h0d, h_out=ho)
+    torch.cuda.synchronize()
+    y_ref, _, h_ref, _ = oracle.ssd_recurrent(
+        x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"], 1, False,
+        return_norm=True, return_state=True, h0=h0)
+    assert rel_err(_np(y), y_ref) <= TOL["bf16"]
+    assert rel_err(_np(ho), h_ref) <= TOL["bf16"]

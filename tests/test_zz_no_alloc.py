@@ -2,8 +2,9 @@
 memory (their host application owns the device memory pool, or they must
 not trigger the synchronisation cudaMalloc can cause).  It runs on a fixed
 scratch buffer inside the library; this test calls it through the C ABI and
-checks it against ssd_fwd on two calls in a row, so a second call that
-wrongly relied on the first call's leftovers would show.
+checks it against ssd_fwd and against the CPU oracle's token recurrence on
+two calls in a row, so a second call that wrongly relied on the first call's
+leftovers would show.
 
 The file is named so that pytest collects it last."""
 import ctypes
@@ -12,6 +13,7 @@ import numpy as np
 import pytest
 
 import mamba_ssd_sequence_b200 as ssd
+import oracle
 from mamba_ssd_sequence_b200 import inputs
 from helpers import TOL, rel_err, to_device
 
@@ -66,6 +68,9 @@ def test_noalloc_matches_ssd_fwd_on_two_calls(shape, dtype, order, normalize, ch
         want = ref.float().cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(got))
         assert rel_err(got, want) <= TOL[dtype]
+        ref = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"],
+                                   order, normalize)
+        assert rel_err(got, ref) <= TOL[dtype]
         outs.append(got)
     assert not np.array_equal(outs[0], outs[1])
 
