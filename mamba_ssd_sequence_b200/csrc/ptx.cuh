@@ -370,6 +370,12 @@ __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_
         "r"(v[29]), "r"(v[30]), "r"(v[31])
         : "memory");
 }
+// 32 lanes x 4 consecutive 32-bit columns (store).
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v0), "r"(v1),
+                 "r"(v2), "r"(v3)
+                 : "memory");
+}
 // 32 lanes x 1 32-bit column.
 __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     uint32_t r;

@@ -61,7 +61,7 @@ constexpr int kC = 64;          // chunk length
 constexpr int kFs = 512;        // feature rows per CTA
 constexpr int kSlab = 128;      // feature rows per slab (one M = 128 tile)
 constexpr int kNs = kFs / kSlab;
-constexpr int kStages = 3;      // Q, K, V tiles
+constexpr int kMaxStages = 3;   // Q, K, V tile ring (3 at d_h 32, 2 at d_h 64)
 constexpr int kNQ = 3;          // Fq ring
 constexpr int kNP = 4;          // partial ring of the reduction through L2
 constexpr int kSTT = 256;       // state team: warps 2-9
@@ -92,9 +92,10 @@ struct Cfg {
     static constexpr int NT = D + 8;               // readout columns: T, Tn, zeros
     static constexpr int PR = D + 4;               // padded partial row (floats)
     static constexpr bool GLOBAL = D == 64;        // reduction through L2 (no cluster)
+    static constexpr int STAGES = D == 64 ? 2 : 3;  // Q, K, V tile ring
     // shared memory map (bytes from a 1024-aligned base)
     static constexpr uint32_t OFF_STAGE = 0;
-    static constexpr uint32_t OFF_HB = kStages * STAGE;                 // kNs x 128 rows
+    static constexpr uint32_t OFF_HB = STAGES * STAGE;                  // kNs x 128 rows
     // z of slab s in logical 16-byte chunk s of each row: the readout's
     // descriptor for slab s starts its second N atom 16 s bytes in
     static constexpr uint32_t OFF_ZB = OFF_HB + kNs * HBT;              // 128 rows
@@ -103,7 +104,10 @@ struct Cfg {
     static constexpr uint32_t OFF_PART = OFF_P + 8192;                  // 2 x 64 x PR (cluster only)
     static constexpr uint32_t OFF_RES = OFF_PART + (GLOBAL ? 0 : 2 * kC * PR * 4);  // ROWS x PR
     static constexpr uint32_t OFF_WK = (OFF_RES + ROWS * PR * 4 + 15) / 16 * 16;      // 2 x NA x 32
-    static constexpr uint32_t OFF_MISC = (OFF_WK + 2 * NA * 32 * 4 + 1023) / 1024 * 1024;
+    // K^T as bf16 pairs of consecutive tokens, per chunk parity: row b holds the
+    // 32 pairs of column b, 16-byte chunk j of row b at position j ^ (b % 8)
+    static constexpr uint32_t OFF_KT = OFF_WK + 2 * NA * 32 * 4;                      // 2 x D x 128 B
+    static constexpr uint32_t OFF_MISC = (OFF_KT + 2 * D * 128 + 1023) / 1024 * 1024;
     static constexpr uint32_t SMEM = OFF_MISC + 2048 + 1024;
     // tensor memory columns.  The readout and S are M = 64 accumulators
     // sharing columns: the readout in lanes 0-15 of each quarter, S in lanes
@@ -124,7 +128,7 @@ struct Misc {
     float rsum[kC];      // row sums of P (chunks whose quadratic part this CTA adds)
     float Dh[64];        // D of the head
     float lam2[2];       // chunk total per chunk parity (state team reads it)
-    uint64_t stage_full[kStages], stage_empty[kStages];
+    uint64_t stage_full[kMaxStages], stage_empty[kMaxStages];
     uint64_t decay_ready[2], decay_free[2];
     uint64_t st_ready[kNs], slab_done[kNs], q_ready[kNQ];
     uint64_t t_full, t_free, s_full, p_full;
@@ -216,6 +220,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     constexpr int R = K::R;
     constexpr uint32_t RB = K::RB;
     constexpr bool GL = K::GLOBAL;
+    constexpr int kStages = K::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -406,16 +411,11 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int c = 0; c < nc; ++c) {
             const int st = c % kStages;
             if (!wait(&misc->stage_full[st], (c / kStages) & 1)) break;
-            // k_jb of the chunk's 64 tokens, as bf16 pairs (j, j + 1)
-            const uint8_t *sK = smem + K::OFF_STAGE + st * K::STAGE + K::TILE;
-            uint32_t kp[32];
-#pragma unroll
-            for (int p = 0; p < 32; ++p)
-                kp[p] = bf16_bits_at(sK + swz_elem<RB>(2 * p, bcol)) | (bf16_bits_at(sK + swz_elem<RB>(2 * p + 1, bcol)) << 16);
             mbar_arrive(&misc->stage_empty[st]);
             if (!wait(&misc->decay_ready[c & 1], (c >> 1) & 1)) break;
             const float dec = ex2_approx(misc->lam2[c & 1]);
             const uint32_t *wk = reinterpret_cast<const uint32_t *>(smem + K::OFF_WK) + (c & 1) * K::NA * 32;
+            const uint8_t *kTrow = smem + K::OFF_KT + (c & 1) * D * 128 + bcol * 128;  // k_jb pairs of column b
 #pragma unroll
             for (int si = 0; si < 2; ++si) {
                 const int s = hh + 2 * si;
@@ -464,20 +464,17 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 {
                     const uint4 *wr = reinterpret_cast<const uint4 *>(wk + (4 * lg + s) * 32);
                     float2 zs = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int th = 0; th < 2; ++th) {
-                        uint32_t fk[16];
-#pragma unroll
-                        for (int v4 = 0; v4 < 4; ++v4) {
-                            const uint4 w = wr[4 * th + v4];
-                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                fk[4 * v4 + e] = mul_bf16x2(ww[e], kp[16 * th + 4 * v4 + e]);
-                                zs = __fadd2_rn(zs, bf2_to_f2(fk[4 * v4 + e]));
-                            }
-                        }
-                        tmem_st16(tmem + lane_off + K::COL_FK + s * 32 + th * 16, fk);
+                    // eight steps of four token pairs: two 16-byte loads, four
+                    // products, one 4-column store (few registers live at a time)
+#pragma unroll 2
+                    for (int q4 = 0; q4 < 8; ++q4) {
+                        const uint4 w = wr[q4];
+                        const uint4 kq = *reinterpret_cast<const uint4 *>(kTrow + (((q4 ^ bcol) & 7) << 4));
+                        const uint32_t f0 = mul_bf16x2(w.x, kq.x), f1 = mul_bf16x2(w.y, kq.y);
+                        const uint32_t f2 = mul_bf16x2(w.z, kq.z), f3 = mul_bf16x2(w.w, kq.w);
+                        zs = __fadd2_rn(zs, __fadd2_rn(__fadd2_rn(bf2_to_f2(f0), bf2_to_f2(f1)),
+                                                       __fadd2_rn(bf2_to_f2(f2), bf2_to_f2(f3))));
+                        tmem_st4(tmem + lane_off + K::COL_FK + s * 32 + 4 * q4, f0, f1, f2, f3);
                     }
                     zr[si] = fmaf(zr[si], dec, zs.x + zs.y);
                 }
@@ -626,13 +623,21 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         auto team_ok = [&](bool good) { return !named_bar_any(kBarQ2, kQ2T, !good); };
         static_assert(K::ROWS * (D / 8) <= kQ2T, "one output item per thread");
         constexpr int NV = D / 4 + 1;  // float4 groups of a row, plus the normaliser
+        // residual input of this thread's output item of chunk cc (fetched
+        // ahead of the waits that precede its use)
+        auto load_residual = [&](int cc) -> uint4 {
+            uint4 vu = make_uint4(0u, 0u, 0u, 0u);
+            if (Dres && cc >= 0 && cc < nc && q2 < K::ROWS * (D / 8)) {
+                const size_t o_grow = (size_t)row0 + (size_t)cc * kC + rank * K::ROWS + q2 / (D / 8);
+                vu = __ldg(reinterpret_cast<const uint4 *>(vglob + o_grow * D + (q2 % (D / 8)) * 8));
+            }
+            return vu;
+        };
         // y of chunk cc from the summed rows in res: y = T / Tn [+ D v]
-        auto write_output = [&](int cc) {
+        auto write_output = [&](int cc, uint4 vu) {
             const int o_rr = q2 / (D / 8), o_ch = q2 % (D / 8);
             if (q2 < K::ROWS * (D / 8)) {
                 const size_t o_grow = (size_t)row0 + (size_t)cc * kC + rank * K::ROWS + o_rr;
-                uint4 vu = make_uint4(0u, 0u, 0u, 0u);
-                if (Dres) vu = __ldg(reinterpret_cast<const uint4 *>(vglob + o_grow * D + o_ch * 8));
                 const float *rrow = res + o_rr * K::PR;
                 const float inv = normalize ? 1.0f / rrow[D] : 1.0f;
                 const uint32_t vw[4] = {vu.x, vu.y, vu.z, vu.w};
@@ -657,14 +662,14 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const bool has_read = c >= 1 || carry;
             const float rs = (owner && row_t) ? misc->rsum[row] : 0.0f;
 #pragma unroll
-            for (int half = 0; half < D / 32; ++half) {
-                float tv[32];
-                tmem_ld32(tmem + lane_off + K::COL_T + 32 * half, tv);
+            for (int part = 0; part < D / 16; ++part) {
+                float tv[16];
+                tmem_ld16(tmem + lane_off + K::COL_T + 16 * part, tv);
                 tmem_wait_ld();
                 if (row_t)
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4 *>(dst_row + 32 * half + e) =
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(dst_row + 16 * part + e) =
                             (has_read || owner) ? make_float4(tv[e], tv[e + 1], tv[e + 2], tv[e + 3])
                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
             }
@@ -680,10 +685,38 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             // consumed their finished reductions; each use of a slot adds
             // exactly R to both, because a slot is rewritten only after all R
             // CTAs have reduced its previous chunk (CTAs may run ahead of one
-            // another by up to kNP chunks)
+            // another by up to kNP chunks).  Software pipeline: iteration c
+            // drains chunk c, publishes chunk c - 1 (its stores were issued an
+            // iteration earlier) and reduces chunk c - 2 (its loads are issued
+            // before the drain, so their latency overlaps it).
+            static_assert(K::ROWS * (D / 4) == kQ2T && K::ROWS * R <= kQ2T, "one float4 group per thread");
             uint32_t *ready_cnt = hcnt, *consumed_cnt = hcnt + kNP;
             float *hpart = gpart + (size_t)bh * kNP * R * kC * K::PR;
-            for (int c = 0; c <= nc; ++c) {
+            const int g_rr = q2 / (D / 4), g_v = q2 % (D / 4);   // this thread's float4 group of T
+            const int n_rr = q2 / R, n_r2 = q2 % R;               // this thread's Tn term (q2 < ROWS R)
+            for (int c = 0; c <= nc + 1; ++c) {
+                const int cr = c - 2;
+                float4 x[R];
+                float xn = 0.0f;
+                uint4 vu = make_uint4(0u, 0u, 0u, 0u);
+                if (cr >= 0) {
+                    bool good = true;
+                    if (q2 == 0)
+                        good = counter_wait(ready_cnt + cr % kNP, (uint32_t)(R * (cr / kNP + 1)), abort_flag, head_abort,
+                                            wait_ns);
+                    if (!team_ok(good)) {
+                        failed = true;
+                        break;
+                    }
+                    const float *cpart = hpart + (size_t)(cr % kNP) * R * kC * K::PR;
+                    const size_t goff = (size_t)(rank * K::ROWS + g_rr) * K::PR + 4 * g_v;
+#pragma unroll
+                    for (int r2 = 0; r2 < R; ++r2)
+                        x[r2] = __ldcg(reinterpret_cast<const float4 *>(cpart + (size_t)r2 * kC * K::PR + goff));
+                    if (q2 < K::ROWS * R)
+                        xn = __ldcg(cpart + ((size_t)n_r2 * kC + rank * K::ROWS + n_rr) * K::PR + D);
+                    vu = load_residual(cr);
+                }
                 if (c < nc) {
                     const bool owner = (c % R) == (int)rank;
                     bool good = mbar_wait_abortable(&misc->t_full, c & 1, abort_flag, wait_ns);
@@ -699,49 +732,28 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     tc_fence_after();
                     drain(c, hpart + (((size_t)(c % kNP) * R + rank) * kC + row) * K::PR, owner);
                     if (owner) ++kown;
-                    __threadfence();
-                    named_bar_sync(kBarQ2, kQ2T);
-                    if (q2 == 0) red_release_gpu_add(ready_cnt + c % kNP, 1u);
                 }
-                if (c >= 1) {
-                    // ---- own rows of chunk cr: sum the R partials
-                    const int cr = c - 1;
-                    bool good = true;
-                    if (q2 == 0)
-                        good = counter_wait(ready_cnt + cr % kNP, (uint32_t)(R * (cr / kNP + 1)), abort_flag, head_abort,
-                                            wait_ns);
-                    if (!team_ok(good)) {
-                        failed = true;
-                        break;
+                // every thread's stores of chunk c - 1 precede this barrier (they
+                // preceded the previous one); one release publishes them
+                named_bar_sync(kBarQ2, kQ2T);
+                if (q2 == 0 && c >= 1 && c <= nc) red_release_gpu_add(ready_cnt + (c - 1) % kNP, 1u);
+                if (cr >= 0) {
+                    float4 acc4 = x[0];
+#pragma unroll
+                    for (int r2 = 1; r2 < R; ++r2) {
+                        acc4.x += x[r2].x;
+                        acc4.y += x[r2].y;
+                        acc4.z += x[r2].z;
+                        acc4.w += x[r2].w;
                     }
-                    const float *cpart = hpart + (size_t)(cr % kNP) * R * kC * K::PR;
-                    for (int itm = q2; itm < K::ROWS * NV; itm += kQ2T) {
-                        const int rr = itm / NV, v = itm % NV;
-                        const size_t off = (size_t)(rank * K::ROWS + rr) * K::PR + (v < D / 4 ? v * 4 : D);
-                        if (v < D / 4) {
-                            float4 x[R];
+                    *reinterpret_cast<float4 *>(res + g_rr * K::PR + 4 * g_v) = acc4;
+                    // Tn of row n_rr: the R terms sit on R consecutive lanes
 #pragma unroll
-                            for (int r2 = 0; r2 < R; ++r2)
-                                x[r2] = __ldcg(reinterpret_cast<const float4 *>(cpart + (size_t)r2 * kC * K::PR + off));
-                            float4 acc4 = x[0];
-#pragma unroll
-                            for (int r2 = 1; r2 < R; ++r2) {
-                                acc4.x += x[r2].x;
-                                acc4.y += x[r2].y;
-                                acc4.z += x[r2].z;
-                                acc4.w += x[r2].w;
-                            }
-                            *reinterpret_cast<float4 *>(res + rr * K::PR + v * 4) = acc4;
-                        } else {
-                            float accs = 0.0f;
-#pragma unroll
-                            for (int r2 = 0; r2 < R; ++r2) accs += __ldcg(cpart + (size_t)r2 * kC * K::PR + off);
-                            res[rr * K::PR + D] = accs;
-                        }
-                    }
+                    for (int o = 1; o < R; o <<= 1) xn += __shfl_xor_sync(0xffffffffu, xn, o);
+                    if (q2 < K::ROWS * R && n_r2 == 0) res[n_rr * K::PR + D] = xn;
                     named_bar_sync(kBarQ2, kQ2T);
                     if (q2 == 0) red_release_gpu_add(consumed_cnt + cr % kNP, 1u);
-                    write_output(cr);
+                    write_output(cr, vu);
                     named_bar_sync(kBarQ2, kQ2T);  // res is reused by the next chunk
                 }
             }
@@ -750,6 +762,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             float *part0 = reinterpret_cast<float *>(smem + K::OFF_PART);
             for (int c = 0; c < nc; ++c) {
                 const bool owner = (c % R) == (int)rank;
+                const uint4 vu = load_residual(c);
                 bool good = mbar_wait_abortable(&misc->t_full, c & 1, abort_flag, wait_ns);
                 if (owner) good = good && mbar_wait_abortable(&misc->p_full, kown & 1, abort_flag, wait_ns);
                 if (c >= 2)
@@ -804,7 +817,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     fence_acq_rel_cluster();
                     mbar_arrive_cluster(mapa_shared(smem_u32(&misc->consumed[c & 1]), (uint32_t)q2));
                 }
-                write_output(c);
+                write_output(c, vu);
                 named_bar_sync(kBarQ2, kQ2T);  // res is reused by the next chunk
             }
         }
@@ -859,15 +872,28 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             uint8_t *sV = sK + K::TILE;
             const float *acs = misc->acs2[c & 1];
             uint32_t *wk = reinterpret_cast<uint32_t *>(smem + K::OFF_WK) + (c & 1) * K::NA * 32;
-            // key weights: lane handles token pair jp = lane for every a of the CTA
+            // K^T pairs and key weights: lane l holds token pair (2l, 2l + 1); for
+            // every column b, kT[b][l] = bf16 pair (k_2l,b, k_2l+1,b), and for the
+            // CTA's a, wk[a][l] = bf16 pair (2^(lam - acs_2l) k_2l,a, same for 2l + 1)
             {
                 const int j = 2 * lane;
                 const float w0 = ex2_approx(lam - acs[j]), w1 = ex2_approx(lam - acs[j + 1]);
-#pragma unroll 4
-                for (int al = 0; al < K::NA; ++al) {
-                    const int av = rank * K::NA + al;
-                    wk[al * 32 + lane] = pack_bf16x2(w0 * bf16_at(sK + swz_elem<RB>(j, av)),
-                                                     w1 * bf16_at(sK + swz_elem<RB>(j + 1, av)));
+                uint32_t *kT = reinterpret_cast<uint32_t *>(smem + K::OFF_KT) + (c & 1) * D * 32;
+#pragma unroll 2
+                for (int ch = 0; ch < D / 8; ++ch) {
+                    const uint4 r0 = *reinterpret_cast<const uint4 *>(sK + swz<RB>(j, ch));
+                    const uint4 r1 = *reinterpret_cast<const uint4 *>(sK + swz<RB>(j + 1, ch));
+                    const uint32_t a0[4] = {r0.x, r0.y, r0.z, r0.w}, a1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int b = 8 * ch + e;
+                        const uint32_t lo = (e & 1) ? (a0[e >> 1] >> 16) : (a0[e >> 1] & 0xFFFFu);
+                        const uint32_t hi = (e & 1) ? (a1[e >> 1] & 0xFFFF0000u) : (a1[e >> 1] << 16);
+                        kT[b * 32 + ((((lane >> 2) ^ b) & 7) << 2) + (lane & 3)] = lo | hi;
+                        const int al = b - (int)rank * K::NA;
+                        if (al >= 0 && al < K::NA)
+                            wk[al * 32 + lane] = pack_bf16x2(w0 * __uint_as_float(lo << 16), w1 * __uint_as_float(hi));
+                    }
                 }
             }
             if (value_dt) {
