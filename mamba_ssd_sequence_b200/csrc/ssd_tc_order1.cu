@@ -106,7 +106,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    const float *__restrict__ dt_p, const float *__restrict__ A_log,
                    const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int value_dt,
                    int H, int N, int n_chunks, float *__restrict__ acs_out, float *__restrict__ vfac_out,
-                   float *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status) {
+                   float *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status, int dbg_skip,
+                   unsigned long long wait_ns) {
     using K = StateCfg<C>;
     constexpr int NG = K::NG;
     constexpr int KP = C / 128;  // keys per thread in the decay scan
@@ -159,10 +160,11 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             for (int t = blockIdx.x; t < n_chunks; t += gridDim.x, ++i) {
                 const int st = i % K::STAGES;
                 if (i >= K::STAGES &&
-                    !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag)) {
+                    !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag, wait_ns)) {
                     set_timeout(status, 100, &misc->abort_flag);
                     break;
                 }
+                if (i == dbg_skip) continue;  // failure test: this step is never published
                 const int row = t * C;  // chunks are contiguous row blocks of [B H N, d]
                 uint8_t *sp = smem + st * K::STAGE;
                 mbar_arrive_expect_tx(&misc->stage_full[st], K::STAGE);
@@ -173,7 +175,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 }
             }
             for (int j = i > K::STAGES ? i - K::STAGES : 0; j < i; ++j)
-                mbar_wait_bounded(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1);
+                if (j != dbg_skip) mbar_wait_bounded(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -183,8 +185,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             int i = 0;
             for (int t = blockIdx.x; t < n_chunks; t += gridDim.x, ++i) {
                 const int st = i % K::STAGES, ub = i % NG, use = i / NG;
-                if (!(ok = mbar_wait_abortable(&misc->kp_full[ub], use & 1, abort_flag))) break;
-                if (use >= 1 && !(ok = mbar_wait_abortable(&misc->u_free[ub], (use - 1) & 1, abort_flag))) break;
+                if (!(ok = mbar_wait_abortable(&misc->kp_full[ub], use & 1, abort_flag, wait_ns))) break;
+                if (use >= 1 && !(ok = mbar_wait_abortable(&misc->u_free[ub], (use - 1) & 1, abort_flag, wait_ns))) break;
                 tc_fence_after();
                 const uint32_t sp = sbase + st * K::STAGE;
                 // D[n][k] = sum_j v_jn k'_jk: A = V (MN-major), B = K' (MN-major)
@@ -274,7 +276,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             }
             if (gt == 0) lam_out[t] = lam;
             // ---- K'_j = 2^(lam - acs_j) k_j in place: eight lanes per 128-byte row
-            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (i / K::STAGES) & 1, abort_flag);
+            bool bad = !mbar_wait_abortable(&misc->stage_full[st], (i / K::STAGES) & 1, abort_flag, wait_ns);
             if (named_bar_any(bar, kStateGroup, bad)) {  // also publishes wk[]
                 failed = true;
                 break;
@@ -299,7 +301,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tc_fence_before();
             mbar_arrive(&misc->kp_full[gi]);
             // ---- U^T epilogue: rows 16 g + lane (lanes 0-15) of the M = 64 accumulator
-            bad = !mbar_wait_abortable(&misc->u_full[gi], use & 1, abort_flag);
+            bad = !mbar_wait_abortable(&misc->u_full[gi], use & 1, abort_flag, wait_ns);
             if (named_bar_any(bar, kStateGroup, bad)) {
                 failed = true;
                 break;
@@ -491,7 +493,8 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_h,
                   const __grid_constant__ CUtensorMap tm_out, const __nv_bfloat16 *__restrict__ vglob,
                   const float *__restrict__ acs_in, const float *__restrict__ vfac_in,
-                  const float *__restrict__ Dres, int H, int N, int n_tiles, DeviceStatus *status) {
+                  const float *__restrict__ Dres, int H, int N, int n_tiles, DeviceStatus *status, int dbg_skip,
+                  unsigned long long wait_ns) {
     using K = ScanCfg<C>;
     constexpr int NG = K::NG;
     extern __shared__ uint8_t smem_raw[];
@@ -546,10 +549,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 const int t = blockIdx.x + i * gridDim.x;
                 const int st = i % K::STAGES;
                 if (i >= K::STAGES &&
-                    !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag)) {
+                    !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag, wait_ns)) {
                     set_timeout(status, 110, &misc->abort_flag);
                     break;
                 }
+                if (i == dbg_skip) continue;  // failure test: this step is never published
                 const TileIdx x = tile_idx<C>(t, nc);
                 const int nkb = x.rb + 1;
                 const int crow = x.bh * N + x.c * C;
@@ -565,7 +569,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             // copies still in flight after an abort land before the CTA exits (bounded)
             for (int j = i > K::STAGES ? i - K::STAGES : 0; j < i; ++j)
-                mbar_wait_bounded(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1);
+                if (j != dbg_skip) mbar_wait_bounded(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -642,7 +646,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 } else if ((++spins & 255u) == 0) {
                     const uint64_t now = globaltimer_ns();
                     if (idle_since == 0) idle_since = now;
-                    if (*abort_flag || now - idle_since > 1000000000ull) {
+                    if (*abort_flag || now - idle_since > wait_ns) {
                         ok = false;
                         break;
                     }
@@ -713,7 +717,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 pend_st = -1;
             }
             // ---- S of this tile
-            bool bad = !mbar_wait_abortable(&misc->s_full[sb], (i / K::NSB) & 1, abort_flag);
+            bool bad = !mbar_wait_abortable(&misc->s_full[sb], (i / K::NSB) & 1, abort_flag, wait_ns);
             if (named_bar_any(bar, 256, bad)) {  // also publishes acs[], colf[], dres[]
                 failed = true;
                 break;
@@ -787,11 +791,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
                 for (int q = 0; q < 4; ++q) vres[q] = __ldg(vp + q);
             }
-            bad = !mbar_wait_abortable(&misc->y_full[tb], (i >> 1) & 1, abort_flag);
+            bad = !mbar_wait_abortable(&misc->y_full[tb], (i >> 1) & 1, abort_flag, wait_ns);
             // the V box is read below: observe the stage's TMA completion here too
             // (long complete; the stage cannot be refilled before this group releases it)
             if (!K::OUT_SLOT)
-                bad = bad || !mbar_wait_abortable(&misc->stage_full[i % K::STAGES], (i / K::STAGES) & 1, abort_flag);
+                bad = bad || !mbar_wait_abortable(&misc->stage_full[i % K::STAGES], (i / K::STAGES) & 1, abort_flag, wait_ns);
             if (named_bar_any(bar, 256, bad)) {
                 failed = true;
                 break;
@@ -951,9 +955,10 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     if (sms <= 0) return SSD_ERR_CUDA;
 
     const int n_chunks = BH * nc;
+    const unsigned long long wait_ns = a.wait_ns ? a.wait_ns : 1000000000ull;
     chunk_state_kernel<C><<<n_chunks < sms ? n_chunks : sms, StateCfg<C>::THREADS, StateCfg<C>::SMEM, a.stream>>>(
         tk, tv, tu, a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N, n_chunks, acs, vfac, U, lam,
-        status);
+        status, a.dbg_skip, wait_ns);
     // The state pass and the chunk scan are launched as programmatic dependents:
     // their CTAs may start while the previous kernel drains, and each waits
     // (griddepcontrol.wait) before it reads that kernel's results.
@@ -983,7 +988,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c3.attrs = pdl;
     c3.numAttrs = 1;
     if (cudaLaunchKernelEx(&c3, chunk_scan_kernel<C>, tq, tk, tv, th, to, (const __nv_bfloat16 *)a.v,
-                           (const float *)acs, (const float *)vfac, a.D, a.H, a.N, n_tiles, status) != cudaSuccess)
+                           (const float *)acs, (const float *)vfac, a.D, a.H, a.N, n_tiles, status, a.dbg_skip,
+                           wait_ns) != cudaSuccess)
         return SSD_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
