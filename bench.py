@@ -75,8 +75,6 @@ DRAM_TRAFFIC = {
     # chunk states 34.10 MB + state pass 0.02 MB + chunk outputs 25.80 MB,
     # captured without cache flushes, as the kernels run in a call
     "order1-bf16-B4H16N2048d64-c128": 59_925_402,
-    # one launch, captured after an L2 flush (as in the bench)
-    "order2-bf16-B4H16N4096d32-c64": 51_539_098,
 }
 
 
