@@ -2,6 +2,7 @@
 // libssd.so.  Nothing here is part of the public ABI (see include/ssd.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -74,6 +75,12 @@ size_t tc_order2_workspace(int B, int H, int N, int d, int chunk);
 int launch_tc_order1(const FwdArgs &a, const Plan &p);
 bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);
 void tc_order1_layout(int B, int H, int N, int chunk, Plan *p);
+
+// 2-D TMA tensor map of a row-major [rows, cols] bf16 (or fp32) tensor read or
+// written in boxes of box_rows x box_cols, with the 0, 32, 64 or 128-byte
+// swizzle (ssd_tmap.cu).  False when the driver rejects it.
+bool encode_tmap_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t cols, uint64_t rows,
+                    uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
 // Decode step (ssd_decode.cu).
 size_t decode_workspace(int B, int H, int d, int order);

@@ -24,7 +24,6 @@
 // in (1); with value discretisation the factor dt_j multiplies key j's
 // weight in U (through K') and in P (through the per-key factors).
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -866,46 +865,15 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 }
 
 // ------------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
 // [rows, 64] bf16 row-major tensor read in boxes of `box_rows` rows, 128-byte swizzle.
 bool make_tmap64(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_rows) {
-    auto enc = get_encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {64, rows};
-    cuuint64_t strides[1] = {64 * 2};
-    cuuint32_t box[2] = {64, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encode_tmap_2d(m, base, true, 64, rows, 64, box_rows, 128);
 }
 
 // [rows, 64] fp32 row-major tensor written in boxes of 64 rows x 32 columns,
 // 128-byte swizzle.
 bool make_tmap_f32x64(CUtensorMap *m, void *base, uint64_t rows) {
-    auto enc = get_encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {64, rows};
-    cuuint64_t strides[1] = {64 * 4};
-    cuuint32_t box[2] = {32, 64};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encode_tmap_2d(m, base, false, 64, rows, 32, 64, 128);
 }
 
 // Sets the dynamic shared-memory limit of `fn` once per device.

@@ -43,7 +43,6 @@
 // and h_out, z_out receive the state after the last chunk.  All exponentials
 // are of non-positive arguments.  Every wait is bounded.
 #include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -160,14 +159,6 @@ __device__ __forceinline__ uint32_t swz_elem(uint32_t row, uint32_t col) {
     return swz<RB>(row, col >> 3) + (col & 7u) * 2u;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 // Waits until the counter reaches `target`; gives up (false) on a raised
 // abort flag (this CTA's or the head's) or after limit_ns of wall time.
 __device__ bool counter_wait(const uint32_t *cnt, uint32_t target, const volatile int *abort,
@@ -930,32 +921,9 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 }
 
 // ------------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-
-// [rows, d] bf16 row-major tensor, boxes of 64 rows, swizzle = row bytes.
+// [rows, d] bf16 tiles of kC rows, swizzled to match the descriptors
 bool make_tmap(CUtensorMap *m, const void *base, uint64_t rows, int d) {
-    auto enc = get_encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)d, rows};
-    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {(cuuint32_t)d, kC};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     d == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return encode_tmap_2d(m, base, true, (uint64_t)d, rows, (uint32_t)d, kC, d == 64 ? 128 : 64);
 }
 
 // Workspace of the reduction through L2 (D = 64): per head, 64 bytes of

@@ -1,5 +1,5 @@
 """Generates the coefficients of the polynomial p with log1p(u) ~ u p(u) on
-[0, 1] that kernel (a) (csrc/ssd_simt.cu, softplus_fast) uses: Chebyshev
+[0, 1] that the decay steps (csrc/ssd_math.cuh, softplus_fast) use: Chebyshev
 interpolation of log1p(u)/u at the degree + 1 Chebyshev nodes of [0, 1],
 converted to powers of u and rounded to float32.  Prints the coefficients
 (constant term first) and the largest relative error of u p(u) against
