@@ -217,6 +217,15 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *tmap, const void
                  "r"(smem_u32(smem_src))
                  : "memory");
 }
+// Untiled bulk copy global -> shared (no multicast): `bytes` a multiple of
+// 16, both addresses 16-byte aligned; completes on `bar` with complete_tx.
+__device__ __forceinline__ void bulk_load(void *smem_dst, const void *gsrc, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

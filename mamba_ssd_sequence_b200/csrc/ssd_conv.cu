@@ -4,12 +4,16 @@
 // page, applied to one [B, H, N, d_h] tensor:
 //     u = bias[c] + sum_{j < width} w[c][j] x[t - j, c]   (x before token 0 is 0)
 //     out = SiLU(u) or u
-// One thread per (b, h, t) and 8 consecutive channels, 16-byte loads for
-// bf16.  HBM-bound: it reads x once (the width-1 earlier rows hit L1/L2) and
-// writes out once.
+// One CTA per tile of kTile consecutive tokens of one (b, h): the tile and the
+// width - 1 rows before it are contiguous in memory, so one bulk copy brings
+// them into shared memory (every input row is read from HBM once); the
+// threads then take (token, 8-channel group) items with 16-byte shared loads
+// and global stores.  All CTAs of a call are resident at once, each with its
+// copy in flight, which keeps HBM busy.  HBM-bound.
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "ptx.cuh"
 #include "ssd_internal.h"
 
 namespace ssd {
@@ -46,32 +50,72 @@ __device__ __forceinline__ void store8(__nv_bfloat16 *p, const float (&y)[8]) {
     *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+constexpr int kTile = 128;   // tokens per CTA
+constexpr int kMaxWidth = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_kernel(const T *__restrict__ x, const float *__restrict__ w, const float *__restrict__ bias, int H,
-              int N, int d, int width, int silu, long long n_items, T *__restrict__ out) {
-    const long long item = (long long)blockIdx.x * kConvThreads + threadIdx.x;
-    if (item >= n_items) return;
+              int N, int d, int width, int silu, T *__restrict__ out) {
+    extern __shared__ __align__(128) uint8_t sm[];
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm);
+    T *xs = reinterpret_cast<T *>(sm + 128);  // row r: token t0 - (kMaxWidth - 1) + r
+    const int tiles = (N + kTile - 1) / kTile;
+    const int tile = (int)(blockIdx.x % tiles);
+    const long long bhrow = blockIdx.x / tiles;  // b H + h
+    const int h = (int)(bhrow % H);
+    const int t0 = tile * kTile, tn = min(kTile, N - t0);
+    const int halo = min(kMaxWidth - 1, t0);  // rows before the tile that exist
+    const int tid = threadIdx.x;
+    const uint32_t bytes = (uint32_t)((halo + tn) * d * sizeof(T));
+    if (tid == 0) {
+        ptx::mbar_init(bar, 1);
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0) {
+        ptx::mbar_arrive_expect_tx(bar, bytes);
+        ptx::bulk_load(xs + (kMaxWidth - 1 - halo) * d, x + ((size_t)bhrow * N + t0 - halo) * d, bytes, bar);
+    }
+    // rows before token 0 are zero
+    for (int e = tid; e < (kMaxWidth - 1 - halo) * d; e += kConvThreads) xs[e] = T(0.0f);
+    // the head's weights, tap-major, and bias through shared memory (coalesced
+    // loads while the tile is in flight); a thread then keeps one channel
+    // group (kConvThreads is a multiple of d / 8) in registers
+    float *sw = reinterpret_cast<float *>(sm + 128 + (size_t)(kTile + kMaxWidth - 1) * d * sizeof(T));
+    for (int i = tid; i < d * width; i += kConvThreads) sw[(i % width) * d + i / width] = __ldg(w + (size_t)h * d * width + i);
+    for (int i = tid; i < d; i += kConvThreads) sw[kMaxWidth * d + i] = bias ? __ldg(bias + h * d + i) : 0.0f;
+    const bool ok = ptx::mbar_wait_bounded(bar, 0);
+    __syncthreads();  // the zero rows and the weights too
+    if (!ok) return;  // never expected: the copy lands unless the device faults
     const int g8 = d / 8;
-    const int cg = (int)(item % g8);
-    const long long row = item / g8;       // (b, h, t) flattened
-    const int t = (int)(row % N);
-    const int h = (int)((row / N) % H);
-    const int c0 = cg * 8;
-    float acc[8];
+    const int c0 = (tid % g8) * 8, k0 = tid / g8, kstep = kConvThreads / g8;
+    float wr[kMaxWidth][8], bs[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = bias ? bias[h * d + c0 + e] : 0.0f;
-    for (int j = 0; j < width && j <= t; ++j) {
-        float xv[8];
-        load8(x + (size_t)(row - j) * d + c0, xv);
+    for (int e = 0; e < 8; ++e) {
+        bs[e] = sw[kMaxWidth * d + c0 + e];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = fmaf(w[(size_t)(h * d + c0 + e) * width + j], xv[e], acc[e]);
+        for (int j = 0; j < kMaxWidth; ++j) wr[j][e] = j < width ? sw[j * d + c0 + e] : 0.0f;
     }
-    if (silu) {
+    for (int k = k0; k < tn; k += kstep) {
+        float acc[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = acc[e] / (1.0f + expf(-acc[e]));
+        for (int e = 0; e < 8; ++e) acc[e] = bs[e];
+#pragma unroll
+        for (int j = 0; j < kMaxWidth; ++j) {
+            if (j < width) {
+                float xv[8];
+                load8(xs + (k + kMaxWidth - 1 - j) * d + c0, xv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[e] = fmaf(wr[j][e], xv[e], acc[e]);
+            }
+        }
+        if (silu) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = __fdividef(acc[e], 1.0f + __expf(-acc[e]));
+        }
+        store8(out + ((size_t)bhrow * N + t0 + k) * d + c0, acc);
     }
-    store8(out + (size_t)row * d + c0, acc);
 }
 
 }  // namespace
@@ -92,15 +136,24 @@ extern "C" int ssd_conv1d(const void *x, const float *w, const float *bias, int 
         return SSD_ERR_ALIGN;
     const size_t bytes = (size_t)B * H * N * d_h * (dtype == SSD_F32 ? 4 : 2);
     if (ax < ao + bytes && ao < ax + bytes) return SSD_ERR_SHAPE;  // out must not overlap x
-    const long long n_items = (long long)B * H * N * (d_h / 8);
-    const unsigned grid = (unsigned)((n_items + kConvThreads - 1) / kConvThreads);
+    const long long grid = (long long)B * H * ((N + kTile - 1) / kTile);
+    if (grid >= (1ll << 31)) return SSD_ERR_SHAPE;
+    const size_t esize = dtype == SSD_F32 ? 4 : 2;
+    const size_t smem = 128 + (size_t)(kTile + kMaxWidth - 1) * d_h * esize + (size_t)(kMaxWidth + 1) * d_h * 4;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dtype == SSD_F32)
-        conv1d_kernel<float><<<grid, kConvThreads, 0, s>>>(static_cast<const float *>(x), w, bias, H, N, d_h,
-                                                            width, silu, n_items, static_cast<float *>(out));
-    else
-        conv1d_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, s>>>(
-            static_cast<const __nv_bfloat16 *>(x), w, bias, H, N, d_h, width, silu, n_items,
+    if (dtype == SSD_F32) {
+        if (cudaFuncSetAttribute(conv1d_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
+            return SSD_ERR_CUDA;
+        conv1d_kernel<float><<<(unsigned)grid, kConvThreads, smem, s>>>(static_cast<const float *>(x), w, bias, H, N,
+                                                                        d_h, width, silu, static_cast<float *>(out));
+    } else {
+        if (cudaFuncSetAttribute(conv1d_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess)
+            return SSD_ERR_CUDA;
+        conv1d_kernel<__nv_bfloat16><<<(unsigned)grid, kConvThreads, smem, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), w, bias, H, N, d_h, width, silu,
             static_cast<__nv_bfloat16 *>(out));
+    }
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }

@@ -16,12 +16,16 @@
 #include <cuda_bf16.h>
 #include <math.h>
 
+#include "ptx.cuh"
 #include "ssd_internal.h"
 
 namespace ssd {
 namespace {
 
 constexpr int kDecThreads = 256;
+// float4s of state a thread updates: a CTA holds at most 64 rows of d_h <= 64
+// columns, 1024 float4s
+constexpr int kPerThread = 4;
 
 __device__ __forceinline__ float softplus_f(float x) {
     return fmaxf(x, 0.0f) + log1pf(expf(-fabsf(x)));
@@ -49,19 +53,30 @@ decode_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
                     int value_dt, int H, int d, int order, float *__restrict__ h,
                     float *__restrict__ z, float *__restrict__ part) {
     __shared__ float qs[64], ks[64], vs[64];
-    __shared__ float ys[65];
+    __shared__ float red[kDecThreads / 32][65];
     const int bh = blockIdx.x, s = blockIdx.y, hd = bh % H;
     const int S = gridDim.y;
     const int R = rows_per_cta(d, order);
     const int Dphi = order == 1 ? d : d * d;
     const int m0 = s * R;
     const int tid = threadIdx.x;
+    const int d4 = d / 4;
+    const int n4 = R * d4;  // float4s of this CTA's state rows
+    float4 *hb = reinterpret_cast<float4 *>(h + ((size_t)bh * Dphi + m0) * d);
+    // this thread's state loads go out first (n4 <= kPerThread kDecThreads):
+    // they depend on nothing else, so their latency overlaps the token's
+    float4 xv[kPerThread];
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int e = tid + u * kDecThreads;
+        if (e < n4) xv[u] = __ldcs(hb + e);
+    }
+    const float zv = (z && tid < R) ? z[(size_t)bh * Dphi + m0 + tid] : 0.0f;
     if (tid < d) {
         qs[tid] = load_elem(q, (size_t)bh * d + tid);
         ks[tid] = load_elem(k, (size_t)bh * d + tid);
         vs[tid] = load_elem(v, (size_t)bh * d + tid);
     }
-    if (tid <= d) ys[tid] = 0.0f;
     // decay and value factor of this token
     float dt = 0.0f;
     if (value_dt || !log_decay) dt = softplus_f(dt_p[bh] + dt_bias[hd]);
@@ -69,50 +84,64 @@ decode_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     const float f = value_dt ? dt : 1.0f;
     __syncthreads();
 
-    const int d4 = d / 4;
-    const int n4 = R * d4;  // float4s of this CTA's state rows
-    float4 *hb = reinterpret_cast<float4 *>(h + ((size_t)bh * Dphi + m0) * d);
     // each thread keeps the partial readout of one column group
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     const int c4 = tid % d4;  // column group of this thread: the same for all its elements
-    for (int e = tid; e < n4; e += kDecThreads) {
+#pragma unroll
+    for (int u = 0; u < kPerThread; ++u) {
+        const int e = tid + u * kDecThreads;
+        if (e >= n4) break;
         const int r = e / d4;
         const int m = m0 + r;
         const float fk = order == 1 ? ks[m] : ks[m / d] * ks[m % d];
         const float fq = order == 1 ? qs[m] : qs[m / d] * qs[m % d];
         const float w = fk * f;
-        float4 x = hb[e];
+        float4 x = xv[u];
         x.x = fmaf(a, x.x, w * vs[4 * c4 + 0]);
         x.y = fmaf(a, x.y, w * vs[4 * c4 + 1]);
         x.z = fmaf(a, x.z, w * vs[4 * c4 + 2]);
         x.w = fmaf(a, x.w, w * vs[4 * c4 + 3]);
-        hb[e] = x;
+        __stcs(hb + e, x);
         acc.x = fmaf(fq, x.x, acc.x);
         acc.y = fmaf(fq, x.y, acc.y);
         acc.z = fmaf(fq, x.z, acc.z);
         acc.w = fmaf(fq, x.w, acc.w);
     }
     float nacc = 0.0f;
-    if (z) {
-        for (int r = tid; r < R; r += kDecThreads) {
-            const int m = m0 + r;
-            const float fk = order == 1 ? ks[m] : ks[m / d] * ks[m % d];
-            const float fq = order == 1 ? qs[m] : qs[m / d] * qs[m % d];
-            float *zp = z + (size_t)bh * Dphi + m;
-            const float zn = fmaf(a, *zp, fk);
-            *zp = zn;
-            nacc = fmaf(fq, zn, nacc);
-        }
+    if (z && tid < R) {  // R <= 64 < kDecThreads: one normaliser entry per thread, loaded at the start
+        const int m = m0 + tid;
+        const float fk = order == 1 ? ks[m] : ks[m / d] * ks[m % d];
+        const float fq = order == 1 ? qs[m] : qs[m / d] * qs[m % d];
+        const float zn = fmaf(a, zv, fk);
+        z[(size_t)bh * Dphi + m] = zn;
+        nacc = fq * zn;
     }
-    // reduce the column groups (kDecThreads is a multiple of d4, so each
-    // thread's group is fixed) and the normaliser through shared memory
-    atomicAdd(&ys[4 * c4 + 0], acc.x);
-    atomicAdd(&ys[4 * c4 + 1], acc.y);
-    atomicAdd(&ys[4 * c4 + 2], acc.z);
-    atomicAdd(&ys[4 * c4 + 3], acc.w);
-    if (z) atomicAdd(&ys[d], nacc);
+    // reduce the column groups: lanes tid, tid ^ d4, ... hold the same group
+    // (d4 divides 32), then the warps through shared memory
+    const int lane = tid & 31, wid = tid >> 5;
+    for (int o = d4; o < 32; o <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) nacc += __shfl_xor_sync(0xffffffffu, nacc, o);
+    if (lane < d4) {  // rows of 65 floats: scalar stores (a row is not 16-byte aligned)
+        red[wid][4 * lane + 0] = acc.x;
+        red[wid][4 * lane + 1] = acc.y;
+        red[wid][4 * lane + 2] = acc.z;
+        red[wid][4 * lane + 3] = acc.w;
+    }
+    if (lane == 0) red[wid][d] = nacc;
     __syncthreads();
-    if (tid <= d) part[((size_t)bh * S + s) * (d + 1) + tid] = ys[tid];
+    if (tid <= d) {
+        float y = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kDecThreads / 32; ++w) y += red[w][tid];
+        part[((size_t)bh * S + s) * (d + 1) + tid] = y;
+    }
+    ptx::pdl_launch_dependents();  // the output kernel waits for this grid before it reads part
 }
 
 // Block (65, 4): thread (c, g) sums column c (c = d: the normaliser) over the
@@ -125,6 +154,7 @@ decode_output_kernel(const T *__restrict__ v, const float *__restrict__ D,
                      int normalize, T *__restrict__ out) {
     __shared__ float red[4][65];
     const int bh = blockIdx.x, c = threadIdx.x, g = threadIdx.y;
+    ptx::pdl_wait();  // every partial of the state kernel is visible
     const float *p = part + (size_t)bh * S * (d + 1);
     float acc = 0.0f;
     if (c <= d) {
@@ -151,8 +181,20 @@ int run_decode(const FwdArgs &a, float *h, float *z) {
     decode_state_kernel<T><<<dim3(BH, S), kDecThreads, 0, a.stream>>>(
         static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.dt_p,
         a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.d, a.order, h, z, part);
-    decode_output_kernel<T><<<BH, dim3(65, 4), 0, a.stream>>>(static_cast<const T *>(a.v), a.D, part, a.H,
-                                                              a.d, S, a.normalize, static_cast<T *>(a.out));
+    // launched as a programmatic dependent: its CTAs may start while the state
+    // kernel drains, and each waits (griddepcontrol.wait) before reading part
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3(BH);
+    c2.blockDim = dim3(65, 4);
+    c2.stream = a.stream;
+    c2.attrs = pdl;
+    c2.numAttrs = 1;
+    if (cudaLaunchKernelEx(&c2, decode_output_kernel<T>, static_cast<const T *>(a.v), a.D, (const float *)part, a.H,
+                           a.d, S, a.normalize, static_cast<T *>(a.out)) != cudaSuccess)
+        return SSD_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
