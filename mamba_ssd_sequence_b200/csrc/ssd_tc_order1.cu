@@ -642,7 +642,10 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (progress) {
                     idle_since = 0;
                     spins = 0;
-                } else if ((++spins & 255u) == 0) {
+                } else {
+                    __nanosleep(32);  // nothing ready: leave the issue slots to the compute groups
+                }
+                if (!progress && (++spins & 63u) == 0) {
                     const uint64_t now = globaltimer_ns();
                     if (idle_since == 0) idle_since = now;
                     if (*abort_flag || now - idle_since > wait_ns) {
@@ -760,15 +763,24 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 pk[2 * e4 + 1] = pack_bf16x2(p1.x, p1.y);
                             }
                         } else {
-                            const float *vfk = misc->vf[gi][slot];
+                            const float4 *a4p = reinterpret_cast<const float4 *>(&acs[k0]);
+                            const float4 *v4p = reinterpret_cast<const float4 *>(&misc->vf[gi][slot][k0]);
 #pragma unroll
-                            for (int e = 0; e < 32; e += 2) {
-                                const int j = k0 + e;
-                                float p0 = sv[e] * ex2_approx(ai - acs[j]) * vfk[j];
-                                float p1 = sv[e + 1] * ex2_approx(ai - acs[j + 1]) * vfk[j + 1];
-                                if (j > ir) p0 = 0.0f;
-                                if (j + 1 > ir) p1 = 0.0f;
-                                pk[e >> 1] = pack_bf16x2(p0, p1);
+                            for (int e4 = 0; e4 < 8; ++e4) {
+                                const float4 a4 = a4p[e4], v4 = v4p[e4];
+                                const int j = k0 + 4 * e4;
+                                const float2 f0 = __fmul2_rn(make_float2(ex2_approx(ai - a4.x), ex2_approx(ai - a4.y)),
+                                                             make_float2(v4.x, v4.y));
+                                const float2 f1 = __fmul2_rn(make_float2(ex2_approx(ai - a4.z), ex2_approx(ai - a4.w)),
+                                                             make_float2(v4.z, v4.w));
+                                float2 p0 = __fmul2_rn(make_float2(sv[4 * e4], sv[4 * e4 + 1]), f0);
+                                float2 p1 = __fmul2_rn(make_float2(sv[4 * e4 + 2], sv[4 * e4 + 3]), f1);
+                                if (j > ir) p0.x = 0.0f;
+                                if (j + 1 > ir) p0.y = 0.0f;
+                                if (j + 2 > ir) p1.x = 0.0f;
+                                if (j + 3 > ir) p1.y = 0.0f;
+                                pk[2 * e4] = pack_bf16x2(p0.x, p0.y);
+                                pk[2 * e4 + 1] = pack_bf16x2(p1.x, p1.y);
                             }
                         }
                     }
