@@ -505,7 +505,11 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nc = N / C;
     // number of tiles this CTA processes
-    const int my_tiles = (int)blockIdx.x < n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    // a contiguous range of tiles per CTA: the row blocks of a chunk (and the
+    // chunks of a head) follow one another on one SM, so key blocks a later
+    // tile shares with an earlier one are still in L2
+    const int tile0 = (int)((long long)blockIdx.x * n_tiles / gridDim.x);
+    const int my_tiles = (int)((long long)(blockIdx.x + 1) * n_tiles / gridDim.x) - tile0;
 
     if (tid == 0) {
         for (int i = 0; i < K::STAGES; ++i) {
@@ -545,7 +549,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             pdl_wait();  // hin (state pass) and everything before it are visible
             int i = 0;
             for (; i < my_tiles; ++i) {
-                const int t = blockIdx.x + i * gridDim.x;
+                const int t = tile0 + i;
                 const int st = i % K::STAGES;
                 if (i >= K::STAGES &&
                     !mbar_wait_abortable(&misc->stage_empty[st], ((i / K::STAGES) - 1) & 1, abort_flag, wait_ns)) {
@@ -588,7 +592,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // ---- Y = P V for tile next_pv, one 128-key block at a time
                 if (next_pv < next_s) {
                     const int i = next_pv, gi = i % NG, tb = i & 1, st = i % K::STAGES;
-                    const TileIdx x = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
+                    const TileIdx x = tile_idx<C>(tile0 + i, nc);
                     const int nkb = x.rb + 1;
                     if (mbar_test(&misc->p_full[gi][pv_kb], np[gi][pv_kb] & 1)) {
                         ++np[gi][pv_kb];
@@ -616,7 +620,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     const bool buf_free = jp < 0 || mbar_test(&misc->ep_done[jp & 1], (jp >> 1) & 1);
                     if (buf_free && mbar_test(&misc->stage_full[st], (j / K::STAGES) & 1)) {
                         tc_fence_after();
-                        const TileIdx x = tile_idx<C>(blockIdx.x + j * gridDim.x, nc);
+                        const TileIdx x = tile_idx<C>(tile0 + j, nc);
                         const int nkb = x.rb + 1;
                         const int sb = j % K::NSB;
                         const uint32_t sp = sbase + st * K::STAGE;
@@ -680,7 +684,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         auto fetch = [&](int i) -> Raw {
             Raw x{0.0f, 1.0f, make_float4(0.f, 0.f, 0.f, 0.f)};
             if (i >= my_tiles) return x;
-            const TileIdx ti = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
+            const TileIdx ti = tile_idx<C>(tile0 + i, nc);
             if (ct < 128 * (ti.rb + 1)) {
                 const size_t key = (size_t)ti.bh * N + (size_t)ti.c * C + ct;
                 x.acs = __ldg(acs_in + key);
@@ -695,7 +699,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         pdl_wait();  // acs (chunk-state kernel) is visible
         Raw raw_next = fetch(gi);
         for (int i = gi; i < my_tiles; i += NG) {
-            const TileIdx x = tile_idx<C>(blockIdx.x + i * gridDim.x, nc);
+            const TileIdx x = tile_idx<C>(tile0 + i, nc);
             const int nkb = x.rb + 1;
             const int sb = i % K::NSB, tb = i & 1, slot = (i / NG) & 1;
             const Raw raw = raw_next;
