@@ -367,35 +367,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
         "r"(v[15])
         : "memory");
 }
-// 32 lanes x 8 consecutive 32-bit columns (store).
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-        : "memory");
-}
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) {
     uint32_t u[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(v[i]);
     tmem_st16(taddr, u);
-}
-// 16 lanes x 64 consecutive 32-bit columns (eight repetitions of the
-// 16x256b pattern).  Thread t of the warp holds lanes (base + t/4) and
-// (base + t/4 + 8); in repetition g, columns 8g + 2(t%4) and 8g + 2(t%4) + 1:
-// v[4g + 0] = (lane t/4, col 8g + 2(t%4)), v[4g + 1] = (lane t/4, col + 1),
-// v[4g + 2] = (lane t/4 + 8, col 8g + 2(t%4)), v[4g + 3] = (lane t/4 + 8, col + 1).
-__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(
-            taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
-        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
-        "r"(v[29]), "r"(v[30]), "r"(v[31])
-        : "memory");
 }
 // 32 lanes x 4 consecutive 32-bit columns (store).
 __device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3) {
@@ -428,25 +404,9 @@ __device__ __forceinline__ void tmem_wait_st() {
 __device__ __forceinline__ uint32_t sw128_chunk(uint32_t row, uint32_t ch) {
     return row * 128u + (((ch ^ (row & 7u)) & 7u) << 4);
 }
-// The same for tiles with 64-byte rows (64-byte swizzle: chunk ^= (row / 2) % 4)
-// and 32-byte rows (32-byte swizzle: chunk ^= (row / 4) % 2).
+// The same for tiles with 64-byte rows (64-byte swizzle: chunk ^= (row / 2) % 4).
 __device__ __forceinline__ uint32_t sw64_chunk(uint32_t row, uint32_t ch) {
     return row * 64u + (((ch ^ (row >> 1)) & 3u) << 4);
-}
-__device__ __forceinline__ uint32_t sw32_chunk(uint32_t row, uint32_t ch) {
-    return row * 32u + (((ch ^ (row >> 2)) & 1u) << 4);
-}
-
-// One lane of the (converged) warp: true on exactly one lane.  Issuing a
-// tensor-core or TMA instruction from an elected lane of a converged warp,
-// rather than from a branch on the lane index, keeps the operands the whole
-// warp computed in uniform registers.
-__device__ __forceinline__ bool elect_one() {
-    uint32_t p;
-    asm volatile(
-        "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n"
-        : "=r"(p));
-    return p != 0;
 }
 
 // ------------------------------------------------- inter-CTA flags in global memory
