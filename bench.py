@@ -68,13 +68,17 @@ def load_peaks():
 
 
 # DRAM bytes of one call, dram__bytes_read.sum + dram__bytes_write.sum summed
-# over the path's kernels, from the ncu captures summarised under profiles/
-# (taken on the kernels in this tree; a workload without a capture of the
-# current kernels reports null).
+# over the path's kernels, each captured by ncu with caches flushed before it
+# (the captures summarised under profiles/, taken on the kernels in this tree;
+# a workload without a capture of the current kernels reports null).
 DRAM_TRAFFIC = {
-    # chunk states 34.10 MB + state pass 0.02 MB + chunk outputs 25.80 MB,
-    # captured without cache flushes, as the kernels run in a call
-    "order1-bf16-B4H16N2048d64-c128": 59_925_402,
+    # chunk states 34.11 MB + state pass 16.79 MB + chunk outputs 59.31 MB
+    "order1-bf16-B4H16N2048d64-c128": 110_209_536,
+    # chunk states 664.2 MB + state pass 169.1 MB + chunk outputs 1128.6 MB
+    "order1-bf16-B1H32N65536d64-c256": 1_961_835_520,
+    # one launch
+    "order2-bf16-B4H16N4096d32-c64": 51_727_360,
+    "order2-bf16-B2H8N16384d64-c64": 122_112_000,
 }
 
 
