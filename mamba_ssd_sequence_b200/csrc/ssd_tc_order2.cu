@@ -30,12 +30,12 @@
 // The (q . k)^2 of the quadratic part and (q (x) q) . (k (x) k) of the state
 // part are the same inner product (Algorithm 5 against Algorithm 6).
 //
-// Roles (608 threads): warp 0 TMA; warp 1 MMA issue; warps 2-9 the state
-// team (slabs 0, 2 and slabs 1, 3: state conversion and scaling, Fk, z);
-// warps 10-13 the query team (Fq, P); warps 14-17 the output team (partials,
-// reduction across the head's CTAs, output); warp 18 the decay warp (kernel
-// (a): the chunk's decay, key weights and value discretisation, one chunk
-// ahead).  Every slab has a buffer of its own in each ring, so a slab's
+// Roles (576 threads): warp 0 the decay warp (kernel (a): the chunk's decay,
+// key weights and value discretisation, one chunk ahead; it also requests the
+// Q, K, V tiles); warp 1 MMA issue; warps 2-9 the state team (slabs 0, 2 and
+// slabs 1, 3: state conversion and scaling, Fk, z); warps 10-13 the query team
+// (Fq, P); warps 14-17 the output team (partials, reduction across the head's
+// CTAs, output).  Every slab has a buffer of its own in each ring, so a slab's
 // preparation for chunk c waits only for that slab's products of chunk c - 1.
 // Options: a per-token log-decay and value discretisation (Algorithm 4; V is
 // scaled by dt in shared memory, the normaliser and the residual use the raw
@@ -68,8 +68,7 @@ constexpr int kQ1T = 128;       // query team: warps 10-13
 constexpr int kQ2T = 128;       // output team: warps 14-17
 constexpr int kQ1W0 = (64 + kSTT) / 32;
 constexpr int kQ2W0 = kQ1W0 + kQ1T / 32;
-constexpr int kDW = kQ2W0 + kQ2T / 32;           // decay warp
-constexpr int kThreads = (kDW + 1) * 32;
+constexpr int kThreads = kQ2W0 * 32 + kQ2T;      // warp 0 decay and TMA, warp 1 MMA, the teams
 constexpr uint32_t kSw128 = 2, kSw64 = 4;        // descriptor swizzle modes
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t kHalf1 = 16u << 16;           // lane offset of the second M = 64 tile
@@ -271,31 +270,143 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tmem = misc->tmem_base;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
+        // ------------------------------------------------------------ decay warp and TMA
+        // kernel (a): chunk-local inclusive cumsum of the log-decay (log2 units),
+        // the chunk total, the key weights wk[a][j / 2] = bf16 pair of
+        // 2^(lam - acs_j) k_ja, and V <- diag(dt) V under value discretisation.
+        // The same warp requests the chunks' Q, K, V tiles: a chunk's tiles
+        // before its decay step needs them (waiting for their stage if it must),
+        // and the next chunks' whenever their stage is already free.
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            int issued = 0;
-            for (int c = 0; c < nc; ++c) {
-                const int st = c % kStages;
-                if (c >= kStages &&
-                    !mbar_wait_abortable(&misc->stage_empty[st], ((c / kStages) - 1) & 1, abort_flag, wait_ns)) {
-                    timeout(10);
-                    break;
+        }
+        int issued = 0;  // chunks whose tiles have been requested
+        // requests tiles for chunks issued .. upto; waits for a busy stage only
+        // when `block` (false: stops at the first busy one)
+        auto request = [&](int upto, bool block) -> bool {
+            while (issued <= upto && issued < nc) {
+                const int st = issued % kStages;
+                if (issued >= kStages) {
+                    const uint32_t par = ((issued / kStages) - 1) & 1;
+                    if (block) {
+                        const bool good = mbar_wait_abortable(&misc->stage_empty[st], par, abort_flag, wait_ns);
+                        if (!__all_sync(0xffffffffu, good)) return false;
+                    } else if (!__shfl_sync(0xffffffffu, (int)mbar_test(&misc->stage_empty[st], par), 0)) {
+                        return true;
+                    }
                 }
-                uint8_t *dst = smem + K::OFF_STAGE + st * K::STAGE;
-                const int r = row0 + c * kC;
-                mbar_arrive_expect_tx(&misc->stage_full[st], K::STAGE);
-                tma_load_2d(dst, &tm_q, 0, r, &misc->stage_full[st]);
-                tma_load_2d(dst + K::TILE, &tm_k, 0, r, &misc->stage_full[st]);
-                tma_load_2d(dst + 2 * K::TILE, &tm_v, 0, r, &misc->stage_full[st]);
+                if (lane == 0) {
+                    uint8_t *dst = smem + K::OFF_STAGE + st * K::STAGE;
+                    const int r = row0 + issued * kC;
+                    mbar_arrive_expect_tx(&misc->stage_full[st], K::STAGE);
+                    tma_load_2d(dst, &tm_q, 0, r, &misc->stage_full[st]);
+                    tma_load_2d(dst + K::TILE, &tm_k, 0, r, &misc->stage_full[st]);
+                    tma_load_2d(dst + 2 * K::TILE, &tm_v, 0, r, &misc->stage_full[st]);
+                }
+                __syncwarp();
                 ++issued;
             }
-            // copies still in flight after an abort land before the CTA exits (bounded)
-            for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
-                mbar_wait_bounded(&misc->stage_full[c % kStages], (c / kStages) & 1);
+            return true;
+        };
+        const float A2 = log_decay ? 0.0f : -expf(A_log[h]) * kLog2e;
+        const float bias = dt_bias ? dt_bias[h] : 0.0f;  // given whenever dt is used
+        const float *dsrc = log_decay ? log_decay : dt_p;
+        const bool vdt_own = value_dt && log_decay;  // the dt projection, when it is not dsrc
+        float2 dnext = make_float2(0.f, 0.f), vnext = make_float2(0.f, 0.f);
+        if (nc > 0) {
+            dnext = *reinterpret_cast<const float2 *>(dsrc + (size_t)row0 + 2 * lane);
+            if (vdt_own) vnext = *reinterpret_cast<const float2 *>(dt_p + (size_t)row0 + 2 * lane);
         }
+        bool ok = request(kStages - 1, true);
+        for (int c = 0; ok && c < nc; ++c) {
+            const int st = c % kStages;
+            if (!(ok = request(c, true))) break;
+            const float2 dv = dnext, vv = vdt_own ? vnext : dnext;
+            if (c + 1 < nc) {
+                dnext = *reinterpret_cast<const float2 *>(dsrc + (size_t)row0 + (size_t)(c + 1) * kC + 2 * lane);
+                if (vdt_own) vnext = *reinterpret_cast<const float2 *>(dt_p + (size_t)row0 + (size_t)(c + 1) * kC + 2 * lane);
+            }
+            // tokens 2 lane and 2 lane + 1
+            const float a0 = log_decay ? dv.x * kLog2e : A2 * softplus_f(dv.x + bias);
+            const float a1 = log_decay ? dv.y * kLog2e : A2 * softplus_f(dv.y + bias);
+            float incl = a0 + a1;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const float lam = __shfl_sync(0xffffffffu, incl, 31);
+            if (c >= 2) {
+                ok = mbar_wait_abortable(&misc->decay_free[c & 1], ((c >> 1) - 1) & 1, abort_flag, wait_ns);
+                if (!__all_sync(0xffffffffu, ok)) break;
+            }
+            misc->acs2[c & 1][2 * lane] = incl - a1;
+            misc->acs2[c & 1][2 * lane + 1] = incl;
+            if (value_dt) {
+                misc->vfac[2 * lane] = softplus_f(vv.x + bias);
+                misc->vfac[2 * lane + 1] = softplus_f(vv.y + bias);
+            }
+            if (lane == 0) misc->lam2[c & 1] = lam;
+            ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag, wait_ns);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            __syncwarp();
+            uint8_t *sK = smem + K::OFF_STAGE + st * K::STAGE + K::TILE;
+            uint8_t *sV = sK + K::TILE;
+            const float *acs = misc->acs2[c & 1];
+            uint32_t *wk = reinterpret_cast<uint32_t *>(smem + K::OFF_WK) + (c & 1) * K::NA * 32;
+            // K^T pairs and key weights: lane l holds token pair (2l, 2l + 1); for
+            // every column b, kT[b][l] = bf16 pair (k_2l,b, k_2l+1,b), and for the
+            // CTA's a, wk[a][l] = bf16 pair (2^(lam - acs_2l) k_2l,a, same for 2l + 1)
+            {
+                const int j = 2 * lane;
+                const float w0 = ex2_approx(lam - acs[j]), w1 = ex2_approx(lam - acs[j + 1]);
+                uint32_t *kT = reinterpret_cast<uint32_t *>(smem + K::OFF_KT) + (c & 1) * D * 32;
+#pragma unroll 2
+                for (int ch = 0; ch < D / 8; ++ch) {
+                    const uint4 r0 = *reinterpret_cast<const uint4 *>(sK + swz<RB>(j, ch));
+                    const uint4 r1 = *reinterpret_cast<const uint4 *>(sK + swz<RB>(j + 1, ch));
+                    const uint32_t a0[4] = {r0.x, r0.y, r0.z, r0.w}, a1[4] = {r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int b = 8 * ch + e;
+                        const uint32_t lo = (e & 1) ? (a0[e >> 1] >> 16) : (a0[e >> 1] & 0xFFFFu);
+                        const uint32_t hi = (e & 1) ? (a1[e >> 1] & 0xFFFF0000u) : (a1[e >> 1] << 16);
+                        kT[b * 32 + ((((lane >> 2) ^ b) & 7) << 2) + (lane & 3)] = lo | hi;
+                        const int al = b - (int)rank * K::NA;
+                        if (al >= 0 && al < K::NA)
+                            wk[al * 32 + lane] = pack_bf16x2(w0 * __uint_as_float(lo << 16), w1 * __uint_as_float(hi));
+                    }
+                }
+            }
+            if (value_dt) {
+                // value discretisation: V <- diag(dt) V in place, before any product reads it
+                constexpr int CPR = D / 8;  // 16-byte chunks per row
+                for (int t = lane; t < kC * CPR; t += 32) {
+                    const int r = t / CPR, ch = t % CPR;
+                    uint4 *pv = reinterpret_cast<uint4 *>(sV + swz<RB>(r, ch));
+                    const float f = misc->vfac[r];
+                    const float2 f2 = make_float2(f, f);
+                    const uint4 x = *pv;
+                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 y = __fmul2_rn(bf2_to_f2(w[e]), f2);
+                        w[e] = pack_bf16x2(y.x, y.y);
+                    }
+                    *pv = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(&misc->decay_ready[c & 1]);
+            mbar_arrive(&misc->stage_empty[st]);
+            request(c + kStages, false);
+        }
+        if (!ok) timeout(50);
+        // copies still in flight after an abort land before the CTA exits (bounded)
+        for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+            mbar_wait_bounded(&misc->stage_full[c % kStages], (c / kStages) & 1);
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -601,7 +712,7 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mbar_arrive(&misc->stage_empty[st]);
         }
         if (!ok) timeout(30);
-    } else if (warp < kDW) {
+    } else {
         // ------------------------------------------------------------ output team
         const int q2 = tid - kQ2W0 * 32;             // 0..127
         const int qq = warp & 3;
@@ -813,103 +924,6 @@ tc_order2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
         }
         if (failed && q2 == 0) timeout(40);
-    } else {
-        // ------------------------------------------------------------ decay warp
-        // kernel (a): chunk-local inclusive cumsum of the log-decay (log2 units),
-        // the chunk total, the key weights wk[a][j / 2] = bf16 pair of
-        // 2^(lam - acs_j) k_ja, and V <- diag(dt) V under value discretisation
-        const float A2 = log_decay ? 0.0f : -expf(A_log[h]) * kLog2e;
-        const float bias = dt_bias ? dt_bias[h] : 0.0f;  // given whenever dt is used
-        const float *dsrc = log_decay ? log_decay : dt_p;
-        const bool vdt_own = value_dt && log_decay;  // the dt projection, when it is not dsrc
-        float2 dnext = make_float2(0.f, 0.f), vnext = make_float2(0.f, 0.f);
-        if (nc > 0) {
-            dnext = *reinterpret_cast<const float2 *>(dsrc + (size_t)row0 + 2 * lane);
-            if (vdt_own) vnext = *reinterpret_cast<const float2 *>(dt_p + (size_t)row0 + 2 * lane);
-        }
-        bool ok = true;
-        for (int c = 0; c < nc; ++c) {
-            const int st = c % kStages;
-            const float2 dv = dnext, vv = vdt_own ? vnext : dnext;
-            if (c + 1 < nc) {
-                dnext = *reinterpret_cast<const float2 *>(dsrc + (size_t)row0 + (size_t)(c + 1) * kC + 2 * lane);
-                if (vdt_own) vnext = *reinterpret_cast<const float2 *>(dt_p + (size_t)row0 + (size_t)(c + 1) * kC + 2 * lane);
-            }
-            // tokens 2 lane and 2 lane + 1
-            const float a0 = log_decay ? dv.x * kLog2e : A2 * softplus_f(dv.x + bias);
-            const float a1 = log_decay ? dv.y * kLog2e : A2 * softplus_f(dv.y + bias);
-            float incl = a0 + a1;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            const float lam = __shfl_sync(0xffffffffu, incl, 31);
-            if (c >= 2) {
-                ok = mbar_wait_abortable(&misc->decay_free[c & 1], ((c >> 1) - 1) & 1, abort_flag, wait_ns);
-                if (!__all_sync(0xffffffffu, ok)) break;
-            }
-            misc->acs2[c & 1][2 * lane] = incl - a1;
-            misc->acs2[c & 1][2 * lane + 1] = incl;
-            if (value_dt) {
-                misc->vfac[2 * lane] = softplus_f(vv.x + bias);
-                misc->vfac[2 * lane + 1] = softplus_f(vv.y + bias);
-            }
-            if (lane == 0) misc->lam2[c & 1] = lam;
-            ok = mbar_wait_abortable(&misc->stage_full[st], (c / kStages) & 1, abort_flag, wait_ns);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            __syncwarp();
-            uint8_t *sK = smem + K::OFF_STAGE + st * K::STAGE + K::TILE;
-            uint8_t *sV = sK + K::TILE;
-            const float *acs = misc->acs2[c & 1];
-            uint32_t *wk = reinterpret_cast<uint32_t *>(smem + K::OFF_WK) + (c & 1) * K::NA * 32;
-            // K^T pairs and key weights: lane l holds token pair (2l, 2l + 1); for
-            // every column b, kT[b][l] = bf16 pair (k_2l,b, k_2l+1,b), and for the
-            // CTA's a, wk[a][l] = bf16 pair (2^(lam - acs_2l) k_2l,a, same for 2l + 1)
-            {
-                const int j = 2 * lane;
-                const float w0 = ex2_approx(lam - acs[j]), w1 = ex2_approx(lam - acs[j + 1]);
-                uint32_t *kT = reinterpret_cast<uint32_t *>(smem + K::OFF_KT) + (c & 1) * D * 32;
-#pragma unroll 2
-                for (int ch = 0; ch < D / 8; ++ch) {
-                    const uint4 r0 = *reinterpret_cast<const uint4 *>(sK + swz<RB>(j, ch));
-                    const uint4 r1 = *reinterpret_cast<const uint4 *>(sK + swz<RB>(j + 1, ch));
-                    const uint32_t a0[4] = {r0.x, r0.y, r0.z, r0.w}, a1[4] = {r1.x, r1.y, r1.z, r1.w};
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int b = 8 * ch + e;
-                        const uint32_t lo = (e & 1) ? (a0[e >> 1] >> 16) : (a0[e >> 1] & 0xFFFFu);
-                        const uint32_t hi = (e & 1) ? (a1[e >> 1] & 0xFFFF0000u) : (a1[e >> 1] << 16);
-                        kT[b * 32 + ((((lane >> 2) ^ b) & 7) << 2) + (lane & 3)] = lo | hi;
-                        const int al = b - (int)rank * K::NA;
-                        if (al >= 0 && al < K::NA)
-                            wk[al * 32 + lane] = pack_bf16x2(w0 * __uint_as_float(lo << 16), w1 * __uint_as_float(hi));
-                    }
-                }
-            }
-            if (value_dt) {
-                // value discretisation: V <- diag(dt) V in place, before any product reads it
-                constexpr int CPR = D / 8;  // 16-byte chunks per row
-                for (int t = lane; t < kC * CPR; t += 32) {
-                    const int r = t / CPR, ch = t % CPR;
-                    uint4 *pv = reinterpret_cast<uint4 *>(sV + swz<RB>(r, ch));
-                    const float f = misc->vfac[r];
-                    const float2 f2 = make_float2(f, f);
-                    const uint4 x = *pv;
-                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 y = __fmul2_rn(bf2_to_f2(w[e]), f2);
-                        w[e] = pack_bf16x2(y.x, y.y);
-                    }
-                    *pv = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-                fence_proxy_async_smem();
-            }
-            mbar_arrive(&misc->decay_ready[c & 1]);
-            mbar_arrive(&misc->stage_empty[st]);
-        }
-        if (!ok) timeout(50);
     }
 
     __syncwarp();
