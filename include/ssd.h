@@ -293,7 +293,8 @@ int ssd_decode_step(const void *q, const void *k, const void *v,
  * Causal depthwise convolution over tokens with optional SiLU, the prologue
  * Q, K, V = SiLU(conv_1d(h W_QKV)) of 2Mamba2Furious Algorithm 3 and the
  * window-2 convolution conv_1d(q_t, q_{t-1}) of its Algorithm 6 page.  Apply
- * it to each of q, k, v before ssd_fwd (it is not fused into the operator).
+ * it to each of q, k, v before ssd_fwd, or call ssd_fwd_conv(), which fuses
+ * it into the order-1 tensor-core path.
  *   x      device, [B, H, N, d_h], element type `dtype` (pre-convolution)
  *   w      device, [H*d_h, width] fp32; w[c][j] multiplies token t - j of
  *          channel c = h*d_h + channel (j = 0 is the current token)
@@ -308,6 +309,51 @@ int ssd_decode_step(const void *q, const void *k, const void *v,
  */
 int ssd_conv1d(const void *x, const float *w, const float *bias, int B, int H, int N, int d_h,
                int width, int silu, int dtype, void *out, void *stream);
+
+/* Taps of the convolution prologue of ssd_fwd_conv(), one set per input. */
+typedef struct {
+    const float *w[3];    /* for q, k, v: device, [H*d_h, width] fp32, as w of ssd_conv1d() */
+    const float *bias[3]; /* device, [H*d_h] fp32, or NULL */
+    int width;            /* 1..4 (the pages use 2) */
+    int silu;             /* nonzero: SiLU after each convolution */
+} ssd_conv_params;
+
+/*
+ * Bytes of device workspace ssd_fwd_conv() needs: the operator's
+ * (ssd_workspace_bytes_ex(..., flags, 0)) plus room for the convolved q, k,
+ * v.  0 for invalid arguments.
+ */
+size_t ssd_fwd_conv_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk,
+                                    int flags);
+
+/*
+ * The operator with its convolution prologue, 2Mamba2Furious Algorithm 3
+ * (Q, K, V = SiLU(conv_1d(h W_QKV))) and the window-2 conv_1d(q_t, q_{t-1})
+ * of its Algorithm 6 page:
+ *   q = act(conv(xq)), k = act(conv(xk)), v = act(conv(xv)),
+ * each exactly as ssd_conv1d() computes it (rounded to `dtype`), then
+ * ssd_fwd_ex(q, k, v, ...) with the remaining arguments.
+ *   xq, xk, xv  device, [B, H, N, d_h], `dtype`, the activations before the
+ *               convolution, 16-byte aligned
+ *   conv        host pointer to the taps (w, bias: 4-byte aligned)
+ *   workspace   at least ssd_fwd_conv_workspace_bytes(...) bytes; the
+ *               convolved q, k, v are left in its last three
+ *               B*H*N*d_h-element blocks (each rounded up to 256 bytes)
+ * On the order-1 tensor-core path at chunk 128 (bf16, d_h = 64) the
+ * convolution is fused: the chunk-state kernel reads the raw tiles, convolves
+ * them in shared memory with a three-token halo and stores the results, which
+ * the chunk scan reads; the separate convolution passes disappear.  Other
+ * shapes, chunk 256 included, run ssd_conv1d() three times, then the
+ * operator.  The result equals
+ * ssd_conv1d() on each input followed by ssd_fwd_ex(), bit for bit.  Errors
+ * as ssd_fwd_ex(), plus SSD_ERR_NULL for missing taps and SSD_ERR_SHAPE for
+ * a width outside 1..4.
+ */
+int ssd_fwd_conv(const void *xq, const void *xk, const void *xv, const ssd_conv_params *conv,
+                 const float *dt_p, const float *A_log, const float *dt_bias, const float *D,
+                 const float *log_decay, int B, int H, int N, int d_h, int dtype, int order,
+                 int normalize, int chunk, int flags, void *out, void *workspace,
+                 size_t workspace_bytes, void *stream);
 
 /*
  * Test hook for the device-side failure detection; the pages have no

@@ -34,6 +34,12 @@ class SSDError(RuntimeError):
         super().__init__(f"{where}: {status_str(code)} (code {code})")
 
 
+class ConvParams(ctypes.Structure):
+    """include/ssd.h ssd_conv_params: the taps of the convolution prologue."""
+    _fields_ = [("w", ctypes.c_void_p * 3), ("bias", ctypes.c_void_p * 3), ("width", ctypes.c_int),
+                ("silu", ctypes.c_int)]
+
+
 def load_library():
     """Load libssd.so (ctypes) and declare the C signatures.  Raises if the
     library has not been built."""
@@ -62,6 +68,10 @@ def load_library():
     lib.ssd_decode_step.restype = ci
     lib.ssd_conv1d.argtypes = [vp] * 3 + [ci] * 7 + [vp, vp]
     lib.ssd_conv1d.restype = ci
+    lib.ssd_fwd_conv_workspace_bytes.argtypes = [ci] * 8
+    lib.ssd_fwd_conv_workspace_bytes.restype = sz
+    lib.ssd_fwd_conv.argtypes = [vp, vp, vp, ctypes.POINTER(ConvParams)] + [vp] * 5 + [ci] * 9 + [vp, vp, sz, vp]
+    lib.ssd_fwd_conv.restype = ci
     lib.ssd_fwd_host.argtypes = [vp] * 7 + [ci] * 8 + [vp] + [vp] * 8 + [vp, sz, vp]
     lib.ssd_fwd_host.restype = ci
     lib.ssd_chunk_cumsum.argtypes = [vp] * 3 + [ci] * 4 + [vp, vp, vp]
@@ -293,6 +303,48 @@ def ssd_status_from_workspace(workspace, stream=None) -> int:
     """Synchronise and read the device status left in the workspace."""
     return int(load_library().ssd_status_from_workspace(_ptr(workspace),
                                                         _stream_handle(stream)))
+
+
+def ssd_fwd_conv_workspace_bytes(B: int, H: int, N: int, d_h: int, dtype: int, order: int, chunk: int,
+                                 flags: int = 0) -> int:
+    return int(load_library().ssd_fwd_conv_workspace_bytes(B, H, N, d_h, dtype, order, chunk, flags))
+
+
+def ssd_fwd_conv(xq, xk, xv, w, bias, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk: int,
+                 silu: bool = True, out=None, workspace=None, stream=None, log_decay=None, value_dt: bool = False):
+    """The operator with its convolution prologue (include/ssd.h, ssd_fwd_conv):
+    q, k, v = SiLU(conv(xq)), SiLU(conv(xk)), SiLU(conv(xv)), then ssd_fwd.
+
+    xq, xk, xv: [B, H, N, d_h] CUDA tensors (before the convolution); w: three
+    [H*d_h, width] float32 tensors (for q, k, v); bias: three [H*d_h] float32
+    tensors or None (the tuple or its entries).  Other arguments as ssd_fwd.
+    Returns `out`."""
+    import torch
+    B, H, N, d = xq.shape
+    dt = _dtype_code(xq)
+    if out is None:
+        out = torch.empty_like(xq)
+    flags = SSD_VALUE_DT if value_dt else 0
+    if workspace is None:
+        nbytes = ssd_fwd_conv_workspace_bytes(B, H, N, d, dt, order, chunk, flags)
+        if nbytes == 0:
+            raise ValueError("invalid ssd arguments")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=xq.device)
+    biases = bias if bias is not None else (None, None, None)
+    cp = ConvParams()
+    for i in range(3):
+        cp.w[i] = _ptr(w[i])
+        cp.bias[i] = _ptr(biases[i])
+    cp.width = int(w[0].shape[1])
+    if any(int(t.shape[1]) != cp.width for t in w):
+        raise ValueError("the three tap tensors must have the same width")
+    cp.silu = int(bool(silu))
+    rc = load_library().ssd_fwd_conv(
+        _ptr(xq), _ptr(xk), _ptr(xv), ctypes.byref(cp), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
+        _ptr(log_decay), B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk), flags,
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _check(rc, "ssd_fwd_conv")
+    return out
 
 
 def ssd_conv1d(x, w, bias=None, silu: bool = True, out=None, stream=None):

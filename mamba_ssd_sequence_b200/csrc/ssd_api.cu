@@ -95,7 +95,8 @@ int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, c
                const float *dt_bias, const float *D, const float *log_decay, int B, int H, int N,
                int d_h, int dtype, int order, int normalize, int chunk, int flags, const float *h0,
                const float *z0, float *h_out, float *z_out, void *out, void *workspace,
-               size_t workspace_bytes, void *stream, int dbg_skip, unsigned long long wait_ns) {
+               size_t workspace_bytes, void *stream, int dbg_skip, unsigned long long wait_ns,
+               const ConvParams *conv = nullptr) {
     if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
     const int value_dt = (flags & SSD_VALUE_DT) ? 1 : 0;
     if (!q || !k || !v || !out) return SSD_ERR_NULL;
@@ -120,6 +121,22 @@ int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, c
               workspace_bytes, static_cast<cudaStream_t>(stream)};
     a.dbg_skip = dbg_skip;
     a.wait_ns = wait_ns;
+    if (conv) {
+        // q, k, v are the workspace buffers for the convolved activations:
+        // the order-1 tensor-core path at chunk 128 computes them inside its
+        // chunk-state kernel; the other paths run the standalone convolution
+        // first
+        if (p.path == PATH_TC_ORDER1 && tc_order1_fuses_conv(chunk)) {
+            a.conv = conv;
+        } else {
+            const void *dst[3] = {q, k, v};
+            for (int i = 0; i < 3; ++i) {
+                rc = ssd_conv1d(conv->x[i], conv->w[i], conv->bias[i], B, H, N, d_h, conv->width, conv->silu,
+                                dtype, const_cast<void *>(dst[i]), stream);
+                if (rc != SSD_OK) return rc;
+            }
+        }
+    }
     switch (p.path) {
     case PATH_TC_ORDER1: return launch_tc_order1(a, p);
     case PATH_TC_ORDER2: return launch_tc_order2(a, p);
@@ -159,6 +176,48 @@ int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,
     return ssd_fwd_state(q, k, v, dt_p, A_log, dt_bias, D, log_decay, B, H, N, d_h, dtype, order,
                          normalize, chunk, flags, nullptr, nullptr, nullptr, nullptr, out, workspace,
                          workspace_bytes, stream);
+}
+
+static size_t act_bytes(int B, int H, int N, int d_h, int dtype) {
+    return align_up((size_t)B * H * N * d_h * (dtype == SSD_F32 ? 4 : 2), 256);
+}
+
+size_t ssd_fwd_conv_workspace_bytes(int B, int H, int N, int d_h, int dtype, int order, int chunk,
+                                    int flags) {
+    const size_t base = ssd_workspace_bytes_ex(B, H, N, d_h, dtype, order, chunk, flags, 0);
+    return base ? base + 3 * act_bytes(B, H, N, d_h, dtype) : 0;
+}
+
+int ssd_fwd_conv(const void *xq, const void *xk, const void *xv, const ssd_conv_params *conv,
+                 const float *dt_p, const float *A_log, const float *dt_bias, const float *D,
+                 const float *log_decay, int B, int H, int N, int d_h, int dtype, int order,
+                 int normalize, int chunk, int flags, void *out, void *workspace,
+                 size_t workspace_bytes, void *stream) {
+    if (!xq || !xk || !xv || !conv || !out) return SSD_ERR_NULL;
+    if (!conv->w[0] || !conv->w[1] || !conv->w[2]) return SSD_ERR_NULL;
+    if (conv->width < 1 || conv->width > 4) return SSD_ERR_SHAPE;
+    if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
+    int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
+    if (rc != SSD_OK) return rc;
+    const void *x16[] = {xq, xk, xv};
+    for (const void *p : x16)
+        if (!aligned16(p)) return SSD_ERR_ALIGN;
+    for (int i = 0; i < 3; ++i)
+        if ((reinterpret_cast<uintptr_t>(conv->w[i]) & 3u) || (reinterpret_cast<uintptr_t>(conv->bias[i]) & 3u))
+            return SSD_ERR_ALIGN;
+    if (!workspace) return SSD_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
+    const size_t need = ssd_fwd_conv_workspace_bytes(B, H, N, d_h, dtype, order, chunk, flags);
+    if (need == 0) return SSD_ERR_SHAPE;
+    if (workspace_bytes < need) return SSD_ERR_WORKSPACE;
+    // the convolved q, k, v sit after the operator's own workspace
+    const size_t act = act_bytes(B, H, N, d_h, dtype);
+    uint8_t *qc = static_cast<uint8_t *>(workspace) + (need - 3 * act);
+    const ConvParams cp{{xq, xk, xv}, {conv->w[0], conv->w[1], conv->w[2]},
+                        {conv->bias[0], conv->bias[1], conv->bias[2]}, conv->width, conv->silu ? 1 : 0};
+    return fwd_common(qc, qc + act, qc + 2 * act, dt_p, A_log, dt_bias, D, log_decay, B, H, N, d_h, dtype,
+                      order, normalize, chunk, flags, nullptr, nullptr, nullptr, nullptr, out, workspace,
+                      need - 3 * act, stream, -1, 0, &cp);
 }
 
 size_t ssd_decode_workspace_bytes(int B, int H, int d_h, int order) {

@@ -15,6 +15,7 @@
 
 #include "ptx.cuh"
 #include "ssd_internal.h"
+#include "ssd_math.cuh"
 
 namespace ssd {
 namespace {
@@ -112,7 +113,7 @@ conv1d_kernel(const T *__restrict__ x, const float *__restrict__ w, const float 
         }
         if (silu) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] = __fdividef(acc[e], 1.0f + __expf(-acc[e]));
+            for (int e = 0; e < 8; ++e) acc[e] = silu_fast(acc[e]);
         }
         store8(out + ((size_t)bhrow * N + t0 + k) * d + c0, acc);
     }

@@ -12,6 +12,16 @@
 namespace ssd {
 
 // Arguments of one forward call after validation.
+// The causal depthwise convolution (+ SiLU) that produces q, k, v from the
+// raw activations x (the prologue Q, K, V = SiLU(conv_1d(h W_QKV))): w and
+// bias per input as for ssd_conv1d().
+struct ConvParams {
+    const void *x[3];     // raw q, k, v: [B, H, N, d_h]
+    const float *w[3];    // [H*d_h, width]
+    const float *bias[3]; // [H*d_h] or NULL
+    int width, silu;
+};
+
 struct FwdArgs {
     const void *q, *k, *v;
     const float *dt_p, *A_log, *dt_bias, *D;
@@ -29,6 +39,10 @@ struct FwdArgs {
     // nanoseconds (0: the default of one second)
     int dbg_skip = -1;
     unsigned long long wait_ns = 0;
+    // with the convolution fused (order-1 tensor-core path): q, k, v above
+    // are the workspace buffers that receive the convolved activations, which
+    // the chunk-state kernel computes from conv->x and stores for the scan
+    const ConvParams *conv = nullptr;
 };
 
 // Device status block at the start of every workspace: status code (an
@@ -73,6 +87,7 @@ int launch_tc_order2(const FwdArgs &a, const Plan &p);
 bool tc_order2_supports(int B, int H, int N, int d, int dtype, int chunk);
 size_t tc_order2_workspace(int B, int H, int N, int d, int chunk);
 int launch_tc_order1(const FwdArgs &a, const Plan &p);
+bool tc_order1_fuses_conv(int chunk);
 bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);
 void tc_order1_layout(int B, int H, int N, int chunk, Plan *p);
 

@@ -27,4 +27,9 @@ __device__ __forceinline__ float softplus_fast(float x) {
     return fmaxf(x, 0.0f) + u * p;
 }
 
+// SiLU of a convolution output, u / (1 + e^-u) with the fast exponential and
+// division.  The standalone convolution and the one fused into the order-1
+// chunk-state kernel both use it, so the two give the same bits.
+__device__ __forceinline__ float silu_fast(float u) { return __fdividef(u, 1.0f + __expf(-u)); }
+
 }  // namespace ssd

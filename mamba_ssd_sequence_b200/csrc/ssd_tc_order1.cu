@@ -31,6 +31,7 @@
 
 #include "ptx.cuh"
 #include "ssd_internal.h"
+#include "ssd_math.cuh"
 
 namespace ssd {
 namespace {
@@ -69,52 +70,130 @@ __device__ void set_timeout(DeviceStatus *status, int where, int *abort_flag) {
 //   others work, which hides most of each chunk's latency chain.
 // U is stored transposed, U^T[n][k] (value index n, feature index k), which
 // is the K-major layout the output kernel's MMA takes for the state.
+// With the convolution prologue fused (CV), the stages hold the raw q, k, v
+// tiles; the group convolves them in place (conv_tile), stores the results
+// for the scan, and writes K' into the Q slot once Q's store has read it.
 // =====================================================================
 constexpr int kStateGroup = 128;
 
-template <int C>
+template <int C, bool CV>
 struct StateCfg {
     static constexpr int NG = C == 128 ? 4 : 2;
     static constexpr int THREADS = 64 + NG * kStateGroup;
-    static constexpr int STAGES = C == 128 ? 6 : 3;
-    static constexpr uint32_t STAGE = 2 * C * kRowB;  // K then V
+    static constexpr int STAGES = CV ? (C == 128 ? 4 : 2) : (C == 128 ? 6 : 3);
+    static constexpr uint32_t TILE = C * kRowB;
+    static constexpr uint32_t STAGE = (CV ? 3 : 2) * TILE;  // K, V [, Q]
     static constexpr uint32_t MISC_OFF = STAGES * STAGE;
     static constexpr uint32_t MISC_BYTES = 4 * NG * C + 1024;
     static constexpr uint32_t SMEM = MISC_OFF + MISC_BYTES + 1024;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <int C>
+template <int C, bool CV>
 struct StateMisc {
-    static constexpr int NG = StateCfg<C>::NG;
+    static constexpr int NG = StateCfg<C, CV>::NG;
     float wk[NG][C];  // per group: 2^(lam - acs_j) per key
     float wtot[NG][4];
-    uint64_t stage_full[StateCfg<C>::STAGES], stage_empty[StateCfg<C>::STAGES];
+    uint64_t stage_full[StateCfg<C, CV>::STAGES], stage_empty[StateCfg<C, CV>::STAGES];
     uint64_t kp_full[NG], u_full[NG], u_free[NG];
     uint64_t drain;
     uint32_t tmem;
     int abort_flag;
 };
-static_assert(sizeof(StateMisc<128>) <= StateCfg<128>::MISC_BYTES, "misc block");
-static_assert(sizeof(StateMisc<256>) <= StateCfg<256>::MISC_BYTES, "misc block");
+static_assert(sizeof(StateMisc<128, false>) <= StateCfg<128, false>::MISC_BYTES, "misc block");
+static_assert(sizeof(StateMisc<256, false>) <= StateCfg<256, false>::MISC_BYTES, "misc block");
+static_assert(sizeof(StateMisc<128, true>) <= StateCfg<128, true>::MISC_BYTES, "misc block");
+static_assert(sizeof(StateMisc<256, true>) <= StateCfg<256, true>::MISC_BYTES, "misc block");
 
+// Raw inputs and taps of the fused convolution (see ConvParams).
+struct ConvTaps {
+    const __nv_bfloat16 *x[3];
+    const float *w[3], *bias[3];
+    int width, silu;
+};
+
+// The causal depthwise convolution (+ SiLU) of one C-row bf16 tile, in place
+// in the 128-byte swizzle of its TMA box.  Lane l of warp gw of the 128-thread
+// group owns the 4-byte word l of each row (channels 2 l, 2 l + 1) in rows
+// [gw C/4, (gw + 1) C/4), so a warp reads and writes whole rows.  Every thread
+// first reads its taps and the three rows before its range (another warp's
+// rows, or, for the first warp, the three tokens before the chunk from global
+// memory: zero at the start of a head); after the group's barrier it walks its
+// own rows in order, eight loads ahead, so every tap sees unconvolved values.
+// The arithmetic is the standalone convolution's (bias, then one fused
+// multiply-add per tap from j = 0, then silu_fast), so the two agree bit for
+// bit.
 template <int C>
-__global__ void __launch_bounds__(StateCfg<C>::THREADS, 1)
+__device__ __forceinline__ void conv_tile(uint8_t *tile, const __nv_bfloat16 *xraw, const float *w,
+                                          const float *bias, int width, int silu, int h, bool head_start,
+                                          size_t row0, int gt, int bar) {
+    constexpr int R = C / 4;  // rows per warp
+    const int wd = gt & 31, r0 = (gt >> 5) * R;
+    auto word = [&](int r) {
+        return reinterpret_cast<uint32_t *>(tile + r * kRowB + ((((wd >> 2) ^ (r & 7)) & 7) << 4) + (wd & 3) * 4);
+    };
+    uint32_t hb[3];  // rows r0 - 3, r0 - 2, r0 - 1
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int r = r0 - 3 + i;
+        if (r >= 0) {
+            hb[i] = *word(r);
+        } else if (!head_start) {
+            hb[i] = __ldg(reinterpret_cast<const uint32_t *>(xraw + (row0 + r) * kD) + wd);
+        } else {
+            hb[i] = 0u;
+        }
+    }
+    const int c = h * kD + 2 * wd;
+    const float2 bs = bias ? make_float2(__ldg(bias + c), __ldg(bias + c + 1)) : make_float2(0.0f, 0.0f);
+    float2 wr[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        wr[j] = j < width ? make_float2(__ldg(w + (size_t)c * width + j), __ldg(w + (size_t)(c + 1) * width + j))
+                          : make_float2(0.0f, 0.0f);
+    named_bar_sync(bar, kStateGroup);
+    float2 x1 = bf2_to_f2(hb[2]), x2 = bf2_to_f2(hb[1]), x3 = bf2_to_f2(hb[0]);  // x[r-1], x[r-2], x[r-3]
+#pragma unroll 1
+    for (int i0 = 0; i0 < R; i0 += 8) {
+        uint32_t xs[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xs[k] = *word(r0 + i0 + k);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float2 xc = bf2_to_f2(xs[k]);
+            float2 acc = __ffma2_rn(wr[0], xc, bs);
+            if (width > 1) acc = __ffma2_rn(wr[1], x1, acc);
+            if (width > 2) acc = __ffma2_rn(wr[2], x2, acc);
+            if (width > 3) acc = __ffma2_rn(wr[3], x3, acc);
+            if (silu) acc = make_float2(silu_fast(acc.x), silu_fast(acc.y));
+            *word(r0 + i0 + k) = pack_bf16x2(acc.x, acc.y);
+            x3 = x2;
+            x2 = x1;
+            x1 = xc;
+        }
+    }
+    fence_proxy_async_smem();  // the TMA store of the tile and the MMA read it
+}
+
+template <int C, bool CV>
+__global__ void __launch_bounds__(StateCfg<C, CV>::THREADS, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_u,
+                   const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_xq,
+                   const __grid_constant__ CUtensorMap tm_sq, const __grid_constant__ CUtensorMap tm_sk,
+                   const __grid_constant__ CUtensorMap tm_sv, const ConvTaps cv,
                    const float *__restrict__ dt_p, const float *__restrict__ A_log,
                    const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int value_dt,
                    int H, int N, int n_chunks, float *__restrict__ acs_out, float *__restrict__ vfac_out,
                    float *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status, int dbg_skip,
                    unsigned long long wait_ns) {
-    using K = StateCfg<C>;
+    using K = StateCfg<C, CV>;
     constexpr int NG = K::NG;
     constexpr int KP = C / 128;  // keys per thread in the decay scan
     pdl_launch_dependents();  // the state pass waits for this grid before it reads anything
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    StateMisc<C> *misc = reinterpret_cast<StateMisc<C> *>(smem + K::MISC_OFF);
+    StateMisc<C, CV> *misc = reinterpret_cast<StateMisc<C, CV> *>(smem + K::MISC_OFF);
     const volatile int *abort_flag = &misc->abort_flag;
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -155,6 +234,12 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
             prefetch_tmap(&tm_u);
+            if (CV) {
+                prefetch_tmap(&tm_xq);
+                prefetch_tmap(&tm_sq);
+                prefetch_tmap(&tm_sk);
+                prefetch_tmap(&tm_sv);
+            }
             int i = 0;
             for (int t = blockIdx.x; t < n_chunks; t += gridDim.x, ++i) {
                 const int st = i % K::STAGES;
@@ -170,7 +255,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
                 for (int b = 0; b < C / 128; ++b) {
                     tma_load_2d(sp + b * kBox, &tm_k, 0, row + 128 * b, &misc->stage_full[st]);
-                    tma_load_2d(sp + C * kRowB + b * kBox, &tm_v, 0, row + 128 * b, &misc->stage_full[st]);
+                    tma_load_2d(sp + K::TILE + b * kBox, &tm_v, 0, row + 128 * b, &misc->stage_full[st]);
+                    if (CV) tma_load_2d(sp + 2 * K::TILE + b * kBox, &tm_xq, 0, row + 128 * b, &misc->stage_full[st]);
                 }
             }
             for (int j = i > K::STAGES ? i - K::STAGES : 0; j < i; ++j)
@@ -188,10 +274,11 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 if (use >= 1 && !(ok = mbar_wait_abortable(&misc->u_free[ub], (use - 1) & 1, abort_flag, wait_ns))) break;
                 tc_fence_after();
                 const uint32_t sp = sbase + st * K::STAGE;
+                const uint32_t kp = sp + (CV ? 2 * K::TILE : 0u);  // K' (in the Q slot with the convolution)
                 // D[n][k] = sum_j v_jn k'_jk: A = V (MN-major), B = K' (MN-major)
 #pragma unroll
                 for (int ks = 0; ks < C / 16; ++ks)
-                    mma_bf16(tmem + 64 * ub, desc_mn(sp + C * kRowB + ks * 2048), desc_mn(sp + ks * 2048), idU,
+                    mma_bf16(tmem + 64 * ub, desc_mn(sp + K::TILE + ks * 2048), desc_mn(kp + ks * 2048), idU,
                              ks > 0);
                 mma_commit(&misc->u_full[ub]);
                 mma_commit(&misc->stage_empty[st]);
@@ -247,7 +334,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
             for (int e = 0; e < KP; ++e) {
                 const float dt = (value_dt || !log_decay) ? softplus_f(raw.dt[e] + raw.bias) : 0.0f;
-                run += log_decay ? raw.ld[e] * kLog2e : A2 * dt;
+                // one explicit fused multiply-add, so every instantiation of
+                // this kernel rounds the decay the same way
+                run = log_decay ? fmaf(raw.ld[e], kLog2e, run) : fmaf(A2, dt, run);
                 a[e] = run;
                 vf[e] = value_dt ? dt : 1.0f;
             }
@@ -281,20 +370,48 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 break;
             }
             uint8_t *sk = smem + st * K::STAGE;
+            uint8_t *skp = sk;  // K'
+            if constexpr (CV) {
+                // q, k, v = SiLU(conv(x)) in place; each tile goes to the
+                // workspace as soon as it is complete (one bulk group per tile)
+                uint8_t *sv = sk + K::TILE, *sq = sk + 2 * K::TILE;
+                const int h = (t / nc) % H;
+                const bool head_start = (t % nc) == 0;
+                const size_t row0 = (size_t)t * C;
+                conv_tile<C>(sq, cv.x[0], cv.w[0], cv.bias[0], cv.width, cv.silu, h, head_start, row0, gt, bar);
+                conv_tile<C>(sk, cv.x[1], cv.w[1], cv.bias[1], cv.width, cv.silu, h, head_start, row0, gt, bar);
+                if (gt == 0) {  // every thread's q rows are final (the barrier inside the k tile's pass)
+#pragma unroll
+                    for (int b = 0; b < C / 128; ++b) tma_store_2d(&tm_sq, sq + b * kBox, 0, t * C + 128 * b);
+                    bulk_commit_group();
+                }
+                conv_tile<C>(sv, cv.x[2], cv.w[2], cv.bias[2], cv.width, cv.silu, h, head_start, row0, gt, bar);
+                named_bar_sync(bar, kStateGroup);
+                if (gt == 0) {
+#pragma unroll
+                    for (int b = 0; b < C / 128; ++b) {
+                        tma_store_2d(&tm_sk, sk + b * kBox, 0, t * C + 128 * b);
+                        tma_store_2d(&tm_sv, sv + b * kBox, 0, t * C + 128 * b);
+                    }
+                    bulk_commit_group();
+                    bulk_wait_group_read<1>();  // the q tile has been read: K' may overwrite it
+                }
+                named_bar_sync(bar, kStateGroup);
+                skp = sq;
+            }
 #pragma unroll 4
             for (int it = 0; it < C / 16; ++it) {
                 const int j = it * 16 + (gt >> 3);
                 const float wj = misc->wk[gi][j];
                 const float2 w2 = make_float2(wj, wj);
-                uint4 *pp = reinterpret_cast<uint4 *>(sk + j * kRowB) + (gt & 7);
-                const uint4 x = *pp;
+                const uint4 x = *(reinterpret_cast<const uint4 *>(sk + j * kRowB) + (gt & 7));
                 uint32_t wv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
                     const float2 f = __fmul2_rn(bf2_to_f2(wv[q]), w2);
                     wv[q] = pack_bf16x2(f.x, f.y);
                 }
-                *pp = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                *(reinterpret_cast<uint4 *>(skp + j * kRowB) + (gt & 7)) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -318,17 +435,17 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const int n = g * 16 + lane;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    *reinterpret_cast<float4 *>(sk + sw128_chunk(n, q)) =
+                    *reinterpret_cast<float4 *>(skp + sw128_chunk(n, q)) =
                         make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
-                    *reinterpret_cast<float4 *>(sk + 8192 + sw128_chunk(n, q)) =
+                    *reinterpret_cast<float4 *>(skp + 8192 + sw128_chunk(n, q)) =
                         make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
                 }
             }
             fence_proxy_async_smem();
             named_bar_sync(bar, kStateGroup);
             if (gt == 0) {
-                tma_store_2d(&tm_u, sk, 0, t * 64);
-                tma_store_2d(&tm_u, sk + 8192, 32, t * 64);
+                tma_store_2d(&tm_u, skp, 0, t * 64);
+                tma_store_2d(&tm_u, skp + 8192, 32, t * 64);
                 bulk_commit_group();
                 bulk_wait_group_read0();
                 mbar_arrive(&misc->stage_empty[st]);
@@ -912,9 +1029,10 @@ int num_sms() {
     return n;
 }
 
-template <int C>
+template <int C, bool CV>
 int launch_c(const FwdArgs &a, const Plan &p) {
     using K = ScanCfg<C>;
+    using SK = StateCfg<C, CV>;
     const int BH = a.B * a.H, nc = a.N / C;
     const uint64_t rows = (uint64_t)BH * a.N;
     uint8_t *ws = static_cast<uint8_t *>(a.workspace);
@@ -931,8 +1049,25 @@ int launch_c(const FwdArgs &a, const Plan &p) {
         return SSD_ERR_CUDA;
     CUtensorMap tu;
     if (!make_tmap_f32x64(&tu, U, (uint64_t)BH * nc * 64)) return SSD_ERR_CUDA;
+    // With the convolution fused, the chunk-state kernel reads the raw
+    // activations and stores the convolved q, k, v (a.q, a.k, a.v, in the
+    // workspace) through the scan's maps, which the scan then reads.
+    CUtensorMap txq = tk, txk = tk, txv = tv;
+    ConvTaps taps{};
+    if (CV) {
+        if (!make_tmap64(&txq, a.conv->x[0], rows, 128) || !make_tmap64(&txk, a.conv->x[1], rows, 128) ||
+            !make_tmap64(&txv, a.conv->x[2], rows, 128))
+            return SSD_ERR_CUDA;
+        for (int i = 0; i < 3; ++i) {
+            taps.x[i] = static_cast<const __nv_bfloat16 *>(a.conv->x[i]);
+            taps.w[i] = a.conv->w[i];
+            taps.bias[i] = a.conv->bias[i];
+        }
+        taps.width = a.conv->width;
+        taps.silu = a.conv->silu;
+    }
     static std::atomic<uint64_t> attr1{0}, attr3{0};
-    if (!smem_attr_once(chunk_state_kernel<C>, (int)StateCfg<C>::SMEM, attr1) ||
+    if (!smem_attr_once(chunk_state_kernel<C, CV>, (int)SK::SMEM, attr1) ||
         !smem_attr_once(chunk_scan_kernel<C>, (int)K::SMEM, attr3))
         return SSD_ERR_CUDA;
     const int sms = num_sms();
@@ -940,9 +1075,9 @@ int launch_c(const FwdArgs &a, const Plan &p) {
 
     const int n_chunks = BH * nc;
     const unsigned long long wait_ns = a.wait_ns ? a.wait_ns : 1000000000ull;
-    chunk_state_kernel<C><<<n_chunks < sms ? n_chunks : sms, StateCfg<C>::THREADS, StateCfg<C>::SMEM, a.stream>>>(
-        tk, tv, tu, a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N, n_chunks, acs, vfac, U, lam,
-        status, a.dbg_skip, wait_ns);
+    chunk_state_kernel<C, CV><<<n_chunks < sms ? n_chunks : sms, SK::THREADS, SK::SMEM, a.stream>>>(
+        txk, txv, tu, txq, tq, tk, tv, taps, a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N,
+        n_chunks, acs, vfac, U, lam, status, a.dbg_skip, wait_ns);
     // The state pass and the chunk scan are launched as programmatic dependents:
     // their CTAs may start while the previous kernel drains, and each waits
     // (griddepcontrol.wait) before it reads that kernel's results.
@@ -980,6 +1115,12 @@ int launch_c(const FwdArgs &a, const Plan &p) {
 
 }  // namespace
 
+// The convolution prologue is fused at chunk 128.  At chunk 256 only two
+// stages of raw q, k, v tiles fit in shared memory, and the convolution,
+// which then runs on two groups per SM, outlasts the loads: there the
+// standalone convolution followed by the operator is faster.
+bool tc_order1_fuses_conv(int chunk) { return chunk == 128; }
+
 bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk) {
     return dtype == SSD_BF16 && d == kD && (chunk == 128 || chunk == 256) && (long long)B * H * N < (1ll << 31);
 }
@@ -998,7 +1139,8 @@ void tc_order1_layout(int B, int H, int N, int chunk, Plan *p) {
 
 int launch_tc_order1(const FwdArgs &a, const Plan &p) {
     if (a.normalize || a.order != 1) return SSD_ERR_UNSUPPORTED;
-    return a.chunk == 256 ? launch_c<256>(a, p) : launch_c<128>(a, p);
+    if (a.conv) return a.chunk == 128 ? launch_c<128, true>(a, p) : SSD_ERR_UNSUPPORTED;
+    return a.chunk == 256 ? launch_c<256, false>(a, p) : launch_c<128, false>(a, p);
 }
 
 }  // namespace ssd

@@ -194,3 +194,31 @@ def test_conv1d_validation_codes(lib):
     assert cv(width=0) == 2 and cv(width=5) == 2 and cv(d=24) == 2 and cv(N=0) == 2
     assert cv(x=1032) == 6 and cv(w=66) == 6
     assert cv(out=1024 + 256) == 2       # out overlaps x
+
+
+def test_fwd_conv_validation_codes(lib):
+    """ssd_fwd_conv rejects bad taps and arguments on the host; its workspace
+    is the operator's plus three activation blocks."""
+    base = ssd.ssd_workspace_bytes_ex(1, 2, 256, 64, ssd.SSD_BF16, 1, 128, 0, 0)
+    need = ssd.ssd_fwd_conv_workspace_bytes(1, 2, 256, 64, ssd.SSD_BF16, 1, 128)
+    assert base > 0 and need == base + 3 * 2 * 256 * 64 * 2
+    assert ssd.ssd_fwd_conv_workspace_bytes(1, 2, 250, 64, ssd.SSD_BF16, 1, 128) == 0
+
+    def fc(**o):
+        a = dict(xq=16, xk=32, xv=48, w=(64, 80, 96), b=(None, None, None), width=2, silu=1, dt_p=112,
+                 A_log=128, dt_bias=144, B=1, H=2, N=256, d=64, dtype=ssd.SSD_BF16, flags=0, out=160, ws=256,
+                 ws_bytes=need, params=True)
+        a.update(o)
+        cp = ssd.ConvParams()
+        for i in range(3):
+            cp.w[i] = a["w"][i]
+            cp.bias[i] = a["b"][i]
+        cp.width, cp.silu = a["width"], a["silu"]
+        return lib.ssd_fwd_conv(a["xq"], a["xk"], a["xv"], ctypes.byref(cp) if a["params"] else None,
+                                a["dt_p"], a["A_log"], a["dt_bias"], None, None, a["B"], a["H"], a["N"], a["d"],
+                                a["dtype"], 1, 0, 128, a["flags"], a["out"], a["ws"], a["ws_bytes"], None)
+    assert fc(xq=None) == 1 and fc(params=False) == 1 and fc(w=(64, None, 96)) == 1   # SSD_ERR_NULL
+    assert fc(width=0) == 2 and fc(width=5) == 2 and fc(N=250) == 2                    # SSD_ERR_SHAPE
+    assert fc(flags=4) == 11                                                           # SSD_ERR_FLAGS
+    assert fc(xk=40) == 6 and fc(w=(64, 82, 96)) == 6 and fc(b=(None, None, 98)) == 6  # SSD_ERR_ALIGN
+    assert fc(ws=None) == 7 and fc(ws_bytes=need - 1) == 7                             # SSD_ERR_WORKSPACE

@@ -63,3 +63,36 @@ def test_prologue_then_operator():
     ref = oracle.ssd_quadratic(ref_in["q"], ref_in["k"], ref_in["v"], x["dt_p"], x["A_log"], x["dt_bias"],
                                x["D"], 1, False)
     assert rel_err(y.float().cpu().numpy().astype(np.float64), ref) <= TOL["bf16"]
+
+
+def test_silu_accuracy():
+    """The convolutions' SiLU (one exponential, a Newton-Raphson reciprocal)
+    against u / (1 + e^-u) in double precision: an identity convolution
+    (width 1, tap 1, no bias) of float32 values spanning [-60, 60] keeps its
+    relative error within a few float32 ulps plus the error of forming the
+    exponent y = |u| log2(e) in float32 (the constant and the product each
+    round by 2^-24 relative, so y is off by up to |y| 2^-23 and 2^y by a
+    relative |y| ln(2) 2^-23 = |u| 2^-23, which any float32 exp of -u
+    carries); far negative inputs give (near) zero."""
+    d = 64
+    u = np.linspace(-60.0, 60.0, 4 * 4096 * d // 4 * 4).astype(np.float32)
+    u = np.concatenate([u, np.array([0.0, 1e-30, -1e-30, 1e-3, -1e-3, 0.5, -0.5], np.float32)])
+    n_tok = -(-u.size // d)
+    x = np.zeros(n_tok * d, np.float32)
+    x[:u.size] = u
+    x = x.reshape(1, 1, n_tok, d)
+    w = np.ones((d, 1), np.float32)
+    y = ssd.ssd_conv1d(torch.from_numpy(x).cuda(), torch.from_numpy(w).cuda(), None, silu=True)
+    torch.cuda.synchronize()
+    got = y.cpu().numpy().reshape(-1)[:u.size].astype(np.float64)
+    ud = u.astype(np.float64)
+    ref = ud / (1.0 + np.exp(-ud))
+    rel = np.abs(got - ref) / np.maximum(np.abs(ref), 1e-30)
+    bound = 4.0 * 2.0 ** -24 + np.abs(ud) * 2.0 ** -23
+    assert np.all(rel <= bound), (rel.max(), ud[np.argmax(rel / bound)])
+    far = np.array([-80.0, -100.0, -1e4], np.float32)
+    xf = np.zeros((1, 1, 1, d), np.float32)
+    xf[0, 0, 0, :3] = far
+    yf = ssd.ssd_conv1d(torch.from_numpy(xf).cuda(), torch.from_numpy(w).cuda(), None, silu=True)
+    torch.cuda.synchronize()
+    assert np.all(np.abs(yf.cpu().numpy()[0, 0, 0, :3]) <= 1e-20)
