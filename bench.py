@@ -437,6 +437,40 @@ def main():
     conv_ms = time_calls(lambda: ssd.ssd_conv1d(dev["q"], cw, None, True, out=cout, stream=stream))
     conv_bytes = 2 * dev["q"].numel() * dev["q"].element_size() + 4 * cw.numel()
 
+    # the operator with its convolution prologue (window 2 + SiLU on q, k,
+    # v), through ssd_fwd_conv (fused into the chunk-state kernel on the
+    # order-1 tensor-core path at chunk 128) against ssd_conv1d x 3 followed by
+    # the operator, on this workload
+    prologue = None
+    if w.order == 1 and w.dtype == "bf16":
+        prng = np.random.default_rng(100 + rank)
+        ptaps = [torch.from_numpy((prng.standard_normal((w.H * w.d, 2)) / 1.5).astype(np.float32)).to(dev_name)
+                 for _ in range(3)]
+        pbias = [torch.from_numpy((0.1 * prng.standard_normal(w.H * w.d)).astype(np.float32)).to(dev_name)
+                 for _ in range(3)]
+        pws = torch.empty(ssd.ssd_fwd_conv_workspace_bytes(w.B, w.H, w.N, w.d, ssd.SSD_BF16, 1, w.chunk),
+                          dtype=torch.uint8, device=dev_name)
+        pc = [torch.empty_like(dev["q"]) for _ in range(3)]
+        pout = torch.empty_like(dev["q"])
+
+        def fused_call():
+            ssd.ssd_fwd_conv(dev["q"], dev["k"], dev["v"], ptaps, pbias, dev["dt_p"], dev["A_log"], dev["dt_bias"],
+                             dev["D"], 1, False, w.chunk, out=pout, workspace=pws, stream=stream)
+
+        def unfused_call():
+            for i, n in enumerate(("q", "k", "v")):
+                ssd.ssd_conv1d(dev[n], ptaps[i], pbias[i], True, out=pc[i], stream=stream)
+            ssd.ssd_fwd(pc[0], pc[1], pc[2], dev["dt_p"], dev["A_log"], dev["dt_bias"], dev["D"], 1, False,
+                        w.chunk, out=pout, workspace=ws, stream=stream)
+
+        fused_ms = time_calls(fused_call)
+        unfused_ms = time_calls(unfused_call)
+        prologue = {"what": "conv1d (width 2, bias) + SiLU on q, k, v, then the operator, on this workload, "
+                            "L2 flushed before each call",
+                    "fused": path == "tc_order1" and w.chunk == 128,
+                    "ms_fused": fused_ms, "ms_conv1d_x3_then_operator": unfused_ms,
+                    "ms_operator_alone": total_ms / args.steps}
+
     # end to end: pinned host inputs -> device -> ssd_fwd -> host, per step
     e2e = None
     if not args.no_e2e:
@@ -513,6 +547,7 @@ def main():
                    "ms_per_call": conv_ms, "bytes_per_call": conv_bytes,
                    "achieved_gbs": conv_bytes / (conv_ms / 1e3) / 1e9,
                    "frac_of_hbm": conv_bytes / (conv_ms / 1e3) / 1e9 / float(peaks["hbm_gbs"])},
+        "conv_prologue": prologue,
         "device_status": status,
         "clocks": clk.summary(),
     }
