@@ -103,7 +103,6 @@ struct StateMisc {
 static_assert(sizeof(StateMisc<128, false>) <= StateCfg<128, false>::MISC_BYTES, "misc block");
 static_assert(sizeof(StateMisc<256, false>) <= StateCfg<256, false>::MISC_BYTES, "misc block");
 static_assert(sizeof(StateMisc<128, true>) <= StateCfg<128, true>::MISC_BYTES, "misc block");
-static_assert(sizeof(StateMisc<256, true>) <= StateCfg<256, true>::MISC_BYTES, "misc block");
 
 // Raw inputs and taps of the fused convolution (see ConvParams).
 struct ConvTaps {
