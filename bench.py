@@ -72,13 +72,13 @@ def load_peaks():
 # (the captures summarised under profiles/, taken on the kernels in this tree;
 # a workload without a capture of the current kernels reports null).
 DRAM_TRAFFIC = {
-    # chunk states 34.11 MB + state pass 16.79 MB + chunk outputs 59.31 MB
-    "order1-bf16-B4H16N2048d64-c128": 110_209_536,
-    # chunk states 664.2 MB + state pass 169.1 MB + chunk outputs 1128.6 MB
-    "order1-bf16-B1H32N65536d64-c256": 1_961_835_520,
+    # chunk states 34.10 MB + state pass 16.79 MB + chunk outputs 59.38 MB
+    "order1-bf16-B4H16N2048d64-c128": 110_275_840,
+    # chunk states 664.0 MB + state pass 169.1 MB + chunk outputs 1129.0 MB
+    "order1-bf16-B1H32N65536d64-c256": 1_962_049_792,
     # one launch
-    "order2-bf16-B4H16N4096d32-c64": 51_727_360,
-    "order2-bf16-B2H8N16384d64-c64": 122_112_000,
+    "order2-bf16-B4H16N4096d32-c64": 51_731_712,
+    "order2-bf16-B2H8N16384d64-c64": 122_030_336,
 }
 
 
