@@ -551,12 +551,18 @@ struct ScanCfg {
     // C = 128 (three stages) stages it over the stage's Q box, which keeps
     // the residual rows at hand in the stage's V box.
     static constexpr bool OUT_SLOT = C == 256;
+    // C = 256 (one compute group): the group runs tile i's P and then tile
+    // i - 1's epilogue, so each tile's P V completes behind the next tile's
+    // P; Z then lives in a TMEM slot per tile parity (see below)
+    static constexpr bool PIPE = C == 256;
     static constexpr uint32_t Y_OFF = STAGES * STAGE;
     static constexpr uint32_t MISC_OFF = Y_OFF + (OUT_SLOT ? NG * kBox : 0);
     static constexpr uint32_t MISC_BYTES = 28 * NG * C + 1024;
     static constexpr uint32_t SMEM = MISC_OFF + MISC_BYTES + 1024;
     // TMEM: C = 128: S' buffers at 0 and 192 (keys at +0, Z at +128);
-    //       C = 256: keys k at 128 (2 - nkb) + k, Z at 256.  Y buffers at 384, 448.
+    //       C = 256: keys k at 128 (2 - nkb) + k, Z of tile j at 256 + 64 (j % 2)
+    //       (a product of its own: the next tile's scores need only this
+    //       tile's P V done, not its epilogue).  Y buffers at 384, 448.
     static constexpr uint32_t COL_Y = 384;
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(STAGE % 1024 == 0, "stage alignment");
@@ -598,8 +604,8 @@ __device__ __forceinline__ uint32_t key_col(int sb, int nkb) {
     return C == 128 ? (uint32_t)sb * 192u : 128u * (uint32_t)(2 - nkb);
 }
 template <int C>
-__device__ __forceinline__ uint32_t z_col(int sb) {
-    return C == 128 ? (uint32_t)sb * 192u + 128u : 256u;
+__device__ __forceinline__ uint32_t z_col(int sb, int j) {
+    return C == 128 ? (uint32_t)sb * 192u + 128u : 256u + 64u * (uint32_t)(j & 1);
 }
 
 template <int C>
@@ -695,6 +701,7 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (lane == 0) {
             constexpr uint32_t idS128 = make_idesc_bf16(128, 128, 0, 0);
             constexpr uint32_t idS192 = make_idesc_bf16(128, 192, 0, 0);
+            constexpr uint32_t idZ = make_idesc_bf16(128, 64, 0, 0);
             constexpr uint32_t idO = make_idesc_bf16(128, 64, 0, 1);
             uint32_t np[NG][K::NKB];
             for (int gi = 0; gi < NG; ++gi)
@@ -729,11 +736,16 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                         progress = true;
                     }
                 }
-                // ---- S' for tile next_s (its TMEM buffer is free once tile next_s - NSB is done)
+                // ---- S' for tile next_s.  C = 128: its TMEM buffer is free once
+                // tile next_s - NSB is done.  C = 256: the key columns once the
+                // previous tile's P V is done, its Z slot once tile next_s - 2 is.
                 if (next_s < my_tiles) {
                     const int j = next_s, st = j % K::STAGES;
                     const int jp = j - K::NSB;  // previous user of the S' buffer
-                    const bool buf_free = jp < 0 || mbar_test(&misc->ep_done[jp & 1], (jp >> 1) & 1);
+                    const bool buf_free =
+                        !K::PIPE ? (jp < 0 || mbar_test(&misc->ep_done[jp & 1], (jp >> 1) & 1))
+                                 : ((j < 1 || mbar_test(&misc->y_full[(j - 1) & 1], ((j - 1) >> 1) & 1)) &&
+                                    (j < 2 || mbar_test(&misc->ep_done[j & 1], ((j - 2) >> 1) & 1)));
                     if (buf_free && mbar_test(&misc->stage_full[st], (j / K::STAGES) & 1)) {
                         tc_fence_after();
                         const TileIdx x = tile_idx<C>(tile0 + j, nc);
@@ -748,12 +760,24 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                                 mma_bf16(tmem + kc, desc_k(sp + K::Q_OFF + ks * 32), desc_k(sp + K::K_OFF + ks * 32),
                                          idS128, ks > 0);
                         }
-                        // last key block and the state readout: B = [K slot NKB - 1 ; hin^T]
                         const uint32_t kl = sp + K::K_OFF + (K::NKB - 1) * kBox;
+                        if (!K::PIPE) {
+                            // last key block and the state readout: B = [K slot NKB - 1 ; hin^T]
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16(tmem + kc + 128 * (nkb - 1), desc_k(sp + K::Q_OFF + ks * 32), desc_k(kl + ks * 32),
-                                     idS192, ks > 0);
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16(tmem + kc + 128 * (nkb - 1), desc_k(sp + K::Q_OFF + ks * 32),
+                                         desc_k(kl + ks * 32), idS192, ks > 0);
+                        } else {
+                            // last key block, then the state readout into the tile's Z slot
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16(tmem + kc + 128 * (nkb - 1), desc_k(sp + K::Q_OFF + ks * 32),
+                                         desc_k(kl + ks * 32), idS128, ks > 0);
+#pragma unroll
+                            for (int ks = 0; ks < 4; ++ks)
+                                mma_bf16(tmem + z_col<C>(sb, j), desc_k(sp + K::Q_OFF + ks * 32),
+                                         desc_k(sp + K::H_OFF + ks * 32), idZ, ks > 0);
+                        }
                         mma_commit(&misc->s_full[sb]);
                         ++next_s;
                         progress = true;
@@ -812,12 +836,92 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
         bool failed = false;
         int pend_st = -1;  // thread ct = 0: stage of an output store not yet waited for
+        auto epilogue = [&](int j) -> bool {
+            const TileIdx x = tile_idx<C>(tile0 + j, nc);
+            const int sb = j % K::NSB, tb = j & 1, slot = (j / NG) & 1;
+            const int ir = 128 * x.rb + r;
+            uint8_t *sp = smem + (j % K::STAGES) * K::STAGE;
+            const float ai = misc->acs[gi][slot][ir];
+        // ---- epilogue of tile j: y = Y + 2^acs_i Z [+ D v], columns [32 hf, 32 hf + 32)
+            // With an output slot the stage may be refilled once P V completes,
+            // so the residual rows v_i (still in L2) are fetched from global
+            // memory while P V runs; otherwise they are read from the V box.
+            uint4 vres[4] = {};
+            if (K::OUT_SLOT && Dres) {
+                const uint4 *vp = reinterpret_cast<const uint4 *>(
+                                      vglob + ((size_t)x.bh * N + (size_t)x.c * C + 128 * x.rb + r) * kD) +
+                                  4 * hf;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) vres[q] = __ldg(vp + q);
+            }
+            bool bad = !mbar_wait_abortable(&misc->y_full[tb], (j >> 1) & 1, abort_flag, wait_ns);
+            // the V box is read below: observe the stage's TMA completion here too
+            // (long complete; the stage cannot be refilled before this group releases it)
+            if (!K::OUT_SLOT)
+                bad = bad || !mbar_wait_abortable(&misc->stage_full[j % K::STAGES], (j / K::STAGES) & 1, abort_flag, wait_ns);
+            if (named_bar_any(bar, 256, bad)) return false;
+            tc_fence_after();
+            const float e = ex2_approx(ai);
+            const float *dh = &misc->dres[gi][slot][hf * 32];
+            // residual v_i: row r of V box rb (this tile's own tokens).  y is
+            // staged in the swizzled layout of the TMA store, over Q (dead since
+            // S' completed) or in the group's slot, whose previous store was
+            // read before this group signalled P of this tile complete.
+            const uint8_t *vrow = sp + K::V_OFF + x.rb * kBox;
+            uint8_t *ytile = K::OUT_SLOT ? smem + K::Y_OFF + gi * kBox : sp + K::Q_OFF;
+            const uint32_t zc = tmem + lane_off + z_col<C>(sb, j) + 32 * hf;
+            const uint32_t yc = tmem + lane_off + K::COL_Y + 64 * tb + 32 * hf;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float yv[16], zv[16];
+                tmem_ld16(yc + 16 * half, yv);
+                tmem_ld16(zc + 16 * half, zv);
+                tmem_wait_ld();
+                if (half == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&misc->ep_done[tb]);
+                }
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int q = 2 * half + q2;
+                    uint32_t wv[4];
+                    uint4 vq = vres[q];
+                    if (!K::OUT_SLOT && Dres) vq = *reinterpret_cast<const uint4 *>(vrow + sw128_chunk(r, 4 * hf + q));
+                    const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w};
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp) {
+                        const int cl = q2 * 8 + 2 * pp;  // column within the half
+                        float y0 = fmaf(e, zv[cl], yv[cl]);
+                        float y1 = fmaf(e, zv[cl + 1], yv[cl + 1]);
+                        if (Dres) {
+                            const float2 vf = bf2_to_f2(vw[pp]);
+                            y0 = fmaf(dh[16 * half + cl], vf.x, y0);
+                            y1 = fmaf(dh[16 * half + cl + 1], vf.y, y1);
+                        }
+                        wv[pp] = pack_bf16x2(y0, y1);
+                    }
+                    *reinterpret_cast<uint4 *>(ytile + sw128_chunk(r, 4 * hf + q)) =
+                        make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                }
+            }
+            // one TMA store per tile; its read of the tile (and, staged over Q,
+            // the stage's release) is settled before the group's next S
+            fence_proxy_async_smem();
+            named_bar_sync(bar, 256);
+            if (ct == 0) {
+                tma_store_2d(&tm_out, ytile, 0, x.bh * N + x.c * C + 128 * x.rb);
+                bulk_commit_group();
+                pend_st = j % K::STAGES;
+            }
+            return true;
+        };
+
         pdl_wait();  // acs (chunk-state kernel) is visible
         Raw raw_next = fetch(gi);
         for (int i = gi; i < my_tiles; i += NG) {
             const TileIdx x = tile_idx<C>(tile0 + i, nc);
             const int nkb = x.rb + 1;
-            const int sb = i % K::NSB, tb = i & 1, slot = (i / NG) & 1;
+            const int sb = i % K::NSB, slot = (i / NG) & 1;
             const Raw raw = raw_next;
             raw_next = fetch(i + NG);
             const int ir = 128 * x.rb + r;  // chunk-local row
@@ -910,81 +1014,18 @@ chunk_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tc_fence_before();
                 mbar_arrive(&misc->p_full[gi][kb]);
             }
-            // ---- epilogue: y = Y + 2^acs_i Z [+ D v], columns [32 hf, 32 hf + 32)
-            // With an output slot the stage may be refilled once P V completes,
-            // so the residual rows v_i (still in L2) are fetched from global
-            // memory while P V runs; otherwise they are read from the V box.
-            uint4 vres[4] = {};
-            if (K::OUT_SLOT && Dres) {
-                const uint4 *vp = reinterpret_cast<const uint4 *>(
-                                      vglob + ((size_t)x.bh * N + (size_t)x.c * C + 128 * x.rb + r) * kD) +
-                                  4 * hf;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) vres[q] = __ldg(vp + q);
-            }
-            bad = !mbar_wait_abortable(&misc->y_full[tb], (i >> 1) & 1, abort_flag, wait_ns);
-            // the V box is read below: observe the stage's TMA completion here too
-            // (long complete; the stage cannot be refilled before this group releases it)
-            if (!K::OUT_SLOT)
-                bad = bad || !mbar_wait_abortable(&misc->stage_full[i % K::STAGES], (i / K::STAGES) & 1, abort_flag, wait_ns);
-            if (named_bar_any(bar, 256, bad)) {
+            if (!K::PIPE) {
+                if (!epilogue(i)) {
+                    failed = true;
+                    break;
+                }
+            } else if (i - NG >= gi && !epilogue(i - NG)) {
                 failed = true;
                 break;
             }
-            tc_fence_after();
-            const float e = ex2_approx(ai);
-            const float *dh = &misc->dres[gi][slot][hf * 32];
-            // residual v_i: row r of V box rb (this tile's own tokens).  y is
-            // staged in the swizzled layout of the TMA store, over Q (dead since
-            // S' completed) or in the group's slot, whose previous store was
-            // read before this group signalled P of this tile complete.
-            const uint8_t *vrow = sp + K::V_OFF + x.rb * kBox;
-            uint8_t *ytile = K::OUT_SLOT ? smem + K::Y_OFF + gi * kBox : sp + K::Q_OFF;
-            const uint32_t zc = tmem + lane_off + z_col<C>(sb) + 32 * hf;
-            const uint32_t yc = tmem + lane_off + K::COL_Y + 64 * tb + 32 * hf;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float yv[16], zv[16];
-                tmem_ld16(yc + 16 * half, yv);
-                tmem_ld16(zc + 16 * half, zv);
-                tmem_wait_ld();
-                if (half == 1) {
-                    tc_fence_before();
-                    mbar_arrive(&misc->ep_done[tb]);
-                }
-#pragma unroll
-                for (int q2 = 0; q2 < 2; ++q2) {
-                    const int q = 2 * half + q2;
-                    uint32_t wv[4];
-                    uint4 vq = vres[q];
-                    if (!K::OUT_SLOT && Dres) vq = *reinterpret_cast<const uint4 *>(vrow + sw128_chunk(r, 4 * hf + q));
-                    const uint32_t vw[4] = {vq.x, vq.y, vq.z, vq.w};
-#pragma unroll
-                    for (int pp = 0; pp < 4; ++pp) {
-                        const int cl = q2 * 8 + 2 * pp;  // column within the half
-                        float y0 = fmaf(e, zv[cl], yv[cl]);
-                        float y1 = fmaf(e, zv[cl + 1], yv[cl + 1]);
-                        if (Dres) {
-                            const float2 vf = bf2_to_f2(vw[pp]);
-                            y0 = fmaf(dh[16 * half + cl], vf.x, y0);
-                            y1 = fmaf(dh[16 * half + cl + 1], vf.y, y1);
-                        }
-                        wv[pp] = pack_bf16x2(y0, y1);
-                    }
-                    *reinterpret_cast<uint4 *>(ytile + sw128_chunk(r, 4 * hf + q)) =
-                        make_uint4(wv[0], wv[1], wv[2], wv[3]);
-                }
-            }
-            // one TMA store per tile; its read of the tile (and, staged over Q,
-            // the stage's release) is settled before the group's next S
-            fence_proxy_async_smem();
-            named_bar_sync(bar, 256);
-            if (ct == 0) {
-                tma_store_2d(&tm_out, ytile, 0, x.bh * N + x.c * C + 128 * x.rb);
-                bulk_commit_group();
-                pend_st = i % K::STAGES;
-            }
         }
+        // the last tile's epilogue (one tile behind)
+        if (K::PIPE && !failed && my_tiles > gi && !epilogue(gi + (my_tiles - 1 - gi) / NG * NG)) failed = true;
         if (ct == 0) bulk_wait_group0();  // every output tile has reached global memory
         if (failed && ct == 0) set_timeout(status, 130, &misc->abort_flag);
     }
