@@ -74,8 +74,8 @@ def load_peaks():
 DRAM_TRAFFIC = {
     # chunk states 34.10 MB + state pass 16.79 MB + chunk outputs 59.38 MB
     "order1-bf16-B4H16N2048d64-c128": 110_275_840,
-    # chunk states 664.0 MB + state pass 169.1 MB + chunk outputs 1129.0 MB
-    "order1-bf16-B1H32N65536d64-c256": 1_962_049_792,
+    # chunk states 664.0 MB + state pass 168.9 MB + chunk outputs 1127.2 MB
+    "order1-bf16-B1H32N65536d64-c256": 1_960_182_528,
     # one launch
     "order2-bf16-B4H16N4096d32-c64": 51_731_712,
     "order2-bf16-B2H8N16384d64-c64": 122_030_336,
