@@ -95,9 +95,11 @@ def test_fused_prologue_equals_unfused_bitwise(chunk, opt):
 
 
 @pytest.mark.parametrize("order,normalize,dtype,d,chunk", [(2, True, "bf16", 32, 64), (1, False, "f32", 32, 64),
-                                                           (2, False, "bf16", 64, 64)])
-def test_unfused_paths_match_oracle(order, normalize, dtype, d, chunk):
-    """Shapes off the fused path run the standalone convolution, then the operator."""
+                                                           (2, False, "bf16", 64, 64), (2, True, "bf16", 64, 64),
+                                                           (1, False, "bf16", 64, 256)])
+def test_other_paths_match_oracle(order, normalize, dtype, d, chunk):
+    """Shapes off the fused path (order 2, fp32, order 1 at chunk 256) run the
+    standalone convolution, then the operator."""
     B, H, N = 1, 2, 3 * chunk
     x = inputs.make_inputs(B, H, N, d, dtype, seed=95, residual=True)
     w, b = _taps(H, d, 2, 96)
@@ -108,7 +110,29 @@ def test_unfused_paths_match_oracle(order, normalize, dtype, d, chunk):
     assert rel_err(_as64(y), ref) <= TOL[dtype]
 
 
-@pytest.mark.parametrize("name", ["order1-bf16-B4H16N2048d64-c128", "order1-bf16-B1H32N65536d64-c256"])
+@pytest.mark.parametrize("d,normalize,opt", [(32, True, "none"), (64, True, "none"), (32, False, "value_dt"),
+                                             (64, True, "log_decay")])
+def test_order2_prologue_equals_unfused_bitwise(d, normalize, opt):
+    """Order 2 through ssd_fwd_conv (the standalone convolution, then the
+    order-2 tensor-core kernel) gives the same bits as ssd_conv1d x 3
+    followed by the operator."""
+    B, H, N = 1, 3, 5 * 64
+    x = inputs.make_inputs(B, H, N, d, "bf16", seed=93, residual=True)
+    dev = to_device(x, "bf16")
+    w, b = _taps(H, d, 2, 94)
+    kw = {}
+    if opt == "log_decay":
+        rng = np.random.default_rng(95)
+        kw["log_decay"] = torch.from_numpy(-rng.uniform(0.0, 0.3, size=(B, H, N)).astype(np.float32)).cuda()
+    if opt == "value_dt":
+        kw["value_dt"] = True
+    yf = _run_fused(dev, w, b, 2, normalize, 64, True, **kw)
+    yu = _run_unfused(dev, w, b, 2, normalize, 64, True, **kw)
+    assert torch.equal(yf, yu)
+
+
+@pytest.mark.parametrize("name", ["order1-bf16-B4H16N2048d64-c128", "order1-bf16-B1H32N65536d64-c256",
+                                  "order2-bf16-B4H16N4096d32-c64", "order2-bf16-B2H8N16384d64-c64"])
 def test_fused_prologue_full_size(name):
     """The order-1 workloads at full size with the prologue: sampled rows
     against the oracle, and every output bit against the unfused sequence."""
@@ -116,11 +140,11 @@ def test_fused_prologue_full_size(name):
     x = inputs.make_workload_inputs(wl, seed=0)
     dev = to_device(x, "bf16")
     w, b = _taps(wl.H, wl.d, 2, 97)
-    yf = _run_fused(dev, w, b, 1, False, wl.chunk, True)
-    yu = _run_unfused(dev, w, b, 1, False, wl.chunk, True)
+    yf = _run_fused(dev, w, b, wl.order, wl.normalize, wl.chunk, True)
+    yu = _run_unfused(dev, w, b, wl.order, wl.normalize, wl.chunk, True)
     assert torch.equal(yf, yu)
     rows = sample_rows(wl.N, wl.chunk, seed=3, n_random=8)
     ri = _oracle_inputs(x, w, b, True, "bf16")
-    ref = oracle.ssd_quadratic(ri["q"], ri["k"], ri["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"], 1, False,
-                               rows=rows)
+    ref = oracle.ssd_quadratic(ri["q"], ri["k"], ri["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"], wl.order,
+                               wl.normalize, rows=rows)
     assert rel_err(_as64(yf)[:, :, rows, :], ref) <= TOL["bf16"]
