@@ -72,10 +72,9 @@ def load_peaks():
 # (the captures summarised under profiles/, taken on the kernels in this tree;
 # a workload without a capture of the current kernels reports null).
 DRAM_TRAFFIC = {
-    # chunk states 34.10 MB + state pass 16.79 MB + chunk outputs 59.38 MB
-    "order1-bf16-B4H16N2048d64-c128": 110_275_840,
-    # chunk states 664.0 MB + state pass 168.9 MB + chunk outputs 1127.2 MB
-    "order1-bf16-B1H32N65536d64-c256": 1_960_182_528,
+    # the order-1 workloads: no capture yet of the kernels that store U in bf16
+    "order1-bf16-B4H16N2048d64-c128": None,
+    "order1-bf16-B1H32N65536d64-c256": None,
     # one launch
     "order2-bf16-B4H16N4096d32-c64": 51_731_712,
     "order2-bf16-B2H8N16384d64-c64": 122_030_336,

@@ -6,7 +6,8 @@
 // chunk and one short recurrence over chunk states.  Three launches:
 //   (1) chunk_state_kernel, persistent, one compute group per chunk c of a head:
 //         acs_t = chunk-local inclusive cumsum of A dt (log2 units), lam = acs_{C-1}
-//         U_c   = sum_j 2^(lam - acs_j) k_j v_j^T          (tcgen05, M = N = 64, K = C)
+//         U_c   = sum_j 2^(lam - acs_j) k_j v_j^T          (tcgen05, M = N = 64, K = C;
+//                                                          accumulated in fp32, stored as bf16)
 //   (2) state_pass_kernel: h_{-1} = h0 (or 0), hin_c = bf16(h_{c-1}),
 //         h_c = 2^lam_c h_{c-1} + U_c                      (fp32, elementwise over the 64 x 64 state)
 //         and h_out = h of the last chunk when asked for
@@ -183,7 +184,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                    const float *__restrict__ dt_p, const float *__restrict__ A_log,
                    const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int value_dt,
                    int H, int N, int n_chunks, float *__restrict__ acs_out, float *__restrict__ vfac_out,
-                   float *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status, int dbg_skip,
+                   __nv_bfloat16 *__restrict__ Ut, float *__restrict__ lam_out, DeviceStatus *status, int dbg_skip,
                    unsigned long long wait_ns) {
     using K = StateCfg<C, CV>;
     constexpr int NG = K::NG;
@@ -428,23 +429,22 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&misc->u_free[gi]);
-            // U^T rows n = 16 g + lane, staged over K' (read by the finished
-            // product) as two 64 x 32 fp32 boxes in the 128-byte swizzle
+            // U^T rows n = 16 g + lane, rounded to bf16 and staged over K' (read
+            // by the finished product) as one 64 x 64 box in the 128-byte swizzle
             if (lane < 16) {
                 const int n = g * 16 + lane;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    *reinterpret_cast<float4 *>(skp + sw128_chunk(n, q)) =
-                        make_float4(v0[4 * q], v0[4 * q + 1], v0[4 * q + 2], v0[4 * q + 3]);
-                    *reinterpret_cast<float4 *>(skp + 8192 + sw128_chunk(n, q)) =
-                        make_float4(v1[4 * q], v1[4 * q + 1], v1[4 * q + 2], v1[4 * q + 3]);
+                    const float *v = q < 4 ? v0 + 8 * q : v1 + 8 * (q - 4);
+                    *reinterpret_cast<uint4 *>(skp + sw128_chunk(n, q)) =
+                        make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                                   pack_bf16x2(v[6], v[7]));
                 }
             }
             fence_proxy_async_smem();
             named_bar_sync(bar, kStateGroup);
             if (gt == 0) {
                 tma_store_2d(&tm_u, skp, 0, t * 64);
-                tma_store_2d(&tm_u, skp + 8192, 32, t * 64);
                 bulk_commit_group();
                 bulk_wait_group_read0();
                 mbar_arrive(&misc->stage_empty[st]);
@@ -466,13 +466,13 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // =====================================================================
 template <int kBatch>
 __global__ void __launch_bounds__(256)
-state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __nv_bfloat16 *__restrict__ hin,
+state_pass_kernel(const __nv_bfloat16 *__restrict__ U, const float *__restrict__ lam, __nv_bfloat16 *__restrict__ hin,
                   int nc, const float *__restrict__ h0, float *__restrict__ h_out) {
     pdl_launch_dependents();  // the chunk scan waits for this grid before it reads hin
     pdl_wait();               // U and lam of the chunk-state kernel
     const int bh = blockIdx.x;
     const int e = (blockIdx.y * 256 + threadIdx.x) * 4;  // 4 consecutive entries of the 64 x 64 state
-    const float4 *u = reinterpret_cast<const float4 *>(U + (size_t)bh * nc * 4096 + e);
+    const uint2 *u = reinterpret_cast<const uint2 *>(U + (size_t)bh * nc * 4096 + e);
     uint2 *out = reinterpret_cast<uint2 *>(hin + (size_t)bh * nc * 4096 + e);
     const float *lm = lam + (size_t)bh * nc;
     // the state carried into the sequence (h0 is [k][n]; this thread holds
@@ -487,7 +487,7 @@ state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __
     // (16: a head of up to 16 chunks costs one L2 round trip; 8 for longer
     // heads, which keeps more threads resident)
     for (int c0 = 0; c0 < nc; c0 += kBatch) {
-        float4 ub[kBatch];
+        uint2 ub[kBatch];
         float fb[kBatch];
 #pragma unroll
         for (int j = 0; j < kBatch; ++j) {
@@ -501,10 +501,11 @@ state_pass_kernel(const float *__restrict__ U, const float *__restrict__ lam, __
             if (c0 + j < nc) {
                 const float f = ex2_approx(fb[j]);
                 out[(size_t)(c0 + j) * 1024] = make_uint2(pack_bf16x2(hs.x, hs.y), pack_bf16x2(hs.z, hs.w));
-                hs.x = fmaf(f, hs.x, ub[j].x);
-                hs.y = fmaf(f, hs.y, ub[j].y);
-                hs.z = fmaf(f, hs.z, ub[j].z);
-                hs.w = fmaf(f, hs.w, ub[j].w);
+                const float2 u01 = bf2_to_f2(ub[j].x), u23 = bf2_to_f2(ub[j].y);
+                hs.x = fmaf(f, hs.x, u01.x);
+                hs.y = fmaf(f, hs.y, u01.y);
+                hs.z = fmaf(f, hs.z, u23.x);
+                hs.w = fmaf(f, hs.w, u23.y);
             }
         }
     }
@@ -1043,12 +1044,6 @@ bool make_tmap64(CUtensorMap *m, const void *base, uint64_t rows, uint32_t box_r
     return encode_tmap_2d(m, base, true, 64, rows, 64, box_rows, 128);
 }
 
-// [rows, 64] fp32 row-major tensor written in boxes of 64 rows x 32 columns,
-// 128-byte swizzle.
-bool make_tmap_f32x64(CUtensorMap *m, void *base, uint64_t rows) {
-    return encode_tmap_2d(m, base, false, 64, rows, 32, 64, 128);
-}
-
 // Sets the dynamic shared-memory limit of `fn` once per device.
 template <typename F>
 bool smem_attr_once(F fn, int bytes, std::atomic<uint64_t> &done) {
@@ -1080,7 +1075,7 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     float *lam = reinterpret_cast<float *>(ws + p.lam_off);
     float *acs = reinterpret_cast<float *>(ws + p.acs_off);
     float *vfac = a.value_dt ? reinterpret_cast<float *>(ws + p.vfac_off) : nullptr;
-    float *U = reinterpret_cast<float *>(ws + p.state_off);
+    __nv_bfloat16 *U = reinterpret_cast<__nv_bfloat16 *>(ws + p.state_off);
     __nv_bfloat16 *hin = reinterpret_cast<__nv_bfloat16 *>(ws + p.aux_off);
     CUtensorMap tq, tk, tv, th, to;
     if (!make_tmap64(&tq, a.q, rows, 128) || !make_tmap64(&tk, a.k, rows, 128) ||
@@ -1088,7 +1083,7 @@ int launch_c(const FwdArgs &a, const Plan &p) {
         !make_tmap64(&to, a.out, rows, 128))
         return SSD_ERR_CUDA;
     CUtensorMap tu;
-    if (!make_tmap_f32x64(&tu, U, (uint64_t)BH * nc * 64)) return SSD_ERR_CUDA;
+    if (!make_tmap64(&tu, U, (uint64_t)BH * nc * 64, 64)) return SSD_ERR_CUDA;
     // With the convolution fused, the chunk-state kernel reads the raw
     // activations and stores the convolved q, k, v (a.q, a.k, a.v, in the
     // workspace) through the scan's maps, which the scan then reads.
@@ -1131,9 +1126,9 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c2.attrs = pdl;
     c2.numAttrs = 1;
     const cudaError_t e2 =
-        nc <= 16 ? cudaLaunchKernelEx(&c2, state_pass_kernel<16>, (const float *)U, (const float *)lam, hin, nc, a.h0,
+        nc <= 16 ? cudaLaunchKernelEx(&c2, state_pass_kernel<16>, (const __nv_bfloat16 *)U, (const float *)lam, hin, nc, a.h0,
                                       a.h_out)
-                 : cudaLaunchKernelEx(&c2, state_pass_kernel<8>, (const float *)U, (const float *)lam, hin, nc, a.h0,
+                 : cudaLaunchKernelEx(&c2, state_pass_kernel<8>, (const __nv_bfloat16 *)U, (const float *)lam, hin, nc, a.h0,
                                       a.h_out);
     if (e2 != cudaSuccess)
         return SSD_ERR_CUDA;
@@ -1166,14 +1161,14 @@ bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk) {
 }
 
 // lam (n_chunks floats), acs and vfac (B H N floats each), U (n_chunks x 64
-// x 64 fp32), hin (n_chunks x 64 x 64 bf16)
+// x 64 bf16), hin (n_chunks x 64 x 64 bf16)
 void tc_order1_layout(int B, int H, int N, int chunk, Plan *p) {
     const size_t n = (size_t)B * H * (N / chunk);
     p->lam_off = kStatusBytes;
     p->acs_off = align_up(p->lam_off + n * sizeof(float), 256);
     p->vfac_off = align_up(p->acs_off + (size_t)B * H * N * sizeof(float), 256);
     p->state_off = align_up(p->vfac_off + (size_t)B * H * N * sizeof(float), 256);
-    p->aux_off = align_up(p->state_off + n * 4096 * sizeof(float), 256);
+    p->aux_off = align_up(p->state_off + n * 4096 * 2, 256);
     p->total = align_up(p->aux_off + n * 4096 * 2, 256);
 }
 
