@@ -149,14 +149,28 @@ int ssd_fwd_ex(const void *q, const void *k, const void *v,
                void *stream);
 
 /*
- * ssd_fwd() with the activations in HOST memory: enqueues on `stream` the
- * host-to-device copies of q, k, v, dt_p, A_log, dt_bias and D (when
- * non-NULL) into the caller's device buffers, the forward pass, and the
- * device-to-host copy of the result into out_host.  Host buffers should be
- * pinned (cudaHostAlloc / torch pin_memory) for the copies to be
- * asynchronous.  The d_* buffers are device buffers of the shapes listed for
- * ssd_fwd(); d_D may be NULL only when D_host is NULL.  The call returns once
- * the work is enqueued; synchronise `stream` before reading out_host.
+ * ssd_fwd() with the activations in HOST memory: enqueues the host-to-device
+ * copies of q, k, v, dt_p, A_log, dt_bias and D (when non-NULL) into the
+ * caller's device buffers, the forward pass, and the device-to-host copy of
+ * the result into out_host.  Host buffers should be pinned (cudaHostAlloc /
+ * torch pin_memory) for the copies to be asynchronous.  The d_* buffers are
+ * device buffers of the shapes listed for ssd_fwd(); every d_* but d_D must
+ * be non-NULL, and d_D may be NULL only when D_host is NULL.
+ *
+ * When q, k and v hold 4 MiB or more, the heads go through in up to four
+ * slices (whole batches when B >= 2; ranges of heads starting at multiples of
+ * 4 when B = 1 and H >= 8): a slice's input copies run on a copy stream of
+ * the library while the previous slice's forward pass and output copy run on
+ * `stream`, so the two directions of the host link overlap.  The copy
+ * stream and its events are created on the first such call in a CUDA context
+ * (per context, kept until exit) and wait for the work enqueued on `stream`
+ * before the call; every later step of the call is enqueued on `stream`, so
+ * synchronising `stream` before reading out_host suffices, as for one slice.
+ * Concurrent calls from several host threads in one context are serialised
+ * while they enqueue.  The status word of the workspace
+ * (ssd_status_from_workspace) reports the first slice that failed.
+ * Errors: as ssd_fwd(), checked on the whole problem before anything is
+ * enqueued; SSD_ERR_CUDA when a copy, the copy stream or an event fails.
  */
 int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                  const float *dt_p_host, const float *A_log_host,

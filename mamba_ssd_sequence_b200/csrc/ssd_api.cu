@@ -1,11 +1,45 @@
 // C entry points of libssd.so: argument validation, workspace planning and
 // dispatch to the kernel paths.  The operator and the conventions are
 // documented in include/ssd.h.
+#include <cuda.h>
 #include <cuda_runtime.h>
+
+#include <mutex>
 
 #include "ssd_internal.h"
 
 namespace ssd {
+
+namespace drv {
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
+
+template <typename F>
+F driver_fn(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<F>(p);
+}
+}  // namespace drv
+
+bool current_context_id(unsigned long long *id) {
+    static drv::PfnCtxGetCurrent get_ctx = drv::driver_fn<drv::PfnCtxGetCurrent>("cuCtxGetCurrent");
+    static drv::PfnCtxGetId get_id = drv::driver_fn<drv::PfnCtxGetId>("cuCtxGetId");
+    if (!get_ctx || !get_id) return false;
+    CUcontext ctx = nullptr;
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return false;
+    if (ctx == nullptr) {
+        // no context current on this thread yet: make the runtime's primary
+        // context of the current device current (this allocates nothing)
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return false;
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    }
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -144,6 +178,88 @@ int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, c
     }
 }
 
+// ---- ssd_fwd_host: slices of heads whose copies overlap the previous
+// slice's forward pass and output copy (PCIe carries both directions at once)
+
+constexpr int kMaxHostSlices = 4;
+constexpr size_t kMinPipelinedBytes = 4u << 20;  // below this one slice is as fast
+
+struct HostSlice {
+    int b0, nb, h0, nh;
+};
+struct HostSlices {
+    int n;
+    HostSlice s[kMaxHostSlices];
+};
+
+// Whole batches when B >= 2; for B = 1, ranges of heads that start at a
+// multiple of 4 (A_log, dt_bias and D stay 16-byte aligned).
+HostSlices host_slices(int B, int H, size_t act_bytes) {
+    HostSlices r{};
+    r.n = 1;
+    r.s[0] = HostSlice{0, B, 0, H};
+    if (act_bytes < kMinPipelinedBytes) return r;
+    if (B >= 2) {
+        r.n = B < kMaxHostSlices ? B : kMaxHostSlices;
+        for (int g = 0; g < r.n; ++g) {
+            const int b0 = (int)((long long)B * g / r.n), b1 = (int)((long long)B * (g + 1) / r.n);
+            r.s[g] = HostSlice{b0, b1 - b0, 0, H};
+        }
+    } else if (H >= 8) {
+        const int quads = H / 4;  // whole groups of four heads; the last slice takes the rest
+        r.n = quads < kMaxHostSlices ? quads : kMaxHostSlices;
+        for (int g = 0; g < r.n; ++g) {
+            const int h0 = 4 * (int)((long long)quads * g / r.n);
+            const int h1 = g + 1 == r.n ? H : 4 * (int)((long long)quads * (g + 1) / r.n);
+            r.s[g] = HostSlice{0, 1, h0, h1 - h0};
+        }
+    }
+    return r;
+}
+
+// The copy stream and events of ssd_fwd_host, one set per CUDA context (keyed
+// by the context's ID, which the driver never reuses), created on first use
+// and kept until exit.  The mutex serialises the enqueueing of one call, so
+// that two host threads never interleave their event records.
+struct HostPipe {
+    unsigned long long ctx_id;
+    cudaStream_t copy;
+    cudaEvent_t entry, ready[kMaxHostSlices];
+    std::mutex *mutex;
+};
+constexpr int kPipeSlots = 16;
+HostPipe g_pipes[kPipeSlots] = {};
+int g_pipe_count = 0;
+std::mutex g_pipe_mutex;
+
+const HostPipe *host_pipe() {
+    unsigned long long id = 0;
+    if (!current_context_id(&id)) return nullptr;
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    for (int i = 0; i < g_pipe_count; ++i)
+        if (g_pipes[i].ctx_id == id) return &g_pipes[i];
+    if (g_pipe_count == kPipeSlots) return nullptr;
+    HostPipe p{};
+    p.ctx_id = id;
+    if (cudaStreamCreateWithFlags(&p.copy, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&p.entry, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    for (cudaEvent_t &e : p.ready)
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    p.mutex = new std::mutex;
+    g_pipes[g_pipe_count] = p;
+    return &g_pipes[g_pipe_count++];
+}
+
+// Each slice's forward pass rewrites the status word; the slot after it in
+// the status block keeps the first failure (first: the first slice; last:
+// copy the kept status back into the word ssd_status_from_workspace reads).
+__global__ void keep_status_kernel(DeviceStatus *st, int first, int last) {
+    if (threadIdx.x != 0) return;
+    DeviceStatus *kept = st + 4;  // bytes 64-79 of the 256-byte status block
+    if (first || kept->code == 0) *kept = *st;
+    if (last) *st = *kept;
+}
+
 }  // namespace
 
 extern "C" {
@@ -276,30 +392,68 @@ int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
     if (!q_host || !k_host || !v_host || !dt_p_host || !A_log_host || !dt_bias_host ||
         !out_host)
         return SSD_ERR_NULL;
+    if (!d_q || !d_k || !d_v || !d_dt_p || !d_A_log || !d_dt_bias || !d_out) return SSD_ERR_NULL;
     if (D_host && !d_D) return SSD_ERR_NULL;
     int rc = check_shape(B, H, N, d_h, dtype, order, chunk);
     if (rc != SSD_OK) return rc;
+    {
+        // the whole problem is validated before anything is enqueued
+        Plan p;
+        rc = make_plan(B, H, N, d_h, dtype, order, normalize, chunk, 0, 0, &p);
+        if (rc != SSD_OK) return rc;
+        if (!workspace) return SSD_ERR_WORKSPACE;
+        if (workspace_bytes < p.total) return SSD_ERR_WORKSPACE;
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t elem = dtype == SSD_F32 ? 4 : 2;
-    const size_t act = (size_t)B * H * N * d_h * elem;
-    const size_t tok = (size_t)B * H * N * sizeof(float);
-    const size_t hp = (size_t)H * sizeof(float);
-    struct Copy { void *dst; const void *src; size_t n; } h2d[] = {
-        {d_q, q_host, act}, {d_k, k_host, act}, {d_v, v_host, act}, {d_dt_p, dt_p_host, tok},
-        {d_A_log, A_log_host, hp}, {d_dt_bias, dt_bias_host, hp},
-        {d_D, D_host, (size_t)H * d_h * sizeof(float)}};
-    for (const Copy &c : h2d) {
-        if (!c.src) continue;
-        if (!c.dst) return SSD_ERR_NULL;
-        if (cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    const size_t row_act = (size_t)N * d_h * elem;  // one (b, h) row of q, k, v or out
+    const size_t row_tok = (size_t)N * sizeof(float);
+    const HostSlices sl = host_slices(B, H, (size_t)B * H * row_act);
+    const HostPipe *pipe = sl.n > 1 ? host_pipe() : nullptr;
+    if (sl.n > 1 && !pipe) return SSD_ERR_CUDA;
+    // one stream (the caller's) when there is a single slice; otherwise the
+    // inputs go in on the library's copy stream, after the caller's earlier work
+    cudaStream_t cs = pipe ? pipe->copy : s;
+    std::unique_lock<std::mutex> lock;
+    if (pipe) {
+        lock = std::unique_lock<std::mutex>(*pipe->mutex);
+        if (cudaEventRecord(pipe->entry, s) != cudaSuccess || cudaStreamWaitEvent(cs, pipe->entry, 0) != cudaSuccess)
             return SSD_ERR_CUDA;
     }
-    rc = ssd_fwd(d_q, d_k, d_v, d_dt_p, d_A_log, d_dt_bias, D_host ? d_D : nullptr, B, H, N,
-                 d_h, dtype, order, normalize, chunk, d_out, workspace, workspace_bytes, stream);
-    if (rc != SSD_OK) return rc;
-    if (cudaMemcpyAsync(out_host, d_out, act, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    auto h2d = [&](void *dst, const void *src, size_t n) {
+        return cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, cs) == cudaSuccess;
+    };
+    const size_t hp = (size_t)H * sizeof(float);
+    if (!h2d(d_A_log, A_log_host, hp) || !h2d(d_dt_bias, dt_bias_host, hp) ||
+        (D_host && !h2d(d_D, D_host, (size_t)H * d_h * sizeof(float))))
         return SSD_ERR_CUDA;
-    return SSD_OK;
+    for (int g = 0; g < sl.n; ++g) {
+        const HostSlice &c = sl.s[g];
+        // slice rows (b, h) for b in [b0, b0 + nb), h in [h0, h0 + nh): contiguous
+        // when the slice is whole batches (nh = H) or one batch (nb = 1)
+        const size_t r0 = (size_t)c.b0 * H + c.h0, nr = (size_t)c.nb * c.nh;
+        auto act = [&](const void *base) { return static_cast<const char *>(base) + r0 * row_act; };
+        auto dact = [&](void *base) { return static_cast<char *>(base) + r0 * row_act; };
+        if (!h2d(dact(d_q), act(q_host), nr * row_act) || !h2d(dact(d_k), act(k_host), nr * row_act) ||
+            !h2d(dact(d_v), act(v_host), nr * row_act) ||
+            !h2d(reinterpret_cast<char *>(d_dt_p) + r0 * row_tok,
+                 reinterpret_cast<const char *>(dt_p_host) + r0 * row_tok, nr * row_tok))
+            return SSD_ERR_CUDA;
+        if (pipe && (cudaEventRecord(pipe->ready[g], cs) != cudaSuccess ||
+                     cudaStreamWaitEvent(s, pipe->ready[g], 0) != cudaSuccess))
+            return SSD_ERR_CUDA;
+        rc = ssd_fwd(dact(d_q), dact(d_k), dact(d_v), reinterpret_cast<float *>(reinterpret_cast<char *>(d_dt_p) +
+                                                                                  r0 * row_tok),
+                     d_A_log + c.h0, d_dt_bias + c.h0, D_host ? d_D + (size_t)c.h0 * d_h : nullptr, c.nb, c.nh, N,
+                     d_h, dtype, order, normalize, chunk, dact(d_out), workspace, workspace_bytes, stream);
+        if (rc != SSD_OK) return rc;
+        if (sl.n > 1)  // the first failure among the slices is the one the status word keeps
+            keep_status_kernel<<<1, 32, 0, s>>>(static_cast<DeviceStatus *>(workspace), g == 0, g == sl.n - 1);
+        if (cudaMemcpyAsync(static_cast<char *>(out_host) + r0 * row_act, dact(d_out), nr * row_act,
+                            cudaMemcpyDeviceToHost, s) != cudaSuccess)
+            return SSD_ERR_CUDA;
+    }
+    return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
 int ssd_chunk_cumsum(const float *dt_p, const float *A_log, const float *dt_bias, int B, int H,

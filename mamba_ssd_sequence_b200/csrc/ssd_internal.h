@@ -97,6 +97,11 @@ void tc_order1_layout(int B, int H, int N, int chunk, Plan *p);
 bool encode_tmap_2d(CUtensorMap *m, const void *base, bool bf16, uint64_t cols, uint64_t rows,
                     uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
 
+// The ID of the calling thread's current CUDA context (the driver never
+// reuses one within a process); when no context is current, the current
+// device's primary context is made current first.  False on a driver error.
+bool current_context_id(unsigned long long *id);
+
 // Decode step (ssd_decode.cu).
 size_t decode_workspace(int B, int H, int d, int order);
 int launch_decode(const FwdArgs &a, float *h, float *z);

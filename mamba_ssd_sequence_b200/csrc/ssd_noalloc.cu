@@ -24,9 +24,6 @@ constexpr int kCacheSlots = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-typedef CUresult (*PfnCtxGetCurrent)(CUcontext *);
-typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long *);
-
 struct CacheSlot {
     unsigned long long ctx_id;
     void *ptr;
@@ -35,34 +32,12 @@ CacheSlot g_cache[kCacheSlots] = {};
 int g_cache_next = 0;
 std::mutex g_scratch_mutex;
 
-template <typename F>
-F driver_fn(const char *name) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-        return nullptr;
-    return reinterpret_cast<F>(p);
-}
-
 // Device address of g_noalloc_scratch in the calling thread's current context
 // (nullptr on error).  The first call in a context loads the library's module
 // there if it is not loaded yet.
 void *scratch_for_current_context() {
-    static PfnCtxGetCurrent get_ctx = driver_fn<PfnCtxGetCurrent>("cuCtxGetCurrent");
-    static PfnCtxGetId get_id = driver_fn<PfnCtxGetId>("cuCtxGetId");
-    if (!get_ctx || !get_id) return nullptr;
-    CUcontext ctx = nullptr;
-    if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
-    if (ctx == nullptr) {
-        // no context current on this thread yet: make the runtime's primary
-        // context of the current device current (this allocates nothing)
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return nullptr;
-        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return nullptr;
-    }
     unsigned long long id = 0;
-    if (get_id(ctx, &id) != CUDA_SUCCESS) return nullptr;
+    if (!ssd::current_context_id(&id)) return nullptr;
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     for (const CacheSlot &s : g_cache)
         if (s.ptr != nullptr && s.ctx_id == id) return s.ptr;

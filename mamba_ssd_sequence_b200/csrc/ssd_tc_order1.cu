@@ -464,7 +464,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 // =====================================================================
 // (2) state passing: one thread per 4 state entries of a head
 // =====================================================================
-template <int kBatch>
+constexpr int kPassBatch = 16;  // chunks whose inputs are in flight at once
 __global__ void __launch_bounds__(256)
 state_pass_kernel(const __nv_bfloat16 *__restrict__ U, const float *__restrict__ lam, __nv_bfloat16 *__restrict__ hin,
                   int nc, const float *__restrict__ h0, float *__restrict__ h_out) {
@@ -483,21 +483,20 @@ state_pass_kernel(const __nv_bfloat16 *__restrict__ U, const float *__restrict__
         const float *hp = h0 + (size_t)bh * 4096 + (size_t)k_ * 64 + n_;
         hs = make_float4(hp[0], hp[64], hp[128], hp[192]);
     }
-    // kBatch chunks' inputs are in flight before the dependent updates run
-    // (16: a head of up to 16 chunks costs one L2 round trip; 8 for longer
-    // heads, which keeps more threads resident)
-    for (int c0 = 0; c0 < nc; c0 += kBatch) {
-        uint2 ub[kBatch];
-        float fb[kBatch];
+    // 16 chunks' inputs (bf16 U, 8 bytes a thread) are in flight before the
+    // dependent updates run: a head of up to 16 chunks costs one L2 round trip
+    for (int c0 = 0; c0 < nc; c0 += kPassBatch) {
+        uint2 ub[kPassBatch];
+        float fb[kPassBatch];
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
+        for (int j = 0; j < kPassBatch; ++j) {
             if (c0 + j < nc) {
                 ub[j] = __ldg(u + (size_t)(c0 + j) * 1024);
                 fb[j] = __ldg(lm + c0 + j);
             }
         }
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
+        for (int j = 0; j < kPassBatch; ++j) {
             if (c0 + j < nc) {
                 const float f = ex2_approx(fb[j]);
                 out[(size_t)(c0 + j) * 1024] = make_uint2(pack_bf16x2(hs.x, hs.y), pack_bf16x2(hs.z, hs.w));
@@ -1125,11 +1124,8 @@ int launch_c(const FwdArgs &a, const Plan &p) {
     c2.stream = a.stream;
     c2.attrs = pdl;
     c2.numAttrs = 1;
-    const cudaError_t e2 =
-        nc <= 16 ? cudaLaunchKernelEx(&c2, state_pass_kernel<16>, (const __nv_bfloat16 *)U, (const float *)lam, hin, nc, a.h0,
-                                      a.h_out)
-                 : cudaLaunchKernelEx(&c2, state_pass_kernel<8>, (const __nv_bfloat16 *)U, (const float *)lam, hin, nc, a.h0,
-                                      a.h_out);
+    const cudaError_t e2 = cudaLaunchKernelEx(&c2, state_pass_kernel, (const __nv_bfloat16 *)U, (const float *)lam,
+                                              hin, nc, a.h0, a.h_out);
     if (e2 != cudaSuccess)
         return SSD_ERR_CUDA;
     const int n_tiles = BH * nc * K::NRB;

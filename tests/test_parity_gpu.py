@@ -181,6 +181,37 @@ def test_host_entry_point_matches_device_entry_point():
     assert torch.equal(out_h, ref.cpu())
 
 
+@pytest.mark.parametrize("B,H,N,d,dtype,order,chunk", [
+    (3, 4, 4096, 64, "bf16", 1, 128),   # three slices of whole batches
+    (1, 10, 4096, 64, "bf16", 1, 256),  # one batch: heads [0, 4) and [4, 10)
+    (2, 8, 4096, 32, "bf16", 2, 64),    # order 2 (clusters of two), two slices
+    (2, 8, 2048, 64, "bf16", 2, 64),    # order 2 with the reduction through L2
+    (4, 2, 4096, 64, "f32", 1, 64),     # the SIMT path, four slices
+])
+def test_host_entry_point_in_slices(B, H, N, d, dtype, order, chunk):
+    """Inputs of 4 MiB and more go in by slices of heads, each slice's copies
+    overlapping the previous slice's pass: the same bytes as the device entry
+    point on the whole problem, twice in a row, with a clean status word."""
+    import torch
+    assert B * H * N * d * (2 if dtype == "bf16" else 4) >= 4 << 20
+    x = inputs.make_inputs(B, H, N, d, dtype, seed=11)
+    dev = to_device(x, dtype)
+    norm = order == 2
+    ref = ssd.ssd_fwd(dev["q"], dev["k"], dev["v"], dev["dt_p"], dev["A_log"],
+                      dev["dt_bias"], dev["D"], order, norm, chunk).cpu()
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in dev.items()}
+    scratch = {k: (torch.empty_like(v) if v is not None else None) for k, v in dev.items()}
+    scratch["out"] = torch.empty_like(dev["q"])
+    ws = ssd.alloc_workspace(B, H, N, d, ssd.SSD_BF16 if dtype == "bf16" else ssd.SSD_F32, order, chunk)
+    for _ in range(2):
+        out_h = torch.empty_like(host["q"]).pin_memory()
+        ssd.ssd_fwd_host(host["q"], host["k"], host["v"], host["dt_p"], host["A_log"],
+                         host["dt_bias"], host["D"], order, norm, chunk, out_h, scratch, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h, ref)
+    assert ssd.ssd_status_from_workspace(ws) == 0
+
+
 # --------------------------------------------- full-size workloads, sampled
 @pytest.mark.parametrize("name", inputs.WORKLOAD_ORDER[1:])
 def test_full_size_workload_sampled_rows(name):
