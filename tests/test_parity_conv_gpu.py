@@ -44,6 +44,25 @@ def test_conv1d_matches_oracle(dtype, width, silu, use_bias):
     assert rel_err(got, ref) <= tol
 
 
+@pytest.mark.parametrize("dtype,B,H,N,d,width", [
+    ("f32", 2, 40, 1000, 16, 3),   # 640 tiles of 128 tokens, ragged last tile of each sequence
+    ("bf16", 1, 16, 4096, 64, 2),  # the bench's sequence length
+    ("bf16", 3, 20, 700, 32, 4),
+])
+def test_conv1d_many_tiles_per_cta(dtype, B, H, N, d, width):
+    """More tiles than two per SM: each CTA walks a range of tiles through its
+    two tile buffers, crossing from one head's sequence to the next."""
+    x = inputs.make_inputs(B, H, N, d, dtype, seed=53)
+    w, b = _weights(H, d, width, 53)
+    dev = to_device(x, dtype)
+    y = ssd.ssd_conv1d(dev["q"], torch.from_numpy(w).cuda(), torch.from_numpy(b).cuda(), silu=True)
+    torch.cuda.synchronize()
+    ref = oracle.conv1d(x["q"], w, b, silu=True)
+    got = y.float().cpu().numpy().astype(np.float64)
+    tol = 1e-5 if dtype == "f32" else 2 ** -8
+    assert rel_err(got, ref) <= tol
+
+
 def test_prologue_then_operator():
     """conv1d + SiLU on q, k, v, then the order-1 tensor-core operator, agrees
     with the oracle's prologue followed by the oracle's operator."""
