@@ -72,9 +72,10 @@ def load_peaks():
 # (the captures summarised under profiles/, taken on the kernels in this tree;
 # a workload without a capture of the current kernels reports null).
 DRAM_TRAFFIC = {
-    # the order-1 workloads: no capture yet of the kernels that store U in bf16
-    "order1-bf16-B4H16N2048d64-c128": None,
-    "order1-bf16-B1H32N65536d64-c256": None,
+    # chunk states 34.11 MB + state pass 8.40 MB + chunk outputs 59.47 MB
+    "order1-bf16-B4H16N2048d64-c128": 101_977_344,
+    # chunk states 607.3 MB + state pass 87.1 MB + chunk outputs 1127.6 MB
+    "order1-bf16-B1H32N65536d64-c256": 1_821_930_752,
     # one launch
     "order2-bf16-B4H16N4096d32-c64": 51_731_712,
     "order2-bf16-B2H8N16384d64-c64": 122_030_336,
