@@ -371,13 +371,18 @@ int ssd_fwd_conv(const void *xq, const void *xk, const void *xv, const ssd_conv_
 
 /*
  * Test hook for the device-side failure detection; the pages have no
- * counterpart.  ssd_fwd() with two arguments that only failure tests use:
+ * counterpart.  ssd_fwd() with three arguments that only failure tests use:
  *   skip_publish  >= 0: on the tensor-core paths, one producer inside the
  *                 kernels skips its publication at that pipeline step, so
  *                 the consumer's bounded wait runs out; -1: none (the call
  *                 is then ssd_fwd())
  *   wait_ns       limit of every bounded device-side wait in nanoseconds
  *                 (0: the default of one second)
+ *   path          -1: the path ssd_fwd() takes; 2: the path of a call that
+ *                 carries a state (the chunked order-2 kernel), although
+ *                 none is carried (the workspace must then be sized with
+ *                 ssd_workspace_bytes_ex(..., state = SSD_STATE_H));
+ *                 other values return SSD_ERR_UNSUPPORTED
  * A wait that runs out never traps: it records SSD_ERR_TIMEOUT in the
  * workspace status, every role of the kernel stops, the copies and matrix
  * products already in flight complete, the tensor memory is freed and the
@@ -392,7 +397,7 @@ int ssd_debug_fwd(const void *q, const void *k, const void *v,
                   int B, int H, int N, int d_h, int dtype,
                   int order, int normalize, int chunk,
                   void *out, void *workspace, size_t workspace_bytes,
-                  void *stream, int skip_publish, long long wait_ns);
+                  void *stream, int skip_publish, long long wait_ns, int path);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *ssd_status_str(int status);
@@ -401,8 +406,12 @@ const char *ssd_status_str(int status);
  * Which kernel sequence ssd_fwd() runs for these arguments: 0 = the general
  * SIMT path (any supported shape, fp32 or bf16), 1 = the order-1 tcgen05
  * path (chunk states, state passing, chunk outputs: three launches),
- * 2 = the order-2 tcgen05 path (one launch); -1 when the arguments are
- * invalid.
+ * 2 = the chunked order-2 tcgen05 path (one launch: the D^2 x D state of a
+ * head spread over a cluster of CTAs; calls that carry a state in or out
+ * take it), 3 = the order-2 tcgen05 path in the masked quadratic form
+ * (Algorithm 5; two launches: the decay factors, then a flash-style loop
+ * over key tiles; bf16, d_h in {32, 64}, N a multiple of 128, no carried
+ * state); -1 when the arguments are invalid.
  * *n_launches (may be NULL) receives the number of kernels one call launches.
  */
 int ssd_fwd_path(int B, int H, int N, int d_h, int dtype, int order, int chunk,

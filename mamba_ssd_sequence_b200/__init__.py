@@ -21,7 +21,7 @@ SSD_BF16 = 1
 SSD_VALUE_DT = 1  # ssd_fwd_ex flag: contract with v * dt (Algorithm 4, V_dt)
 SSD_STATE_H = 1   # state-mask bits for ssd_workspace_bytes_ex
 SSD_STATE_Z = 2
-PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2"}
+PATH_NAMES = {0: "simt", 1: "tc_order1", 2: "tc_order2", 3: "tc_order2_quad"}
 
 _lib = None
 
@@ -82,7 +82,7 @@ def load_library():
     lib.ssd_status_str.restype = ctypes.c_char_p
     lib.ssd_fwd_path.argtypes = [ci] * 7 + [ctypes.POINTER(ci)]
     lib.ssd_fwd_path.restype = ci
-    lib.ssd_debug_fwd.argtypes = [vp] * 7 + [ci] * 8 + [vp, vp, sz, vp, ci, ctypes.c_longlong]
+    lib.ssd_debug_fwd.argtypes = [vp] * 7 + [ci] * 8 + [vp, vp, sz, vp, ci, ctypes.c_longlong, ci]
     lib.ssd_debug_fwd.restype = ci
     _lib = lib
     return lib
@@ -189,11 +189,12 @@ def ssd_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk
 
 
 def ssd_debug_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool, chunk: int,
-                  skip_publish: int, wait_ns: int, out=None, workspace=None, stream=None):
+                  skip_publish: int, wait_ns: int, out=None, workspace=None, stream=None, path: int = -1):
     """Failure-detection test hook (include/ssd.h: ssd_debug_fwd): ssd_fwd in
     which one producer skips its publication at pipeline step `skip_publish`
     (-1: none) and every bounded device-side wait gives up after `wait_ns`
-    nanoseconds.  Returns `out`; read the device status with
+    nanoseconds; `path` 2 runs the chunked order-2 kernel that calls with a
+    carried state take.  Returns `out`; read the device status with
     ssd_status_from_workspace(workspace)."""
     import torch
     B, H, N, d = q.shape
@@ -201,12 +202,13 @@ def ssd_debug_fwd(q, k, v, dt_p, A_log, dt_bias, D, order: int, normalize: bool,
     if out is None:
         out = torch.empty_like(q)
     if workspace is None:
-        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device)
+        workspace = alloc_workspace(B, H, N, d, dt, order, chunk, q.device,
+                                    state=SSD_STATE_H if path == 2 else 0)
     rc = load_library().ssd_debug_fwd(
         _ptr(q), _ptr(k), _ptr(v), _ptr(dt_p), _ptr(A_log), _ptr(dt_bias), _ptr(D),
         B, H, N, d, dt, int(order), int(bool(normalize)), int(chunk),
         _ptr(out), _ptr(workspace), workspace.numel(), _stream_handle(stream),
-        int(skip_publish), int(wait_ns))
+        int(skip_publish), int(wait_ns), int(path))
     _check(rc, "ssd_debug_fwd")
     return out
 

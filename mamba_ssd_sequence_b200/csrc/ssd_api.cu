@@ -76,6 +76,11 @@ int make_plan(int B, int H, int N, int d, int dtype, int order, int normalize, i
         p.path = PATH_TC_ORDER1;
         p.n_launches = 3;
         tc_order1_layout(B, H, N, chunk, &p);
+    } else if (order == 2 && state == 0 && tc_order2q_supports(B, H, N, d, dtype)) {
+        // without a carried state the masked quadratic form needs no D^2 x D state
+        p.path = PATH_TC_ORDER2Q;
+        p.n_launches = 2;
+        tc_order2q_layout(B, H, N, &p);
     } else if (order == 2 && tc_order2_supports(B, H, N, d, dtype, chunk)) {
         p.path = PATH_TC_ORDER2;
         p.n_launches = 1;
@@ -130,7 +135,7 @@ int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, c
                int d_h, int dtype, int order, int normalize, int chunk, int flags, const float *h0,
                const float *z0, float *h_out, float *z_out, void *out, void *workspace,
                size_t workspace_bytes, void *stream, int dbg_skip, unsigned long long wait_ns,
-               const ConvParams *conv = nullptr) {
+               const ConvParams *conv = nullptr, int state_hint = 0) {
     if ((flags & ~SSD_VALUE_DT) != 0) return SSD_ERR_FLAGS;
     const int value_dt = (flags & SSD_VALUE_DT) ? 1 : 0;
     if (!q || !k || !v || !out) return SSD_ERR_NULL;
@@ -144,7 +149,7 @@ int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, c
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return SSD_ERR_ALIGN;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return SSD_ERR_ALIGN;
-    const int state = ((h0 || h_out) ? SSD_STATE_H : 0) | ((z0 || z_out) ? SSD_STATE_Z : 0);
+    const int state = ((h0 || h_out) ? SSD_STATE_H : 0) | ((z0 || z_out) ? SSD_STATE_Z : 0) | state_hint;
     Plan p;
     rc = make_plan(B, H, N, d_h, dtype, order, normalize, chunk, value_dt, state, &p);
     if (rc != SSD_OK) return rc;
@@ -174,6 +179,7 @@ int fwd_common(const void *q, const void *k, const void *v, const float *dt_p, c
     switch (p.path) {
     case PATH_TC_ORDER1: return launch_tc_order1(a, p);
     case PATH_TC_ORDER2: return launch_tc_order2(a, p);
+    case PATH_TC_ORDER2Q: return launch_tc_order2q(a, p);
     default: return launch_simt(a, p);
     }
 }
@@ -277,12 +283,15 @@ int ssd_debug_fwd(const void *q, const void *k, const void *v, const float *dt_p
                   const float *A_log, const float *dt_bias, const float *D, int B, int H, int N,
                   int d_h, int dtype, int order, int normalize, int chunk, void *out,
                   void *workspace, size_t workspace_bytes, void *stream, int skip_publish,
-                  long long wait_ns) {
+                  long long wait_ns, int path) {
     if (wait_ns < 0) return SSD_ERR_SHAPE;
+    if (path != -1 && path != PATH_TC_ORDER2) return SSD_ERR_UNSUPPORTED;
     if (!dt_p || !A_log || !dt_bias) return SSD_ERR_NULL;
+    // path 2: the path a call with a carried state takes (the chunked order-2
+    // kernel), selected as if a state were carried, though none is
     return fwd_common(q, k, v, dt_p, A_log, dt_bias, D, nullptr, B, H, N, d_h, dtype, order, normalize,
                       chunk, 0, nullptr, nullptr, nullptr, nullptr, out, workspace, workspace_bytes, stream,
-                      skip_publish, (unsigned long long)wait_ns);
+                      skip_publish, (unsigned long long)wait_ns, nullptr, path == PATH_TC_ORDER2 ? SSD_STATE_H : 0);
 }
 
 int ssd_fwd_ex(const void *q, const void *k, const void *v, const float *dt_p,

@@ -57,7 +57,7 @@ constexpr size_t kStatusBytes = 256;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-enum Path { PATH_SIMT = 0, PATH_TC_ORDER1 = 1, PATH_TC_ORDER2 = 2 };
+enum Path { PATH_SIMT = 0, PATH_TC_ORDER1 = 1, PATH_TC_ORDER2 = 2, PATH_TC_ORDER2Q = 3 };
 
 // Workspace plan for one call: which path runs and where its buffers sit.
 struct Plan {
@@ -86,6 +86,9 @@ int launch_simt(const FwdArgs &a, const Plan &p);
 int launch_tc_order2(const FwdArgs &a, const Plan &p);
 bool tc_order2_supports(int B, int H, int N, int d, int dtype, int chunk);
 size_t tc_order2_workspace(int B, int H, int N, int d, int chunk);
+int launch_tc_order2q(const FwdArgs &a, const Plan &p);
+bool tc_order2q_supports(int B, int H, int N, int d, int dtype);
+void tc_order2q_layout(int B, int H, int N, Plan *p);
 int launch_tc_order1(const FwdArgs &a, const Plan &p);
 bool tc_order1_fuses_conv(int chunk);
 bool tc_order1_supports(int B, int H, int N, int d, int dtype, int chunk);

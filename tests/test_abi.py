@@ -99,9 +99,13 @@ def test_path_selection(lib):
     assert path == "tc_order1" and n == 3
     path, n = ssd.ssd_fwd_path(1, 4, 1024, 64, ssd.SSD_BF16, 1, 64)
     assert path == "simt" and n == 4
+    # order 2 without a carried state: the quadratic form when N is a multiple
+    # of 128, else the chunked kernel
     path, n = ssd.ssd_fwd_path(4, 16, 4096, 32, ssd.SSD_BF16, 2, 64)
-    assert path == "tc_order2" and n == 1
+    assert path == "tc_order2_quad" and n == 2
     path, n = ssd.ssd_fwd_path(2, 8, 16384, 64, ssd.SSD_BF16, 2, 64)
+    assert path == "tc_order2_quad" and n == 2
+    path, n = ssd.ssd_fwd_path(2, 8, 16320, 64, ssd.SSD_BF16, 2, 64)
     assert path == "tc_order2" and n == 1
     path, n = ssd.ssd_fwd_path(2, 8, 1024, 16, ssd.SSD_BF16, 2, 64)
     assert path == "simt" and n == 4

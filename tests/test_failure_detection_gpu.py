@@ -32,32 +32,37 @@ SSD_ERR_TIMEOUT = 9
 CASES = [
     (1, 2, 1024, 64, 1, False, 128, 0, "tc_order1"),
     (1, 2, 2048, 64, 1, False, 256, 0, "tc_order1"),
-    (1, 2, 256, 32, 2, True, 64, 1, "tc_order2"),
+    (1, 2, 256, 32, 2, True, 64, 1, "tc_order2"),       # the chunked kernel (a slab's state)
     (1, 2, 256, 64, 2, True, 64, 5, "tc_order2"),
+    (1, 2, 256, 32, 2, True, 64, 1, "tc_order2_quad"),  # the quadratic form (a K, V stage)
+    (1, 2, 512, 64, 2, True, 64, 2, "tc_order2_quad"),
 ]
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[8]}-d{c[3]}-c{c[6]}")
 def test_skipped_publication_times_out_then_clean_call(case):
     B, H, N, d, order, normalize, chunk, skip, path = case
-    assert ssd.ssd_fwd_path(B, H, N, d, ssd.SSD_BF16, order, chunk)[0] == path
+    force = 2 if path == "tc_order2" else -1  # the chunked kernel: as a call with a carried state
+    if force < 0:
+        assert ssd.ssd_fwd_path(B, H, N, d, ssd.SSD_BF16, order, chunk)[0] == path
     x = inputs.make_inputs(B, H, N, d, "bf16", seed=5, residual=True)
     dev = to_device(x, "bf16")
-    ws = ssd.alloc_workspace(B, H, N, d, ssd.SSD_BF16, order, chunk)
+    ws = ssd.alloc_workspace(B, H, N, d, ssd.SSD_BF16, order, chunk, state=ssd.SSD_STATE_H if force == 2 else 0)
     out = torch.empty_like(dev["q"])
     args = (dev["q"], dev["k"], dev["v"], dev["dt_p"], dev["A_log"], dev["dt_bias"], dev["D"])
 
     t0 = time.monotonic()
     ssd.ssd_debug_fwd(*args, order, normalize, chunk, skip_publish=skip, wait_ns=2_000_000,
-                      out=out, workspace=ws)
+                      out=out, workspace=ws, path=force)
     torch.cuda.synchronize()  # the kernels returned: no trap, the context is usable
     elapsed = time.monotonic() - t0
     assert ssd.ssd_status_from_workspace(ws) == SSD_ERR_TIMEOUT
     assert elapsed < 5.0
 
-    # the same workspace and context serve the next call
+    # the same workspace and context serve the next call (on the same path)
     out.zero_()
-    ssd.ssd_fwd(*args, order, normalize, chunk, out=out, workspace=ws)
+    ssd.ssd_debug_fwd(*args, order, normalize, chunk, skip_publish=-1, wait_ns=0, out=out, workspace=ws,
+                      path=force)
     torch.cuda.synchronize()
     assert ssd.ssd_status_from_workspace(ws) == 0
     ref = oracle.ssd_recurrent(x["q"], x["k"], x["v"], x["dt_p"], x["A_log"], x["dt_bias"], x["D"],

@@ -31,10 +31,10 @@ if not torch.cuda.is_available():
 CASES = [
     (2, 4, 1024, 64, 1, False, 128, "bf16", "tc_order1"),
     (2, 3, 1024, 64, 1, False, 256, "bf16", "tc_order1"),
-    (2, 3, 512, 32, 2, True, 64, "bf16", "tc_order2"),
-    (2, 3, 512, 32, 2, False, 64, "bf16", "tc_order2"),
-    (2, 3, 512, 64, 2, True, 64, "bf16", "tc_order2"),
-    (2, 3, 512, 64, 2, False, 64, "bf16", "tc_order2"),
+    (2, 3, 512, 32, 2, True, 64, "bf16", "tc_order2_quad"),
+    (2, 3, 512, 32, 2, False, 64, "bf16", "tc_order2_quad"),
+    (2, 3, 512, 64, 2, True, 64, "bf16", "tc_order2_quad"),
+    (2, 3, 512, 64, 2, False, 64, "bf16", "tc_order2_quad"),
     (2, 3, 256, 16, 1, False, 64, "f32", "simt"),
     (2, 3, 256, 16, 2, True, 64, "f32", "simt"),
 ]

@@ -82,7 +82,8 @@ def test_full_size_options_and_state_sampled(case):
         else:
             z0 = None
     path, _ = ssd.ssd_fwd_path(w.B, w.H, w.N, w.d, ssd.SSD_BF16, w.order, w.chunk)
-    assert path == ("tc_order1" if w.order == 1 else "tc_order2"), "the workload runs on its tensor-core path"
+    # without a carried state order 2 takes the quadratic form; with one, the chunked kernel
+    assert path == ("tc_order1" if w.order == 1 else "tc_order2_quad"), "the workload runs on its tensor-core path"
     y = ssd.ssd_fwd_state(dev["q"], dev["k"], dev["v"], dev["dt_p"], None if use_ld else dev["A_log"],
                           dev["dt_bias"], dev["D"], w.order, w.normalize, w.chunk,
                           h0=h0d, z0=z0d, h_out=ho, z_out=zo,
