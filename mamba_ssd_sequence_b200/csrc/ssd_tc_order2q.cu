@@ -29,8 +29,10 @@
 // through a ring of four stages); warp 1 MMA issue (S of step s + 1 goes
 // out before P V of step s); warps 2-9 the compute team (P, then each
 // query tile's epilogue: y = Y / n [+ D v], staged in shared memory and
-// written by one TMA store).  CTAs take the query tiles in a snake order of
-// decreasing length (longest key range first).  Every wait is bounded.
+// written by one TMA store).  CTAs take the query tiles one at a time from a
+// counter in the workspace (which kernel (a) zeroes), the latest tiles, whose
+// key ranges are the longest, first: where a head's decay skips its early
+// tiles, work per query tile differs from head to head.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,6 +49,7 @@ using namespace ptx;
 
 constexpr int kT = 128;              // tokens per tile
 constexpr int kNS = 4;               // K, V stages
+constexpr int kSB = 2;               // S buffers in TMEM
 constexpr int kCT = 256;             // compute threads
 constexpr int kQThreads = 64 + kCT;
 constexpr uint32_t kQBar = 1;        // named barrier of the compute team
@@ -68,17 +71,20 @@ struct QCfg {
     static constexpr uint32_t OFF_OUT = OFF_KV + kNS * STAGE;  // 2 x TILE: output staging per Y buffer
     static constexpr uint32_t OFF_MISC = OFF_OUT + 2 * TILE;
     static constexpr uint32_t SMEM = OFF_MISC + 2048 + 1024;
-    // TMEM: S buffers at 0 and 128 (P packed over columns [64 h, 64 h + 32) of
-    // each half h), Y buffers at 256 and 256 + D
-    static constexpr uint32_t COL_Y = 256;
+    // TMEM: S buffers at 128 b (P packed over columns [64 h, 64 h + 32) of
+    // each half h), then the two Y buffers
+    static constexpr uint32_t COL_Y = 128 * kSB;
+    static_assert(COL_Y + 2 * D <= 512, "TMEM budget");
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(STAGE % 1024 == 0 && TILE % 1024 == 0, "swizzle atoms");
 };
 
 struct QMisc {
+    uint64_t item_full[2], item_empty[2];  // the work item the TMA warp took, to the other roles
+    long long item[2];
     uint64_t q_full[2], q_empty[2];
     uint64_t st_full[kNS], st_empty[kNS];
-    uint64_t s_full[2], p_full[2], pv_done[2];
+    uint64_t s_full[kSB], p_full[kSB], pv_done[kSB];
     uint64_t y_full[2], ep_done[2];
     uint64_t drain;
     float rs[2][kT];  // the two column halves' row sums of w
@@ -125,12 +131,6 @@ struct Walk {
     }
 };
 
-// Query tile of work item k of this CTA (snake order over items sorted by
-// decreasing query tile, so every CTA gets a like mix of long and short key
-// ranges): item t -> tile I = NT - 1 - t / BH of head bh = t % BH.
-__device__ __forceinline__ long long q_item(long long k, int G, int c) {
-    return (k & 1) ? k * G + (G - 1 - c) : k * G + c;
-}
 
 // Kernel (a) of this path: per 128-token tile of a head, the tile-local
 // inclusive cumulative log2-decay a_t, the tile total lam, the key factor
@@ -139,13 +139,14 @@ __global__ void __launch_bounds__(kT)
 quad_decay_kernel(const float *__restrict__ dt_p, const float *__restrict__ A_log,
                   const float *__restrict__ dt_bias, const float *__restrict__ log_decay, int value_dt, int H,
                   int N, float *__restrict__ acs, float *__restrict__ colf, float *__restrict__ fval,
-                  float *__restrict__ lam) {
+                  float *__restrict__ lam, int *__restrict__ next_item) {
     __shared__ float wsum[kT / 32];
     __shared__ float total_s;
     const int NT = N / kT;
     const int tile = blockIdx.x, bh = tile / NT, h = bh % H;
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const size_t tok = (size_t)tile * kT + t;
+    if (tile == 0 && t == 0) *next_item = 0;  // the work counter of the kernel that follows
     float dt = 0.0f;
     if (!log_decay || value_dt) dt = softplus_f(dt_p[tok] + dt_bias[h]);
     const float a = log_decay ? log_decay[tok] * kLog2e : (-expf(A_log[h]) * kLog2e) * dt;
@@ -175,8 +176,8 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_out,
                   const __nv_bfloat16 *__restrict__ vglob, const float *__restrict__ acs,
                   const float *__restrict__ colf, const float *__restrict__ fval, const float *__restrict__ lam,
-                  const float *__restrict__ Dres, int BH, int H, int N, int normalize, DeviceStatus *status,
-                  int dbg_skip, unsigned long long wait_ns) {
+                  const float *__restrict__ Dres, int BH, int H, int N, int normalize, int *__restrict__ next_item,
+                  DeviceStatus *status, int dbg_skip, unsigned long long wait_ns) {
     using K = QCfg<D>;
     constexpr uint32_t RB = K::RB;
     extern __shared__ uint8_t smem_raw[];
@@ -186,8 +187,11 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int NT = N / kT;
+    // work items t = 0, 1, ...: query tile I = NT - 1 - t / BH of head bh = t %
+    // BH, longest key ranges first; CTAs take them one at a time from a
+    // counter (the key ranges of different heads end at different tiles)
     const long long n_items = (long long)BH * NT;
-    const int G = (int)gridDim.x, cta = (int)blockIdx.x;
+    const int cta = (int)blockIdx.x;
 
     if (tid == 0) {
         if (cta == 0 && status) {
@@ -195,13 +199,17 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             status->detail = 0;
         }
         for (int i = 0; i < 2; ++i) {
+            mbar_init(&misc->item_full[i], 1);
+            mbar_init(&misc->item_empty[i], 1 + kCT);
             mbar_init(&misc->q_full[i], 1);
             mbar_init(&misc->q_empty[i], 1);
+            mbar_init(&misc->y_full[i], 1);
+            mbar_init(&misc->ep_done[i], kCT);
+        }
+        for (int i = 0; i < kSB; ++i) {
             mbar_init(&misc->s_full[i], 1);
             mbar_init(&misc->p_full[i], kCT);
             mbar_init(&misc->pv_done[i], 1);
-            mbar_init(&misc->y_full[i], 1);
-            mbar_init(&misc->ep_done[i], kCT);
         }
         for (int i = 0; i < kNS; ++i) {
             mbar_init(&misc->st_full[i], 1);
@@ -220,8 +228,7 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = misc->tmem;
 
-    auto item_of = [&](long long k, int &I, int &bh) {
-        const long long t = q_item(k, G, cta);
+    auto item_of = [&](long long t, int &I, int &bh) {
         I = NT - 1 - (int)(t / BH);
         bh = (int)(t % BH);
     };
@@ -235,9 +242,19 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             prefetch_tmap(&tm_out);
             long long kv = 0, ti = 0;
             bool ok = true;
-            for (long long k = 0; ok && q_item(k, G, cta) < n_items; ++k, ++ti) {
+            for (;; ++ti) {
+                const int slot = (int)(ti & 1);
+                if (ti >= 2 && !mbar_wait_abortable(&misc->item_empty[slot], (uint32_t)(((ti >> 1) - 1) & 1),
+                                                    abort_flag, wait_ns)) {
+                    ok = false;
+                    break;
+                }
+                const long long t = atomicAdd(next_item, 1);
+                misc->item[slot] = t;
+                mbar_arrive(&misc->item_full[slot]);
+                if (t >= n_items) break;
                 int I, bh;
-                item_of(k, I, bh);
+                item_of(t, I, bh);
                 const int qb = (int)(ti & 1);
                 if (ti >= 2 && !mbar_wait_abortable(&misc->q_empty[qb], (uint32_t)(((ti >> 1) - 1) & 1), abort_flag,
                                                     wait_ns)) {
@@ -271,7 +288,7 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // copies still in flight after an abort land before the CTA exits (bounded)
             for (long long j = kv > kNS ? kv - kNS : 0; j < kv; ++j)
                 if (j != dbg_skip) mbar_wait_bounded(&misc->st_full[j % kNS], (uint32_t)((j / kNS) & 1));
-            if (ti >= 1) mbar_wait_bounded(&misc->q_full[(ti - 1) & 1], (uint32_t)(((ti - 1) >> 1) & 1));
+            if (ok && ti >= 1) mbar_wait_bounded(&misc->q_full[(ti - 1) & 1], (uint32_t)(((ti - 1) >> 1) & 1));
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -289,10 +306,10 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 int st, first, last;
             };
             Pend pv{-1, 0, 0, 0, 0};
-            // Y += P V of step p.s (its P in S buffer s & 1, its V in stage st)
+            // Y += P V of step p.s (its P in S buffer s % kSB, its V in stage st)
             auto issue_pv = [&](const Pend &p) {
-                const int sb = (int)(p.s & 1), yb = (int)(p.ti & 1);
-                if (!wait(&misc->p_full[sb], (uint32_t)((p.s >> 1) & 1))) return;
+                const int sb = (int)(p.s % kSB), yb = (int)(p.ti & 1);
+                if (!wait(&misc->p_full[sb], (uint32_t)((p.s / kSB) & 1))) return;
                 if (p.first && p.ti >= 2 && !wait(&misc->ep_done[yb], (uint32_t)(((p.ti >> 1) - 1) & 1))) return;
                 tc_fence_after();
                 const uint64_t dV = make_sdesc(sbase + K::OFF_KV + p.st * K::STAGE + K::TILE, 16, K::SBO, K::SW);
@@ -308,20 +325,25 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             };
             long long kv = 0, s = 0, ti = 0;
-            for (long long k = 0; ok && q_item(k, G, cta) < n_items; ++k, ++ti) {
+            for (; ok; ++ti) {
+                const int slot = (int)(ti & 1);
+                if (!wait(&misc->item_full[slot], (uint32_t)((ti >> 1) & 1))) break;
+                const long long t = misc->item[slot];
+                mbar_arrive(&misc->item_empty[slot]);
+                if (t >= n_items) break;
                 int I, bh;
-                item_of(k, I, bh);
+                item_of(t, I, bh);
                 const int qb = (int)(ti & 1);
                 if (!wait(&misc->q_full[qb], (uint32_t)((ti >> 1) & 1))) break;
                 const uint64_t dQ = make_sdesc(sbase + K::OFF_Q + qb * K::TILE, 16, K::SBO, K::SW);
                 Walk wk{lam + (size_t)bh * NT, I, I, 0.0f};
                 bool more = true;
                 while (more && ok) {
-                    const int sb = (int)(s & 1), st = (int)(kv % kNS);
+                    const int sb = (int)(s % kSB), st = (int)(kv % kNS);
                     const bool first = wk.J == I;
                     more = wk.next();
-                    // the S buffer: the P V of step s - 2 has read its P
-                    if (s >= 2 && !wait(&misc->pv_done[sb], (uint32_t)(((s >> 1) - 1) & 1))) break;
+                    // the S buffer: the P V of step s - kSB has read its P
+                    if (s >= kSB && !wait(&misc->pv_done[sb], (uint32_t)(((s / kSB) - 1) & 1))) break;
                     if (!wait(&misc->st_full[st], (uint32_t)((kv / kNS) & 1))) break;
                     tc_fence_after();
                     const uint64_t dK = make_sdesc(sbase + K::OFF_KV + st * K::STAGE, 16, K::SBO, K::SW);
@@ -352,20 +374,30 @@ tc_order2q_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int ct = tid - 64;
         bool failed = false;
         long long s = 0, ti = 0;
-        for (long long k = 0; q_item(k, G, cta) < n_items; ++k, ++ti) {
+        for (;; ++ti) {
+            const int slot = (int)(ti & 1);
+            const bool badi = !mbar_wait_abortable(&misc->item_full[slot], (uint32_t)((ti >> 1) & 1), abort_flag,
+                                                   wait_ns);
+            if (named_bar_any(kQBar, kCT, badi)) {
+                failed = true;
+                break;
+            }
+            const long long t = misc->item[slot];
+            mbar_arrive(&misc->item_empty[slot]);
+            if (t >= n_items) break;
             int I, bh;
-            item_of(k, I, bh);
+            item_of(t, I, bh);
             const size_t qtok = (size_t)bh * N + (size_t)I * kT;  // first token of the query tile
             const float ai = acs[qtok + r];
             float rsum = 0.0f;
             Walk wk{lam + (size_t)bh * NT, I, I, 0.0f};
             bool more = true;
             while (more) {
-                const int sb = (int)(s & 1), st = (int)(s % kNS);
+                const int sb = (int)(s % kSB), st = (int)(s % kNS);
                 const int J = wk.J;
                 const float Gd = wk.G;
                 more = wk.next();
-                bool bad = !mbar_wait_abortable(&misc->s_full[sb], (uint32_t)((s >> 1) & 1), abort_flag, wait_ns);
+                bool bad = !mbar_wait_abortable(&misc->s_full[sb], (uint32_t)((s / kSB) & 1), abort_flag, wait_ns);
                 // the stage's key factors are read below: observe its TMA completion
                 // too (long complete; the stage is refilled only after this P)
                 bad = bad || !mbar_wait_abortable(&misc->st_full[st], (uint32_t)((s / kNS) & 1), abort_flag, wait_ns);
@@ -512,6 +544,7 @@ int launch_q(const FwdArgs &a, const Plan &p) {
     float *colf = reinterpret_cast<float *>(ws + p.state_off);
     float *fval = a.value_dt ? reinterpret_cast<float *>(ws + p.vfac_off) : nullptr;
     float *lam = reinterpret_cast<float *>(ws + p.lam_off);
+    int *next_item = reinterpret_cast<int *>(ws + p.aux_off);
     static std::atomic<uint64_t> attr_set{0};  // one bit per device
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -525,7 +558,7 @@ int launch_q(const FwdArgs &a, const Plan &p) {
         attr_set.fetch_or(bit);
     }
     quad_decay_kernel<<<BH * NT, kT, 0, a.stream>>>(a.dt_p, a.A_log, a.dt_bias, a.log_decay, a.value_dt, a.H, a.N,
-                                                   acs, colf, fval, lam);
+                                                   acs, colf, fval, lam, next_item);
     // the CTAs split the query tiles of all heads among themselves
     const long long items = (long long)BH * NT;
     const int grid = items < sms ? (int)items : sms;
@@ -533,7 +566,7 @@ int launch_q(const FwdArgs &a, const Plan &p) {
     const unsigned long long wait_ns = a.wait_ns ? a.wait_ns : 1000000000ull;
     tc_order2q_kernel<D><<<grid, kQThreads, K::SMEM, a.stream>>>(
         tq, tk, tv, to, static_cast<const __nv_bfloat16 *>(a.v), acs, colf, fval, lam, a.D, BH, a.H, a.N,
-        a.normalize, status, a.dbg_skip, wait_ns);
+        a.normalize, next_item, status, a.dbg_skip, wait_ns);
     return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
 
@@ -544,15 +577,16 @@ bool tc_order2q_supports(int B, int H, int N, int d, int dtype) {
            (long long)B * H <= 65535;
 }
 
-// status block | acs (B H N) | key factors (B H N) | value factors (B H N) | lam (B H N / 128)
+// status block | acs (B H N) | key factors (B H N) | value factors (B H N) |
+// lam (B H N / 128) | the work counter
 void tc_order2q_layout(int B, int H, int N, Plan *p) {
     const size_t tok = (size_t)B * H * N;
     p->acs_off = kStatusBytes;
     p->state_off = align_up(p->acs_off + tok * sizeof(float), 256);
     p->vfac_off = align_up(p->state_off + tok * sizeof(float), 256);
     p->lam_off = align_up(p->vfac_off + tok * sizeof(float), 256);
-    p->aux_off = 0;
-    p->total = align_up(p->lam_off + tok / kT * sizeof(float), 256);
+    p->aux_off = align_up(p->lam_off + tok / kT * sizeof(float), 256);
+    p->total = p->aux_off + 256;
 }
 
 int launch_tc_order2q(const FwdArgs &a, const Plan &p) {
