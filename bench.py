@@ -76,9 +76,10 @@ DRAM_TRAFFIC = {
     "order1-bf16-B4H16N2048d64-c128": 101_977_344,
     # chunk states 607.3 MB + state pass 87.1 MB + chunk outputs 1127.6 MB
     "order1-bf16-B1H32N65536d64-c256": 1_821_930_752,
-    # the order-2 workloads: no capture yet of the quadratic-form kernels
-    "order2-bf16-B4H16N4096d32-c64": None,
-    "order2-bf16-B2H8N16384d64-c64": None,
+    # quadratic form: decay factors 1.05 MB + the loop over key tiles 53.2 MB
+    "order2-bf16-B4H16N4096d32-c64": 54_286_336,
+    # quadratic form: decay factors 1.05 MB + the loop over key tiles 117.5 MB
+    "order2-bf16-B2H8N16384d64-c64": 118_563_328,
 }
 
 
@@ -97,6 +98,32 @@ def algorithmic_work(w: inputs.Workload):
     per_tok_flops = 2 * (C + 1) * d + 4 * dphi * d + ((4 * dphi + C + 1) if w.normalize else 0)
     T = w.token_heads
     return T * per_tok_bytes, T * per_tok_flops, per_tok_bytes, per_tok_flops
+
+
+def quad_tile_pairs(w: inputs.Workload, x) -> int:
+    """(query tile, key tile) pairs of 128 tokens that the order-2 quadratic
+    form multiplies on these inputs: per query tile I its own tile, tile
+    I - 1, and earlier tiles while the decay over the tiles between stays at
+    or above 2^-200 (the kernel's rule, evaluated here in float64 from the
+    same inputs, so a pair at the boundary may count differently)."""
+    T = 128
+    NT = w.N // T
+    dt_p = x["dt_p"].reshape(w.B, w.H, w.N).astype(np.float64)
+    dt = np.logaddexp(0.0, dt_p + x["dt_bias"].astype(np.float64)[None, :, None])
+    a = -np.exp(x["A_log"].astype(np.float64))[None, :, None] * dt / np.log(2.0)
+    lam = a.reshape(w.B, w.H, NT, T).sum(-1)
+    pairs = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            negc = -np.concatenate([[0.0], np.cumsum(lam[b, h])])  # -sum of lam over tiles < k, increasing
+            for I in range(NT):
+                n = 1 + (1 if I >= 1 else 0)
+                if I >= 2:  # tiles J <= I - 2: decay over tiles J + 1 .. I - 1 = negc[J + 1] - negc[I] <= 200
+                    m0 = int(np.searchsorted(negc, negc[I] - 200.0, side="left"))
+                    lo = max(m0, 1)
+                    n += max(0, (I - 1) - lo + 1)
+                pairs += n
+    return pairs
 
 
 def roofline_of(w: inputs.Workload, mean_ms: float, peaks, peak_src: str):
@@ -345,7 +372,7 @@ def main():
             if name == w.name:
                 continue
             ow = inputs.WORKLOADS[name]
-            _, oh = make_device_inputs(ow, seed=rank, torch=torch)
+            ox, oh = make_device_inputs(ow, seed=rank, torch=torch)
             od = {k: (v.to(dev_name) if v is not None else None) for k, v in oh.items()}
             del oh
             oout = torch.empty_like(od["q"])
@@ -372,7 +399,11 @@ def main():
             others[name] = {"ms": oms, "steps": osteps, "path": opath, "launches_per_step": olaunch,
                             "status": ssd.ssd_status_from_workspace(ows),
                             "value": weak_scaling_rate(ow.tokens, osteps, world, oms * osteps)}
-            del od, oout, ows
+            if opath == "tc_order2_quad":
+                # the tensor work the quadratic form actually does, next to the
+                # algorithmic FLOPs of the chunked form that the roofline counts
+                others[name]["quad_pairs"] = quad_tile_pairs(ow, ox)
+            del od, oout, ows, ox
             torch.cuda.empty_cache()
 
     # kernel (a) on its own: the chunk-local cumsum of A dt and the chunk
@@ -563,6 +594,15 @@ def main():
                         "config": {"B": ow.B, "H": ow.H, "N": ow.N, "d_h": ow.d, "chunk": ow.chunk,
                                    "order": ow.order, "normalize": ow.normalize,
                                    "residual": ow.residual}}
+            if "quad_pairs" in o:
+                # S = Q K^T and Y += P V per pair: 2 (128 x 128 x d) + 2 (128 x d x 128)
+                ex = o["quad_pairs"] * 4 * 128 * 128 * ow.d
+                extf = ex / (o["ms"] / 1e3) / 1e12
+                wl[name]["executed"] = {
+                    "what": "tensor FLOPs the quadratic form performs (tile pairs x 4 x 128^2 x d_h); the "
+                            "roofline counts the chunked form's algorithmic FLOPs",
+                    "tile_pairs": o["quad_pairs"], "tensor_flops": ex, "tflops": extf,
+                    "frac_of_peak": extf / float(peaks["bf16_tflops"])}
         line["workloads"] = wl
     if e2e is not None:
         line["e2e"] = e2e

@@ -47,3 +47,36 @@ def test_clock_summary_parses_samples(tmp_path):
 def test_clock_summary_without_nvidia_smi():
     s = bench.ClockSampler(0)
     assert s.summary()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_quad_tile_pairs_matches_a_walk_over_the_tiles():
+    """The bench's count of the quadratic form's (query, key) tile pairs
+    equals a direct walk over each query tile's key tiles with the kernel's
+    rule (its own tile, the tile before, then earlier tiles while the decay
+    over the tiles between is at least 2^-200)."""
+    import numpy as np
+    w = inputs.Workload("t", 2, 3, 2048, 32, 64, 2, True, False, "bf16")
+    x = inputs.make_inputs(w.B, w.H, w.N, w.d, "bf16", seed=4)
+    # strong decays in some heads, so that walks stop early
+    x["A_log"] = np.log(np.array([1.0, 8.0, 16.0], np.float32))
+    x["dt_bias"] = np.array([-6.0, 0.0, 1.0], np.float32)
+    T, NT = 128, w.N // 128
+    dt = np.logaddexp(0.0, x["dt_p"].reshape(w.B, w.H, w.N).astype(np.float64) + x["dt_bias"][None, :, None])
+    a = -np.exp(x["A_log"].astype(np.float64))[None, :, None] * dt / np.log(2.0)
+    lam = a.reshape(w.B, w.H, NT, T).sum(-1)
+    want = 0
+    for b in range(w.B):
+        for h in range(w.H):
+            for I in range(NT):
+                want += 1
+                J, G = I, 0.0
+                while J > 0:
+                    J -= 1
+                    if J <= I - 2:
+                        G += lam[b, h, J + 1]
+                        if G < -200.0:
+                            break
+                    want += 1
+    got = bench.quad_tile_pairs(w, x)
+    assert got == want
+    assert got < w.B * w.H * NT * (NT + 1) // 2  # the strong decays skip tiles
