@@ -226,3 +226,27 @@ def test_fwd_conv_validation_codes(lib):
     assert fc(flags=4) == 11                                                           # SSD_ERR_FLAGS
     assert fc(xk=40) == 6 and fc(w=(64, 82, 96)) == 6 and fc(b=(None, None, 98)) == 6  # SSD_ERR_ALIGN
     assert fc(ws=None) == 7 and fc(ws_bytes=need - 1) == 7                             # SSD_ERR_WORKSPACE
+
+
+def test_debug_hook_and_order2_paths(lib):
+    """The failure hook validates its path argument and wait limit on the
+    host; the order-2 paths and workspaces follow the carried state."""
+    def dbg(**o):
+        a = dict(q=16, k=32, v=48, dt_p=64, A_log=80, dt_bias=96, D=None, B=1, H=2, N=256, d=32,
+                 dtype=ssd.SSD_BF16, order=2, normalize=1, chunk=64, out=112, ws=256, wsb=1 << 30,
+                 skip=-1, wait=0, path=-1)
+        a.update(o)
+        return lib.ssd_debug_fwd(a["q"], a["k"], a["v"], a["dt_p"], a["A_log"], a["dt_bias"], a["D"],
+                                 a["B"], a["H"], a["N"], a["d"], a["dtype"], a["order"], a["normalize"],
+                                 a["chunk"], a["out"], a["ws"], a["wsb"], None, a["skip"], a["wait"], a["path"])
+    assert dbg(path=3) == 10 and dbg(path=0) == 10   # only -1 and the chunked order-2 path
+    assert dbg(wait=-1) == 2                         # a negative wait limit
+    assert dbg(path=2, dt_p=None) == 1
+    # without a carried state order 2 takes the quadratic form, whose scratch
+    # (per-token decay factors) differs from the chunked kernel's (partials)
+    quad = ssd.ssd_workspace_bytes_ex(2, 8, 16384, 64, ssd.SSD_BF16, 2, 64, 0, 0)
+    chunked = ssd.ssd_workspace_bytes_ex(2, 8, 16384, 64, ssd.SSD_BF16, 2, 64, 0, ssd.SSD_STATE_H)
+    assert quad >= 256 + 3 * 2 * 8 * 16384 * 4 and chunked > 0 and quad != chunked
+    assert ssd.ssd_fwd_path(1, 2, 256, 32, ssd.SSD_BF16, 2, 64)[0] == "tc_order2_quad"
+    assert ssd.ssd_fwd_path(1, 2, 192, 32, ssd.SSD_BF16, 2, 64)[0] == "tc_order2"   # N % 128 != 0
+    assert ssd.ssd_fwd_path(1, 2, 256, 16, ssd.SSD_BF16, 2, 64)[0] == "simt"        # d_h 16
