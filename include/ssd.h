@@ -106,7 +106,10 @@ size_t ssd_workspace_bytes_ex(int B, int H, int N, int d_h, int dtype, int order
  *   dt_bias    device, [H] fp32
  *   D          device, [H*d_h] fp32, or NULL for no residual
  *   normalize  nonzero: divide each row by its row sum (Algorithm 1, y / N)
- *   chunk      chunk length in tokens (64, 128 or 256), N % chunk == 0
+ *   chunk      chunk length in tokens (64, 128 or 256), N % chunk == 0; the
+ *              order-2 path in the masked quadratic form (ssd_fwd_path() = 3)
+ *              does not chunk the sequence, and its result does not depend
+ *              on it
  *   out        device, [B, H, N, d_h], element type `dtype`; must not alias
  *              an input
  *   workspace  device, at least ssd_workspace_bytes(...) bytes, 256-byte
