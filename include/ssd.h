@@ -166,14 +166,15 @@ int ssd_fwd_ex(const void *q, const void *k, const void *v,
  * the library while the previous slice's forward pass and output copy run on
  * `stream`, so the two directions of the host link overlap.  The copy
  * stream and its events are created on the first such call in a CUDA context
- * (per context, kept until exit) and wait for the work enqueued on `stream`
+ * (per context, kept until exit; where they cannot be created the call runs
+ * as one slice on `stream`) and wait for the work enqueued on `stream`
  * before the call; every later step of the call is enqueued on `stream`, so
  * synchronising `stream` before reading out_host suffices, as for one slice.
  * Concurrent calls from several host threads in one context are serialised
  * while they enqueue.  The status word of the workspace
  * (ssd_status_from_workspace) reports the first slice that failed.
  * Errors: as ssd_fwd(), checked on the whole problem before anything is
- * enqueued; SSD_ERR_CUDA when a copy, the copy stream or an event fails.
+ * enqueued; SSD_ERR_CUDA when a copy or an event record or wait fails.
  */
 int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                  const float *dt_p_host, const float *A_log_host,

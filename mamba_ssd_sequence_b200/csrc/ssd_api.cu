@@ -225,7 +225,8 @@ HostSlices host_slices(int B, int H, size_t act_bytes) {
 
 // The copy stream and events of ssd_fwd_host, one set per CUDA context (keyed
 // by the context's ID, which the driver never reuses), created on first use
-// and kept until exit.  The mutex serialises the enqueueing of one call, so
+// and kept until exit; nullptr when they cannot be made (or after 16
+// contexts), and the call then runs as one slice.  The mutex serialises the enqueueing of one call, so
 // that two host threads never interleave their event records.
 struct HostPipe {
     unsigned long long ctx_id;
@@ -247,10 +248,21 @@ const HostPipe *host_pipe() {
     if (g_pipe_count == kPipeSlots) return nullptr;
     HostPipe p{};
     p.ctx_id = id;
-    if (cudaStreamCreateWithFlags(&p.copy, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
-    if (cudaEventCreateWithFlags(&p.entry, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-    for (cudaEvent_t &e : p.ready)
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&p.copy, cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();  // not sticky: the caller goes on with one slice
+        return nullptr;
+    }
+    cudaEvent_t *ev[1 + kMaxHostSlices];
+    ev[0] = &p.entry;
+    for (int i = 0; i < kMaxHostSlices; ++i) ev[1 + i] = &p.ready[i];
+    for (int i = 0; i < 1 + kMaxHostSlices; ++i) {
+        if (cudaEventCreateWithFlags(ev[i], cudaEventDisableTiming) != cudaSuccess) {
+            for (int j = 0; j < i; ++j) cudaEventDestroy(*ev[j]);
+            cudaStreamDestroy(p.copy);
+            cudaGetLastError();
+            return nullptr;
+        }
+    }
     p.mutex = new std::mutex;
     g_pipes[g_pipe_count] = p;
     return &g_pipes[g_pipe_count++];
@@ -417,9 +429,9 @@ int ssd_fwd_host(const void *q_host, const void *k_host, const void *v_host,
     const size_t elem = dtype == SSD_F32 ? 4 : 2;
     const size_t row_act = (size_t)N * d_h * elem;  // one (b, h) row of q, k, v or out
     const size_t row_tok = (size_t)N * sizeof(float);
-    const HostSlices sl = host_slices(B, H, (size_t)B * H * row_act);
+    HostSlices sl = host_slices(B, H, (size_t)B * H * row_act);
     const HostPipe *pipe = sl.n > 1 ? host_pipe() : nullptr;
-    if (sl.n > 1 && !pipe) return SSD_ERR_CUDA;
+    if (!pipe) sl = host_slices(B, H, 0);  // no copy stream (or none needed): one slice
     // one stream (the caller's) when there is a single slice; otherwise the
     // inputs go in on the library's copy stream, after the caller's earlier work
     cudaStream_t cs = pipe ? pipe->copy : s;
